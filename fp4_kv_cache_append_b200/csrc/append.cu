@@ -1,0 +1,224 @@
+// Append kernel: pool m tokens into a compressed entry, quantise it to FP4
+// (E2M1 + one E4M3 scale per 16 channels), project and FP8-quantise its
+// indexer key, and write FP8 window rows.
+//   DeepSeek-V4.1-Flash (jaehun.me review), section "2) CSA2": m tokens -> one
+//   entry with no overlap and no absolute-position term; the indexer key is
+//   projected from the main KV.  Section "3) FP4 main KV + SWA Bounded
+//   Replay": FP4 main KV, FP8 window KV.
+// One block per group of up to 8 new entries (blockDim = D/2, thread t owns
+// channels 2t, 2t+1 and writes code byte t) and one block per window row.  The quantised bytes are
+// decided in binary32 with IEEE division, no contraction (explicit _rn
+// intrinsics), so they are reproducible bit for bit.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa2 {
+
+// e^x for x in [-80, 0], binary32: Cody-Waite reduction x = n ln2 + r with
+// ln2 split into a 17-bit head (exact n*head for |n| < 128) and the rounded
+// tail, then the degree-7 Taylor polynomial of e^r by Horner's rule with
+// fused multiply-adds, scaled by 2^n built from its exponent field.  Below
+// -80 the result is 0.  The gate weights of an m = 2 entry depend on this
+// exact operation sequence.
+__device__ __forceinline__ float gate_exp(float x) {
+  if (!(x >= -80.0f)) return 0.0f;
+  if (x > 0.0f) x = 0.0f;
+  const float n = rintf(__fmul_rn(x, 0x1.715476p+0f));
+  float r = __fmaf_rn(-n, 0x1.62e4p-1f, x);
+  r = __fmaf_rn(-n, 0x1.7f7d1cp-20f, r);
+  float p = 0x1.a01a02p-13f;
+  p = __fmaf_rn(p, r, 0x1.6c16c2p-10f);
+  p = __fmaf_rn(p, r, 0x1.111112p-7f);
+  p = __fmaf_rn(p, r, 0x1.555556p-5f);
+  p = __fmaf_rn(p, r, 0x1.555556p-3f);
+  p = __fmaf_rn(p, r, 0.5f);
+  p = __fmaf_rn(p, r, 1.0f);
+  p = __fmaf_rn(p, r, 1.0f);
+  return __fmul_rn(p, __uint_as_float((uint32_t)((int)n + 127) << 23));
+}
+
+// Softmax-gated pair (per channel): the larger logit gets 1/(1+e), the other
+// e/(1+e), e = exp(-|z_a - z_b|); pooled = fl(w_a kv_a) + fl(w_b kv_b).
+__device__ __forceinline__ float pool_pair(float ka, float kb, float za, float zb) {
+  const float e = gate_exp(-fabsf(__fsub_rn(za, zb)));
+  const float s = __fadd_rn(1.0f, e);
+  const float w_big = __fdiv_rn(1.0f, s), w_small = __fdiv_rn(e, s);
+  const float wa = (za >= zb) ? w_big : w_small;
+  const float wb = (za >= zb) ? w_small : w_big;
+  return __fadd_rn(__fmul_rn(wa, ka), __fmul_rn(wb, kb));
+}
+
+__device__ __forceinline__ float block_max(float v, float *red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  v = lane < nw ? red[lane] : 0.0f;
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Entries j0 .. j0+count-1 (count <= kEntriesPerBlock) of sequence b.  The
+// projection reads each W_ik element once for all of the block's entries.
+__device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
+  const int t = threadIdx.x;
+  const int D = a.D, dI = a.dI, m = a.m, G = D / 32;
+  const int p0 = a.pos0[b];
+  if (p0 < 0) {
+    if (t == 0 && j0 == 0) flag(a.status, CSA2_DEV_BAD_POSITION);
+    return;
+  }
+  if (j0 == 0 && t == 0) a.n_entries[b] = (p0 + a.T) / m;
+  const int n_new = (p0 + a.T) / m - p0 / m;
+  int count = n_new - j0;
+  if (count > a.entries_per_block) count = a.entries_per_block;
+
+  float *xh = sm;                                   // [E][D]
+  float *part = xh + a.entries_per_block * D;       // [E][G][dI]
+  float *red = part + a.entries_per_block * G * dI; // [32]
+
+  // ---- pool + FP4 per entry (thread t: channels 2t, 2t+1; 8 threads per group)
+  for (int jj = 0; jj < count; ++jj) {
+    const int e = p0 / m + j0 + jj;
+    float x0, x1;
+    if (m == 1) {
+      const uint32_t v = reinterpret_cast<const uint32_t *>(a.kv + ((size_t)b * a.T + (e - p0)) * D)[t];
+      x0 = bf16_to_f32((uint16_t)(v & 0xFFFFu));
+      x1 = bf16_to_f32((uint16_t)(v >> 16));
+    } else {
+      const int ta = 2 * e - p0;  // -1 only for the block's first entry with p0 odd: the pending token
+      const uint16_t *kva = ta < 0 ? a.pending_kv + (size_t)b * D : a.kv + ((size_t)b * a.T + ta) * D;
+      const uint16_t *za = ta < 0 ? a.pending_gate + (size_t)b * D : a.gate + ((size_t)b * a.T + ta) * D;
+      const uint16_t *kvb = a.kv + ((size_t)b * a.T + ta + 1) * D;
+      const uint16_t *zb = a.gate + ((size_t)b * a.T + ta + 1) * D;
+      const uint32_t ka = reinterpret_cast<const uint32_t *>(kva)[t];
+      const uint32_t kb = reinterpret_cast<const uint32_t *>(kvb)[t];
+      const uint32_t ga = reinterpret_cast<const uint32_t *>(za)[t];
+      const uint32_t gb = reinterpret_cast<const uint32_t *>(zb)[t];
+      x0 = pool_pair(bf16_to_f32(ka & 0xFFFFu), bf16_to_f32(kb & 0xFFFFu), bf16_to_f32(ga & 0xFFFFu),
+                     bf16_to_f32(gb & 0xFFFFu));
+      x1 = pool_pair(bf16_to_f32(ka >> 16), bf16_to_f32(kb >> 16), bf16_to_f32(ga >> 16), bf16_to_f32(gb >> 16));
+    }
+    float amax = fmaxf(fabsf(x0), fabsf(x1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    uint32_t sb = amax == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+    const float s = e4m3_to_f32(sb);
+    uint32_t c0 = 0, c1 = 0;
+    if (s != 0.0f) {
+      c0 = f32_to_e2m1(__fdiv_rn(x0, s));
+      c1 = f32_to_e2m1(__fdiv_rn(x1, s));
+    } else {
+      sb = 0;
+    }
+    if (e < a.cap) {
+      const size_t row = (size_t)b * a.cap + e;
+      a.codes[row * (D / 2) + t] = (uint8_t)(c0 | (c1 << 4));
+      if ((t & 7) == 0) a.scales[row * (D / 16) + (t >> 3)] = (uint8_t)sb;
+    } else if (t == 0) {
+      flag(a.status, CSA2_DEV_APPEND_RANGE);
+    }
+    xh[jj * D + 2 * t] = __fmul_rn(e2m1_to_f32(c0), s);
+    xh[jj * D + 2 * t + 1] = __fmul_rn(e2m1_to_f32(c1), s);
+  }
+  // m = 2: the chunk's last token opens a pair -> it waits in the pending
+  // buffer.  Block j0 == 0 is the only one that reads or writes it; it reads
+  // first (above) and writes after the barrier.
+  __syncthreads();
+  if (m == 2 && j0 == 0 && ((p0 + a.T) & 1)) {
+    const size_t src = ((size_t)b * a.T + (a.T - 1)) * D;
+    reinterpret_cast<uint32_t *>(a.pending_kv + (size_t)b * D)[t] = reinterpret_cast<const uint32_t *>(a.kv + src)[t];
+    reinterpret_cast<uint32_t *>(a.pending_gate + (size_t)b * D)[t] = reinterpret_cast<const uint32_t *>(a.gate + src)[t];
+  }
+  if (count <= 0) return;
+
+  // ---- indexer key: k_i = sum_c x^_c W[c][i] in a fixed order (32-channel
+  // groups by fmaf in ascending channel order from +0, then pairwise sums)
+  constexpr int E = 8;
+  for (int p = t; p < G * dI; p += blockDim.x) {
+    const int i = p % dI, g = p / dI;
+    const uint16_t *wcol = a.w_ik + (size_t)(32 * g) * dI + i;
+    float acc[E];
+#pragma unroll
+    for (int jj = 0; jj < E; ++jj) acc[jj] = 0.0f;
+#pragma unroll 4
+    for (int c = 0; c < 32; ++c) {
+      const float wv = bf16_to_f32(wcol[(size_t)c * dI]);
+#pragma unroll
+      for (int jj = 0; jj < E; ++jj)
+        if (jj < count) acc[jj] = __fmaf_rn(xh[jj * D + 32 * g + c], wv, acc[jj]);
+    }
+#pragma unroll
+    for (int jj = 0; jj < E; ++jj)
+      if (jj < count) part[(jj * G + g) * dI + i] = acc[jj];
+  }
+  __syncthreads();
+  for (int jj = 0; jj < count; ++jj) {
+    const int e = p0 / m + j0 + jj;
+    float k = 0.0f;
+    if (t < dI) {
+      int n = G;
+      float v[16];
+#pragma unroll
+      for (int g = 0; g < 16; ++g) v[g] = g < G ? part[(jj * G + g) * dI + t] : 0.0f;
+      while (n > 1) {
+        const int h = n >> 1;
+        for (int q = 0; q < h; ++q) v[q] = __fadd_rn(v[2 * q], v[2 * q + 1]);
+        if (n & 1) { v[h] = v[n - 1]; n = h + 1; } else n = h;
+      }
+      k = v[0];
+    }
+    const float kmax = block_max(t < dI ? fabsf(k) : 0.0f, red);
+    const float sk = __fdiv_rn(kmax, 448.0f);
+    if (e < a.cap) {
+      const size_t row = (size_t)b * a.cap + e;
+      if (t < dI) a.ik[row * dI + t] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(k, sk)));
+      if (t == 0) a.ik_scale[row] = sk;
+    }
+  }
+}
+
+__device__ void append_window_row(const AppendArgs &a, int b, int r) {
+  const int t = threadIdx.x;
+  const int p0 = a.pos0[b];
+  const int cnt = a.T < a.W_cap ? a.T : a.W_cap;
+  const int tau = a.T - cnt + r;
+  const int p = p0 + tau;
+  if (p < 0) {
+    if (t == 0) flag(a.status, CSA2_DEV_BAD_POSITION);
+    return;
+  }
+  const uint32_t v = reinterpret_cast<const uint32_t *>(a.kv_swa + ((size_t)b * a.T + tau) * a.D)[t];
+  const uint32_t lo = f32_to_e4m3(__fdiv_rn(bf16_to_f32((uint16_t)(v & 0xFFFFu)), a.s_swa));
+  const uint32_t hi = f32_to_e4m3(__fdiv_rn(bf16_to_f32((uint16_t)(v >> 16)), a.s_swa));
+  uint8_t *dst = a.swa_rows + ((size_t)b * a.W_cap + (p % a.W_cap)) * a.D;
+  reinterpret_cast<uint16_t *>(dst)[t] = (uint16_t)(lo | (hi << 8));
+}
+
+__global__ void append_kernel(const AppendArgs a) {
+  extern __shared__ float sm[];
+  const int nm = a.B * a.main_blocks_per_seq;
+  if ((int)blockIdx.x < nm) {
+    append_entries(a, blockIdx.x / a.main_blocks_per_seq,
+                   (blockIdx.x % a.main_blocks_per_seq) * a.entries_per_block, sm);
+  } else {
+    const int i = blockIdx.x - nm;
+    append_window_row(a, i / a.swa_blocks_per_seq, i % a.swa_blocks_per_seq);
+  }
+}
+
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
+  const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq);
+  if (blocks == 0) return cudaSuccess;
+  const int threads = a.D / 2;
+  const size_t smem =
+      a.codes ? sizeof(float) * ((size_t)a.entries_per_block * (a.D + (a.D / 32) * a.dI) + 32) : 0;
+  cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  append_kernel<<<blocks, threads, smem, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csa2

@@ -1,0 +1,99 @@
+// Host-side launchers of the libcsa2 kernels (internal; the public ABI is
+// include/csa2.h).  Each returns the cudaError_t of its launch.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/csa2.h"
+
+namespace csa2 {
+
+struct AppendArgs {
+  // main cache (codes == nullptr: no main part)
+  uint8_t *codes, *scales, *ik;
+  float *ik_scale;
+  int32_t *n_entries;
+  uint16_t *pending_kv, *pending_gate;
+  int B, cap, D, dI, m;
+  const uint16_t *kv, *gate, *w_ik;
+  // window cache (rows == nullptr: no window part)
+  uint8_t *swa_rows;
+  float s_swa;
+  int W_cap;
+  const uint16_t *kv_swa;
+  const int32_t *pos0;
+  int T;
+  int main_blocks_per_seq, swa_blocks_per_seq;
+  int entries_per_block;   // 1 .. 8
+  unsigned int *status;
+};
+cudaError_t launch_append(const AppendArgs &a, cudaStream_t s);
+
+struct IndexArgs {
+  const float *ik_scale;
+  const int32_t *n_entries;
+  int B, cap, m, dI;
+  const uint16_t *q_idx;  // [B][T_q][H_I][dI]
+  const float *w;         // [B][T_q][H_I]
+  const int32_t *q_pos;   // [B][T_q]
+  int T_q, H_I;
+  float *scores;          // [B*T_q][ld]
+  int64_t ld;
+  int32_t *n_valid;       // full mode, optional
+  const int32_t *pool;    // reindex mode: [B*T_q][P]
+  int P;
+  int tiles_per_row, tiles_per_cta;
+  unsigned int *status;
+};
+cudaError_t launch_index(const CUtensorMap &ik_map, const IndexArgs &a, bool reindex, int sms,
+                         cudaStream_t s);
+
+struct TopkArgs {
+  const float *scores;
+  int rows;
+  int64_t ld;
+  int n_cols;
+  const int32_t *n_valid;
+  const int32_t *pool_blocks;
+  int K;
+  int32_t *out_idx;
+  int P_out;
+  int32_t *out_pool;
+  void *ws;
+};
+struct TopkPlan {
+  int chunk;      // columns per first-stage block
+  int nchunks;
+  int k1;         // candidates kept per chunk
+  int p1;         // pool candidates kept per chunk
+  size_t bytes;   // workspace bytes
+};
+TopkPlan plan_topk(int rows, int n_cols, int K, int P_out);
+cudaError_t launch_topk(const TopkArgs &a, const TopkPlan &p, cudaStream_t s);
+
+struct AttnArgs {
+  const uint8_t *codes, *scales;
+  int cap, D;
+  const uint8_t *swa_rows;
+  float s_swa;
+  int W_cap, window;
+  const uint16_t *q;      // [B][T_q][H][D]
+  const int32_t *q_pos;   // [B][T_q]
+  int B, T_q, H;
+  const int32_t *idx;     // [B][T_q][K]
+  int K;
+  float scale;
+  uint16_t *out;          // [B][T_q][H][D]
+  float *ws;              // split partials (nullptr when unsplit)
+  int nsplit, chunks_per_split;
+  unsigned int *status;
+};
+struct AttnPlan {
+  int nsplit, chunks_per_split;
+  size_t bytes;
+};
+AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms);
+cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s);
+
+}  // namespace csa2

@@ -1,0 +1,71 @@
+"""The C-ABI library loads on a machine without a GPU, exports every symbol
+include/csa2.h declares, and rejects bad arguments on the host before any
+CUDA work (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_kv_cache_append_b200 import csa2 as C
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared():
+    src = open(os.path.join(ROOT, "include", "csa2.h")).read()
+    return re.findall(r"CSA2_API\s+[\w\s\*]+?\b(csa2_\w+)\s*\(", src)
+
+
+def test_header_declares_the_five_entry_points():
+    names = declared()
+    for n in ("csa2_append_quant", "csa2_index_full", "csa2_index_reindex", "csa2_topk", "csa2_sparse_attn_decode"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = C.lib()
+    for n in declared():
+        assert hasattr(lib, n), n
+    assert set(declared()) == set(C.SIGNATURES), "binding and header disagree"
+
+
+def test_version():
+    assert C.csa2_version() >> 16 == 1
+
+
+def _err(st):
+    return st != 0 and C.lib().csa2_last_error().decode() != ""
+
+
+def test_host_validation_rejects_bad_arguments_without_a_gpu():
+    L = C.lib()
+    d = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 1, 128, 512, 128, 1)
+    p = ctypes.c_void_p(16)
+    # no main and no window cache
+    assert L.csa2_append_quant(None, p, None, p, None, p, p, 1, None) == 1
+    # misaligned pointer
+    assert L.csa2_index_full(ctypes.byref(d), ctypes.c_void_p(18), p, p, 1, 64, p, 128, None, None) == 1
+    # unsupported D
+    bad = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 1, 128, 384, 128, 1)
+    assert L.csa2_index_full(ctypes.byref(bad), p, p, p, 1, 64, p, 128, None, None) == 2
+    # cap not a multiple of 128
+    bad = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 1, 100, 512, 128, 1)
+    assert L.csa2_index_full(ctypes.byref(bad), p, p, p, 1, 64, p, 128, None, None) == 2
+    # H_I out of range
+    assert L.csa2_index_full(ctypes.byref(d), p, p, p, 1, 65, p, 128, None, None) == 2
+    # ld < cap
+    assert L.csa2_index_full(ctypes.byref(d), p, p, p, 1, 64, p, 64, None, None) in (1, 3)
+    # K out of range, P not a multiple of 16, workspace too small
+    assert L.csa2_topk(p, 1, 128, 128, None, None, 0, p, 0, None, p, 1 << 20, None) == 2
+    assert L.csa2_index_reindex(ctypes.byref(d), p, p, p, 1, 64, p, 20, p, None) in (2, 3)
+    assert L.csa2_topk(p, 1, 128, 128, None, None, 64, p, 0, None, p, 0, None) == 5
+    assert "workspace" in L.csa2_last_error().decode()
+    # m = 2 without pending buffers
+    m2 = C.MainCacheDesc(16, 16, 16, 16, 16, None, None, 1, 128, 512, 128, 2)
+    assert L.csa2_append_quant(ctypes.byref(m2), p, p, p, None, None, p, 2, None) == 1
+
+
+def test_workspace_sizes_are_pure_host_functions():
+    assert C.csa2_topk_workspace_size(8, 65536, 512, 2048) > 0
+    assert C.csa2_topk_workspace_size(0, 65536, 512, 2048) == 0

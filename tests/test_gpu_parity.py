@@ -1,0 +1,356 @@
+"""GPU parity of every libcsa2 entry point against the oracle (same seeded
+inputs, calls through the C ABI).
+
+Bars: cache bytes (FP4 codes, E4M3 scales, window FP8 rows, indexer-key FP8
+codes and f32 scales) bit-exact; Top-K of identical fp32 scores exact; Top-K of
+the whole scoring chain equal up to the 1e-3 tie band around the K-th oracle
+score; attention max|err| <= 1e-2 max|ref| and sum|err|/sum|ref| <= 1e-3.
+Indexer scores: |gpu - oracle| <= 1e-4 |oracle| + 1e-6 max|oracle| (fp32
+accumulation of exact FP8 products over <= 64 heads: ~64 * 2^-24 relative,
+with headroom for the tensor-core accumulation order).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_kv_cache_append_b200 import csa2 as C
+from fp4_kv_cache_append_b200 import inputs as I
+
+pytestmark = pytest.mark.gpu
+
+SCORE_RTOL, SCORE_ATOL_REL = 1e-4, 1e-6
+BAND = 1e-3
+
+
+def bits(t):
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def gen(seed):
+    return torch.Generator().manual_seed(seed)
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    C.csa2_device_status(clear=True)
+    yield
+    torch.cuda.synchronize()
+
+
+def build_pair(B, cap, D, dI, m, T, pos0, seed, W_cap=128, s_swa=1.0, window=128, swa=True):
+    """Same append on GPU and oracle; returns (gpu caches, oracle caches, inputs)."""
+    g = gen(seed)
+    kv = torch.randn(B, T, D, generator=g).to(torch.bfloat16)
+    gate = torch.randn(B, T, D, generator=g).mul(2).to(torch.bfloat16) if m == 2 else None
+    W = (torch.randn(D, dI, generator=g) / math.sqrt(D)).to(torch.bfloat16)
+    kvs = torch.randn(B, T, D, generator=g).to(torch.bfloat16)
+    pos = np.asarray(pos0, np.int32)
+    gm = C.MainCache(B, cap, D, dI, m)
+    gs = C.SwaCache(B, W_cap, D, scale=s_swa, window=window) if swa else None
+    C.csa2_append_quant(gm, kv.cuda(), gate.cuda() if gate is not None else None, W.cuda(), gs,
+                        kvs.cuda() if swa else None, torch.from_numpy(pos).cuda(), T)
+    om = oracle.MainCache(B, cap, D, dI, m)
+    osw = oracle.SwaCache(B, W_cap, D, scale=s_swa, window=window) if swa else None
+    oracle.append(om, bits(kv), bits(gate) if gate is not None else None, bits(W), osw,
+                  bits(kvs) if swa else None, pos, T)
+    torch.cuda.synchronize()
+    return gm, gs, om, osw, W
+
+
+def assert_cache_equal(gm, om, gs=None, osw=None):
+    for name in ("codes", "scales", "ik", "n_entries"):
+        np.testing.assert_array_equal(getattr(gm, name).cpu().numpy(), getattr(om, name), err_msg=name)
+    np.testing.assert_array_equal(gm.ik_scale.cpu().numpy().view(np.uint32), om.ik_scale.view(np.uint32))
+    if gm.m == 2:
+        np.testing.assert_array_equal(bits(gm.pending_kv), om.pending_kv)
+        np.testing.assert_array_equal(bits(gm.pending_gate), om.pending_gate)
+    if gs is not None:
+        np.testing.assert_array_equal(gs.rows.cpu().numpy(), osw.rows)
+
+
+# ------------------------------------------------------------------ A1 / A1' / A2 append
+
+
+@pytest.mark.parametrize("D,dI", [(128, 64), (256, 128), (512, 128), (512, 64)])
+def test_append_m1_bit_exact(D, dI):
+    gm, gs, om, osw, _ = build_pair(B=3, cap=512, D=D, dI=dI, m=1, T=300, pos0=[0, 17, 200], seed=D + dI,
+                                    s_swa=0.5)
+    assert_cache_equal(gm, om, gs, osw)
+    assert C.csa2_device_status() == 0
+
+
+def test_append_decode_single_token_and_ring_wrap():
+    B, D, dI, cap = 2, 512, 128, 1024
+    gm, gs, om, osw, W = build_pair(B=B, cap=cap, D=D, dI=dI, m=1, T=700, pos0=[0, 5], seed=3)
+    g = gen(4)
+    for step in range(3):
+        kv = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+        kvs = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+        pos = np.array([700 + step, 705 + step], np.int32)
+        C.csa2_append_quant(gm, kv.cuda(), None, W.cuda(), gs, kvs.cuda(), torch.from_numpy(pos).cuda(), 1)
+        oracle.append(om, bits(kv), None, bits(W), osw, bits(kvs), pos, 1)
+    torch.cuda.synchronize()
+    assert_cache_equal(gm, om, gs, osw)
+
+
+def test_append_m2_pending_across_calls():
+    B, D, dI, cap = 2, 256, 64, 256
+    g = gen(5)
+    T_all = 77
+    kv = torch.randn(B, T_all, D, generator=g).to(torch.bfloat16)
+    gate = torch.randn(B, T_all, D, generator=g).mul(3).to(torch.bfloat16)
+    W = (torch.randn(D, dI, generator=g) / 16).to(torch.bfloat16)
+    gm = C.MainCache(B, cap, D, dI, 2)
+    om = oracle.MainCache(B, cap, D, dI, 2)
+    start = 0
+    for ln in (1, 5, 2, 1, 30, 38):
+        sl = slice(start, start + ln)
+        pos = np.array([start, start], np.int32)
+        C.csa2_append_quant(gm, kv[:, sl].contiguous().cuda(), gate[:, sl].contiguous().cuda(), W.cuda(), None,
+                            None, torch.from_numpy(pos).cuda(), ln)
+        oracle.append(om, bits(kv[:, sl]), bits(gate[:, sl]), bits(W), None, None, pos, ln)
+        start += ln
+    torch.cuda.synchronize()
+    assert start == T_all
+    assert_cache_equal(gm, om)
+
+
+def test_append_m2_bulk_prefill_chunk():
+    gm, gs, om, osw, _ = build_pair(B=1, cap=2048, D=512, dI=128, m=2, T=2000, pos0=[100], seed=6,
+                                    W_cap=2176, s_swa=2.0)
+    assert_cache_equal(gm, om, gs, osw)
+
+
+# ------------------------------------------------------------------ A3 Full scoring
+
+
+def _rows_queries(B, T_q, H_I, dI, seed):
+    g = gen(seed)
+    q = torch.randn(B, T_q, H_I, dI, generator=g).to(torch.bfloat16)
+    w = torch.rand(B, T_q, H_I, generator=g)
+    return q, w
+
+
+def _check_scores(got, ref):
+    ref = np.asarray(ref)
+    atol = SCORE_ATOL_REL * np.abs(ref).max()
+    err = np.abs(got.astype(np.float64) - ref)
+    assert np.all(err <= SCORE_RTOL * np.abs(ref) + atol), f"max err {err.max()} (max ref {np.abs(ref).max()})"
+
+
+@pytest.mark.parametrize("D,dI,H_I,n,T_q,m", [(128, 64, 4, 1000, 1, 1), (512, 128, 64, 2047, 3, 1),
+                                              (256, 128, 17, 700, 2, 1), (512, 128, 64, 900, 4, 2)])
+def test_index_full_vs_oracle(D, dI, H_I, n, T_q, m):
+    B = 2
+    cap = (n // m + 127) // 128 * 128 + 128
+    T = n
+    gm, _, om, _, _ = build_pair(B=B, cap=cap, D=D, dI=dI, m=m, T=T, pos0=[0, 0], seed=n + dI, swa=False)
+    q, w = _rows_queries(B, T_q, H_I, dI, seed=7)
+    # causal positions: the last T_q tokens, and one early query
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[1, 0] = 300
+    scores = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nval = torch.zeros(B * T_q, dtype=torch.int32, device="cuda")
+    C.csa2_index_full(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), scores, nval)
+    torch.cuda.synchronize()
+    sc = scores.cpu().numpy()
+    nv = nval.cpu().numpy()
+    for b in range(B):
+        for j in range(T_q):
+            r = b * T_q + j
+            n_vis = oracle.n_visible(int(om.n_entries[b]), int(qpos[b, j]), m)
+            assert nv[r] == n_vis
+            ref = oracle.index_scores(om, b, bits(q[b, j]), w[b, j].numpy(), n_vis)
+            _check_scores(sc[r, :n_vis], ref)
+            assert np.all(np.isnan(sc[r, n_vis:])), "columns beyond n_vis must not be written"
+    assert C.csa2_device_status() == 0
+
+
+# ------------------------------------------------------------------ A4 Top-K
+
+
+def _ref_topk_rows(s, n_valid, K):
+    return np.stack([oracle.topk(s[r, :n_valid[r]].astype(np.float64), K) for r in range(s.shape[0])])
+
+
+@pytest.mark.parametrize("rows,n,K,P,levels", [(3, 4096, 64, 2048, None), (2, 65536, 512, 2048, None),
+                                               (4, 20000, 512, 2048, 50), (2, 300, 512, 2048, None),
+                                               (1, 262144, 512, 2048, None), (2, 9000, 2048, 0, 3),
+                                               (2, 70000, 17, 64, None)])
+def test_topk_exact_on_same_scores(rows, n, K, P, levels):
+    rng = np.random.default_rng(rows * n + K)
+    s = rng.standard_normal((rows, n)).astype(np.float32)
+    if levels:
+        s = (np.round(s * levels) / levels).astype(np.float32)
+    s[:, rng.choice(n, n // 20, replace=False)] = -np.inf
+    s[0, 5] = np.nan
+    s[0, 6] = np.inf
+    n_valid = np.array([n - 7 * r for r in range(rows)], np.int32)
+    ld = n + 32
+    sd = torch.full((rows, ld), 12345.0)
+    sd[:, :n] = torch.from_numpy(s)
+    out = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    pool = torch.empty(rows, max(P, 1), dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_topk_workspace_size(rows, n, K, P))
+    C.csa2_topk(sd.cuda(), n, K, out, n_valid=torch.from_numpy(n_valid).cuda(), P_out=P,
+                out_pool=pool if P else None, ws=ws)
+    torch.cuda.synchronize()
+    ref = _ref_topk_rows(s, n_valid, K)
+    np.testing.assert_array_equal(out.cpu().numpy(), ref)
+    if P:
+        refp = np.stack([oracle.block_pool(s[r, :n_valid[r]].astype(np.float64), P) for r in range(rows)])
+        np.testing.assert_array_equal(pool.cpu().numpy(), refp)
+
+
+def test_topk_pool_mapping_for_reindex_rows():
+    rows, P, K = 3, 64, 40
+    rng = np.random.default_rng(11)
+    pool = np.sort(rng.choice(5000, size=(rows, P), replace=False), axis=1).astype(np.int32)
+    pool[2, 50:] = -1
+    s = rng.standard_normal((rows, P * 8)).astype(np.float32)
+    s[2, 400:] = -np.inf
+    out = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_topk_workspace_size(rows, P * 8, K, 0))
+    C.csa2_topk(torch.from_numpy(s).cuda(), P * 8, K, out, pool_blocks=torch.from_numpy(pool).cuda(), ws=ws)
+    torch.cuda.synchronize()
+    for r in range(rows):
+        cols = oracle.topk(s[r].astype(np.float64), K)
+        np.testing.assert_array_equal(out[r].cpu().numpy(), oracle.columns_to_entries(cols, pool[r]))
+
+
+# ------------------------------------------------------------------ A6 Reindex
+
+
+def test_index_reindex_vs_oracle():
+    B, D, dI, H_I, n = 2, 512, 128, 64, 5000
+    cap = 5120
+    gm, _, om, _, _ = build_pair(B=B, cap=cap, D=D, dI=dI, m=1, T=n, pos0=[0, 0], seed=21, swa=False)
+    rng = np.random.default_rng(22)
+    P = 256
+    pool = np.stack([np.sort(rng.choice(cap // 8, P, replace=False)) for _ in range(B)]).astype(np.int32)
+    pool[1, -10:] = -1
+    q, w = _rows_queries(B, 1, H_I, dI, seed=23)
+    qpos = np.array([[n - 1], [n - 400]], np.int32)
+    out = torch.empty(B, P * 8, device="cuda")
+    C.csa2_index_reindex(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), torch.from_numpy(pool).cuda(), out)
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    for b in range(B):
+        n_vis = oracle.n_visible(int(om.n_entries[b]), int(qpos[b, 0]), 1)
+        ref = oracle.reindex_scores(om, b, bits(q[b, 0]), w[b, 0].numpy(), n_vis, pool[b])
+        fin = np.isfinite(ref)
+        assert np.array_equal(np.isfinite(got[b]), fin)
+        _check_scores(got[b][fin], ref[fin])
+
+
+# ------------------------------------------------------------------ A5 attention
+
+
+def _check_attn(got_bf16, ref_bits):
+    ref = oracle.bf16_to_f32(ref_bits).astype(np.float64)
+    got = got_bf16.float().cpu().numpy().astype(np.float64)
+    err = np.abs(got - ref)
+    assert err.max() <= 1e-2 * np.abs(ref).max(), f"max err {err.max()} vs {np.abs(ref).max()}"
+    assert err.sum() <= 1e-3 * np.abs(ref).sum(), f"mean rel err {err.sum() / np.abs(ref).sum()}"
+
+
+@pytest.mark.parametrize("D,H,K,T_q,window,W_cap,use_ws", [(512, 64, 512, 1, 128, 128, True),
+                                                           (512, 64, 512, 1, 128, 128, False),
+                                                           (128, 8, 64, 1, 128, 128, True),
+                                                           (256, 19, 100, 3, 128, 200, True),
+                                                           (512, 64, 512, 5, 128, 256, False)])
+def test_attention_vs_oracle(D, H, K, T_q, window, W_cap, use_ws):
+    B, n = 2, 1500
+    cap = 1536
+    gm, gs, om, osw, _ = build_pair(B=B, cap=cap, D=D, dI=64, m=1, T=n, pos0=[0, 0], seed=D + H, W_cap=W_cap,
+                                    s_swa=0.75, window=window)
+    g = gen(31)
+    q = torch.randn(B, T_q, H, D, generator=g).to(torch.bfloat16)
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[0, 0] = 60   # window shorter than 128
+    idx = torch.stack([torch.stack([I.random_indices(int(qpos[b, j]) + 1, K, g, n_missing=(b + j) % 5)
+                                    for j in range(T_q)]) for b in range(B)])
+    out = torch.empty(B, T_q, H, D, dtype=torch.bfloat16, device="cuda")
+    ws = C.workspace(C.csa2_attn_workspace_size(B, T_q, H, D, K, window)) if use_ws else None
+    scale = 1 / math.sqrt(D)
+    C.csa2_sparse_attn_decode(gm, gs, q.cuda(), torch.from_numpy(qpos).cuda(), idx.cuda(), scale, out, ws=ws)
+    torch.cuda.synchronize()
+    for b in range(B):
+        for j in range(T_q):
+            ref = oracle.attention(om, osw, b, bits(q[b, j]), idx[b, j].numpy(), int(qpos[b, j]), scale)
+            _check_attn(out[b, j], ref)
+    assert C.csa2_device_status() == 0
+
+
+def test_attention_out_of_range_index_is_masked_and_flagged():
+    B, D, n, cap, K = 1, 128, 300, 384, 16
+    gm, gs, om, osw, _ = build_pair(B=B, cap=cap, D=D, dI=64, m=1, T=n, pos0=[0], seed=41)
+    g = gen(42)
+    q = torch.randn(B, 1, 8, D, generator=g).to(torch.bfloat16)
+    idx = torch.arange(K, dtype=torch.int32).view(1, 1, K) * 7
+    idx[0, 0, 3] = cap + 5          # out of the cache: masked, flagged
+    out = torch.empty(B, 1, 8, D, dtype=torch.bfloat16, device="cuda")
+    C.csa2_sparse_attn_decode(gm, gs, q.cuda(), torch.tensor([[n - 1]], dtype=torch.int32).cuda(), idx.cuda(),
+                              0.1, out)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() & C.DEV_INDEX_RANGE
+    ref = oracle.attention(om, osw, 0, bits(q[0, 0]), idx[0, 0].numpy(), n - 1, 0.1)
+    _check_attn(out[0, 0], ref)
+
+
+# ------------------------------------------------------------------ whole steps
+
+
+def _oracle_decode_chain(st, b, layer_q_idx, layer_w):
+    """Oracle cache, scores, Top-K of one sequence of a runner.Step."""
+    wl = st.wl
+    om = oracle.MainCache(1, st.cap, wl.D, wl.dI, wl.m)
+    oracle.append(om, bits(st._kv_ctx[b])[None], None, bits(st.w_ik), None, None, np.zeros(1, np.int32),
+                  wl.total_tokens)
+    t = wl.total_tokens - 1
+    n_vis = oracle.n_visible(int(om.n_entries[0]), t, wl.m)
+    sc = oracle.index_scores(om, 0, bits(layer_q_idx[b, 0]), layer_w[b, 0].cpu().numpy(), n_vis)
+    return om, sc, t
+
+
+def _band_ok(sel_gpu, sel_ref, scores, K):
+    fin = scores[np.isfinite(scores)]
+    kth = np.sort(fin)[-K] if fin.size >= K else -np.inf
+    diff = set(sel_gpu.tolist()) ^ set(sel_ref.tolist())
+    diff.discard(-1)
+    return all(abs(scores[i] - kth) <= BAND * abs(kth) for i in diff), len(diff)
+
+
+def test_tiny_step_end_to_end():
+    from fp4_kv_cache_append_b200 import runner
+    wl = I.WORKLOADS["tiny"]
+    st = runner.Step(wl, seed=0)
+    st.prefill()
+    st.run()
+    torch.cuda.synchronize()
+    b = 0
+    om, sc, t = _oracle_decode_chain(st, b, st.q_idx[0], st.w[0])
+    for name in ("codes", "scales", "ik"):
+        np.testing.assert_array_equal(getattr(st.main[0], name)[b].cpu().numpy(), getattr(om, name)[0])
+    gsc = st.scores[b, :wl.entries].cpu().numpy()
+    _check_scores(gsc, sc)
+    top = oracle.topk(sc, wl.K)
+    got = st.idx[b].cpu().numpy()
+    ok, nd = _band_ok(got, top, sc, wl.K)
+    assert ok, "Top-K differs outside the tie band"
+    planted = I.planted_positions(wl, 0, b).numpy()
+    assert set(planted.tolist()) <= set(got.tolist())
+    pool = st.pool[b].cpu().numpy()
+    assert set((got // 8).tolist()) <= set(pool.tolist())
+    osw = oracle.SwaCache(1, st.W_cap, wl.D, window=wl.window)
+    lo = I.window_lo(wl)
+    oracle.append(None, None, None, None, osw, bits(st.win_rows[0][b])[None], np.array([lo], np.int32),
+                  st.win_rows[0][b].shape[0])
+    np.testing.assert_array_equal(st.swa[0][0].rows[b].cpu().numpy(), osw.rows[0])
+    ref = oracle.attention(om, osw, 0, bits(st.q[0][b, 0]), got, t, st.scale)
+    _check_attn(st.out[0][b, 0], ref)
