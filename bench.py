@@ -150,6 +150,29 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(loaded)}
 
 
+# --------------------------------------------------------------------------- multi-rank plumbing
+
+
+def rank_seed(rank: int) -> int:
+    """Each rank decodes its own batch of sequences (weak scaling)."""
+    return rank
+
+
+def max_over_ranks(ms: float, dist, device) -> float:
+    """The job's time is the slowest rank's (device-timed) region."""
+    if dist is None:
+        return ms
+    import torch
+    tt = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
+def job_throughput(world: int, steps: int, ms: float) -> float:
+    """Steps of all ranks per second of the slowest rank."""
+    return world * steps / (ms / 1e3)
+
+
 # --------------------------------------------------------------------------- our arm
 
 
@@ -163,7 +186,7 @@ def run_ours(args, rank, world, dist):
     C.lib()   # fails loudly without the CUDA library
     dev = torch.device("cuda", torch.cuda.current_device())
     wl = I.WORKLOADS[WORKLOAD]
-    st = runner.Step(wl, seed=rank, copies=args.copies)
+    st = runner.Step(wl, seed=rank_seed(rank), copies=args.copies)
     st.prefill()
 
     # eager warm-up: initialises per-device state and every kernel
@@ -220,11 +243,7 @@ def run_ours(args, rank, world, dist):
     barrier()
     if sampler:
         sampler.__exit__()
-    ms = t0.elapsed_time(t1)
-    if dist is not None:
-        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     assert C.csa2_device_status() == 0, "device status flagged during the timed region"
 
     # per-entry-point durations: the event pairs of the last replay of the timed region
@@ -236,7 +255,7 @@ def run_ours(args, rank, world, dist):
 
     if rank != 0:
         return None
-    steps_per_s = world * K / (ms / 1e3)
+    steps_per_s = job_throughput(world, K, ms)
     B, n = wl.B, wl.entries
     alg = st.algorithmic_bytes()
     step_bytes = sum(alg.values()) + B * (wl.D + wl.D) * 2 + B * (wl.D // 2 + wl.D // 16 + wl.dI + 4)
