@@ -48,6 +48,7 @@ SIGNATURES = {
     "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P]),
     "csa2_topk": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P, _SZ, _P]),
     "csa2_topk_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "csa2_topk_noalloc": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P]),
     "csa2_sparse_attn_decode": (_I, [_PM, _PS, _P, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _P]),
     "csa2_attn_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "csa2_last_error": (ctypes.c_char_p, []),
@@ -173,6 +174,16 @@ def csa2_topk(scores, n_cols: int, K: int, out_idx, n_valid=None, pool_blocks=No
                            _ptr(n_valid, torch.int32), _ptr(pool_blocks, torch.int32), int(K),
                            _ptr(out_idx, torch.int32), int(P_out), _ptr(out_pool, torch.int32),
                            _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def csa2_topk_noalloc(scores, n_cols: int, K: int, out_idx, n_valid=None, pool_blocks=None, P_out: int = 0,
+                      out_pool=None, stream=None):
+    """csa2_topk with the library's built-in scratch (no workspace argument)."""
+    rows = out_idx.shape[0]
+    _check(lib().csa2_topk_noalloc(_ptr(scores, torch.float32), rows, scores.shape[-1], int(n_cols),
+                                   _ptr(n_valid, torch.int32), _ptr(pool_blocks, torch.int32), int(K),
+                                   _ptr(out_idx, torch.int32), int(P_out), _ptr(out_pool, torch.int32),
+                                   _stream(stream)))
 
 
 def csa2_attn_workspace_size(B: int, T_q: int, H: int, D: int, K: int, window: int) -> int:

@@ -130,6 +130,9 @@ csa2_status check_swa(const csa2_swa_cache *s) {
 }
 
 }  // namespace
+
+void set_last_error_message(const char *msg) { t_err = msg; }
+
 }  // namespace csa2
 
 using namespace csa2;

@@ -198,6 +198,29 @@ CSA2_API csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const 
                                     csa2_stream_t stream);
 CSA2_API size_t csa2_attn_workspace_size(int B, int T_q, int H, int D, int K, int window);
 
+/*
+ * 6. Top-K selection without a caller workspace.  (No counterpart in the
+ *    paper: this is a deployment variant of entry point 4.)
+ *  For callers that cannot allocate device memory when they call the
+ *  library -- e.g. a plugin inside another framework's engine whose memory
+ *  is planned and owned by that framework, or code that must not allocate
+ *  on its serving path.  Same arguments, outputs and results as csa2_topk,
+ *  without ws/ws_bytes: the scratch is a 4 MiB array in device global memory
+ *  built into the library (present on every GPU that loads it, until the
+ *  process exits).
+ *  - Selections needing more scratch than that (see
+ *    csa2_topk_workspace_size) return CSA2_ERR_WORKSPACE, nothing enqueued.
+ *  - All calls share the array: calls whose kernels may overlap on the GPU
+ *    (unordered streams) race and give undefined results; calls on one
+ *    stream are safe.  Nothing in the array needs to start at zero.
+ *  - The first call on a device looks up the array's device address; make
+ *    it before any stream capture on that device.
+ */
+CSA2_API csa2_status csa2_topk_noalloc(const float *scores, int rows, int64_t ld, int n_cols,
+                                       const int32_t *n_valid, const int32_t *pool_blocks, int K,
+                                       int32_t *out_idx, int P_out, int32_t *out_pool,
+                                       csa2_stream_t stream);
+
 /* Thread-local description of the last error of this thread ("" if none). */
 CSA2_API const char *csa2_last_error(void);
 
