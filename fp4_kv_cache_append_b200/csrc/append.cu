@@ -77,6 +77,14 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   float *xh = sm;                                   // [E][D]
   float *part = xh + a.entries_per_block * D;       // [E][G][dI]
   float *red = part + a.entries_per_block * G * dI; // [32]
+  uint16_t *ws = reinterpret_cast<uint16_t *>(red + 32);  // W_ik [D][dI] bf16, 16-byte aligned
+  // stage W_ik in shared memory with 16-byte loads (issued before the
+  // quantisation so their latency overlaps it)
+  if (count > 0) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.w_ik);
+    uint4 *dst = reinterpret_cast<uint4 *>(ws);
+    for (int i = t; i < D * dI / 8; i += blockDim.x) dst[i] = src[i];
+  }
 
   // ---- pool + FP4 per entry (thread t: channels 2t, 2t+1; 8 threads per group)
   for (int jj = 0; jj < count; ++jj) {
@@ -139,13 +147,13 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   constexpr int E = 8;
   for (int p = t; p < G * dI; p += blockDim.x) {
     const int i = p % dI, g = p / dI;
-    const uint16_t *wcol = a.w_ik + (size_t)(32 * g) * dI + i;
+    const uint16_t *wcol = ws + (32 * g) * dI + i;
     float acc[E];
 #pragma unroll
     for (int jj = 0; jj < E; ++jj) acc[jj] = 0.0f;
 #pragma unroll 4
     for (int c = 0; c < 32; ++c) {
-      const float wv = bf16_to_f32(wcol[(size_t)c * dI]);
+      const float wv = bf16_to_f32(wcol[c * dI]);
 #pragma unroll
       for (int jj = 0; jj < E; ++jj)
         if (jj < count) acc[jj] = __fmaf_rn(xh[jj * D + 32 * g + c], wv, acc[jj]);
@@ -213,8 +221,10 @@ cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
   const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq);
   if (blocks == 0) return cudaSuccess;
   const int threads = a.D / 2;
-  const size_t smem =
-      a.codes ? sizeof(float) * ((size_t)a.entries_per_block * (a.D + (a.D / 32) * a.dI) + 32) : 0;
+  // [E][D] + [E][G][dI] floats, 32 floats, then W_ik [D][dI] bf16
+  const size_t smem = a.codes ? sizeof(float) * ((size_t)a.entries_per_block * (a.D + (a.D / 32) * a.dI) + 32) +
+                                    sizeof(uint16_t) * (size_t)a.D * a.dI
+                              : 0;
   cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   append_kernel<<<blocks, threads, smem, s>>>(a);

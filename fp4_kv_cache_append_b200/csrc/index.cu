@@ -4,13 +4,23 @@
 //   DeepSeek-V4.1-Flash (jaehun.me review), section "2) CSA2": each Full layer
 //   scores the whole context with its own indexer; the Hierarchical Sparse
 //   Indexer lets later Reindex layers rescore only the <= 2,048 x 8 pool.
-// Layout of the work: entries on the M side (128-entry tiles), indexer heads
-// on N (<= 64), d_I on K.  Tiles stream from HBM by 2D TMA (boxes of 8 rows x
-// d_I bytes, hardware 128B/64B swizzle) through a STAGES-deep mbarrier ring;
-// a Reindex tile is 16 boxes at the pool's block rows, a Full tile 16 boxes
-// at consecutive rows.  The head reduction happens in the epilogue on the
-// accumulator registers, so each entry's score is produced by one quad of
-// lanes and written once.
+//
+// Work layout: entries on M (128-entry tiles), indexer heads on N (64, zero
+// padded), d_I on K.  Per block (one query row, a run of tiles), 6 warps:
+//   warp 0     TMA producer: each tile is 16 boxes of 8 rows x d_I bytes (a
+//              Full tile at consecutive rows, a Reindex tile at the pool's
+//              block rows), hardware 128B/64B swizzle, into a STAGES ring
+//   warp 1     allocates 128 TMEM columns and issues tcgen05.mma kind::f8f6f4
+//              (M=128, N=64, K=32 per instruction) into one of two TMEM
+//              accumulators; tcgen05.commit frees the smem stage and hands
+//              the accumulator to the epilogue
+//   warps 2-5  epilogue: each thread owns one TMEM lane (= one entry), reads
+//              its 64 head accumulators with tcgen05.ld and reduces
+//              s_k * sum_h (w_h s_q,h) * max(acc_h, 0) -> one fp32 score
+// The head reduction never leaves registers; scores are written once,
+// coalesced.  All waits are bounded: a wait that gives up sets the device
+// status bit and an abort flag that stops every role; in-flight copies and
+// MMAs are then drained (bounded) and TMEM is freed before the block exits.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -18,33 +28,53 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kThreads = 128;      // 4 warps x 32 entries
+constexpr int kThreads = 192;
 constexpr int kStages = 4;
 constexpr int kTileRows = 128;
-constexpr int kMaxHeads = 64;
+constexpr int kHeads = 64;          // N of the MMA (indexer heads, zero padded)
+constexpr uint32_t kTmemCols = 128; // two 64-column fp32 accumulators
 constexpr uint32_t kWaitLimit = 1u << 22;
 
 template <int DI>
 struct IndexSmem {
-  alignas(1024) uint8_t tile[kStages][kTileRows * DI];
-  uint8_t q8[kMaxHeads][DI + 16];       // padded rows: conflict-free 32-bit reads
-  float wq[kMaxHeads];                  // w_h * s_q,h
-  uint64_t full[kStages];
+  alignas(1024) uint8_t tile[kStages][kTileRows * DI];   // A operand ring (K-major, swizzled)
+  alignas(1024) uint8_t q8[kHeads * DI];                 // B operand (K-major, swizzled)
+  float wq[kHeads];                                      // w_h * s_q,h
+  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain;
+  uint32_t tmem_base;
+  int abort;
+  int n_issued, n_mma;
 };
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Bounded wait that also gives up early once another role raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && *abort) return false;
+  }
+  *abort = 1;
+  return false;
+}
 
 }  // namespace
 
 template <int DI, bool REINDEX>
-__global__ void __launch_bounds__(kThreads) index_kernel(const __grid_constant__ CUtensorMap ik_map,
-                                                         const IndexArgs a) {
+__global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constant__ CUtensorMap ik_map,
+                                                            const IndexArgs a) {
   constexpr int MASK = DI == 128 ? 7 : 3;
-  constexpr int KS = DI / 32;          // k-steps of 32 bytes
+  constexpr int KS = DI / 32;   // MMA k-steps (32 bytes of E4M3 each)
+  constexpr uint32_t kIdesc = mma_idesc(128, kHeads, 0u /*E4M3*/, 0u /*E4M3*/);
   extern __shared__ uint8_t smem_raw[];
   IndexSmem<DI> &S = *reinterpret_cast<IndexSmem<DI> *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  volatile int *abort = &S.abort;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int row = blockIdx.y;                 // b * T_q + query
+  const int row = blockIdx.y;   // b * T_q + query
   const int b = row / a.T_q;
   const int t = a.q_pos[row];
   int n_vis = (t + 1) / a.m;
@@ -54,24 +84,31 @@ __global__ void __launch_bounds__(kThreads) index_kernel(const __grid_constant__
   if (n_vis < 0 || t < 0) n_vis = 0;
 
   const int tile0 = blockIdx.x * a.tiles_per_cta;
-  int tiles_row = REINDEX ? a.tiles_per_row : (n_vis + kTileRows - 1) / kTileRows;
+  const int tiles_row = REINDEX ? a.tiles_per_row : (n_vis + kTileRows - 1) / kTileRows;
   int tile1 = tile0 + a.tiles_per_cta;
   if (tile1 > tiles_row) tile1 = tiles_row;
   if (!REINDEX && blockIdx.x == 0 && tid == 0 && a.n_valid) a.n_valid[row] = n_vis;
   const int ntiles = tile1 - tile0;
   if (ntiles <= 0) return;
-
   const int32_t *pool = REINDEX ? a.pool + (size_t)row * a.P : nullptr;
 
-  // ---- barriers, then the producer starts streaming immediately
+  // ---- set-up: barriers (warp 0), TMEM (warp 1)
   if (tid == 0) {
-    prefetch_tmap(&ik_map);
-    for (int s = 0; s < kStages; ++s) mbar_init(&S.full[s], 1);
+    for (int s = 0; s < kStages; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
+    for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 4); }
+    mbar_init(&S.drain, 1);
+    S.abort = 0;
+    S.n_issued = 0;
+    S.n_mma = 0;
     fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
+    tmem_relinquish();
   }
   __syncthreads();
 
-  auto issue = [&](int i) {  // tile0 + i into stage i % kStages (thread 0 only)
+  auto issue = [&](int i) {   // tile tile0+i into stage i % kStages
     const int s = i % kStages;
     const int tile = tile0 + i;
     mbar_arrive_expect_tx(&S.full[s], kTileRows * DI);
@@ -80,7 +117,7 @@ __global__ void __launch_bounds__(kThreads) index_kernel(const __grid_constant__
       int r;
       if (REINDEX) {
         int blk = pool[tile * 16 + g];
-        if (blk < 0 || blk >= a.cap / 8) blk = 0;
+        if (blk < 0 || blk >= a.cap / 8) blk = 0;   // masked in the epilogue
         r = b * a.cap + blk * 8;
       } else {
         r = b * a.cap + tile * kTileRows + g * 8;
@@ -89,131 +126,129 @@ __global__ void __launch_bounds__(kThreads) index_kernel(const __grid_constant__
     }
   };
   if (tid == 0) {
-    for (int i = 0; i < ntiles && i < kStages; ++i) issue(i);
+    prefetch_tmap(&ik_map);
+    const int first = ntiles < kStages ? ntiles : kStages;
+    for (int i = 0; i < first; ++i) issue(i);
+    S.n_issued = first;
   }
 
-  // ---- indexer query: per head, FP8 with scale amax/448 (same rule as the keys)
+  // ---- indexer query (all warps): per head FP8 with scale amax/448, stored
+  // in the swizzled K-major layout the MMA reads
   const uint16_t *qrow = a.q_idx + (size_t)row * a.H_I * DI;
   const float *wrow = a.w + (size_t)row * a.H_I;
-  for (int h = warp; h < kMaxHeads; h += kThreads / 32) {
+  for (int h = warp; h < kHeads; h += kThreads / 32) {
+    float v[DI / 32];
+    float amax = 0.f;
     if (h < a.H_I) {
-      float v[DI / 32];
-      float amax = 0.f;
 #pragma unroll
       for (int i = 0; i < DI / 32; ++i) {
         v[i] = bf16_to_f32(qrow[h * DI + lane + 32 * i]);
         amax = fmaxf(amax, fabsf(v[i]));
       }
       for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float sq = __fdiv_rn(amax, 448.0f);
-#pragma unroll
-      for (int i = 0; i < DI / 32; ++i)
-        S.q8[h][lane + 32 * i] = (uint8_t)(sq == 0.f ? 0u : f32_to_e4m3(__fdiv_rn(v[i], sq)));
-      if (lane == 0) S.wq[h] = wrow[h] * sq;
-    } else {
-#pragma unroll
-      for (int i = 0; i < DI / 32; ++i) S.q8[h][lane + 32 * i] = 0;
-      if (lane == 0) S.wq[h] = 0.f;
     }
+    const float sq = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+    for (int i = 0; i < DI / 32; ++i) {
+      const int c = lane + 32 * i;
+      const uint32_t code = (h < a.H_I && sq != 0.f) ? f32_to_e4m3(__fdiv_rn(v[i], sq)) : 0u;
+      S.q8[swz<MASK>(h * DI + c)] = (uint8_t)code;
+    }
+    if (lane == 0) S.wq[h] = h < a.H_I ? wrow[h] * sq : 0.f;
   }
+  fence_proxy_async();   // generic-proxy writes of q8 -> visible to the tensor core
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
 
-  // B fragments (q8 as the 32x8 col-major operand: column n = head) and the
-  // head weights of this lane's accumulator columns.
-  const int gid = lane >> 2, tq = lane & 3;
-  const int ntn = (a.H_I + 7) / 8;
-  uint32_t bf[8][KS][2];
-  float wl[8][2];
-#pragma unroll
-  for (int n = 0; n < 8; ++n) {
-#pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      bf[n][k][0] = *reinterpret_cast<const uint32_t *>(&S.q8[n * 8 + gid][k * 32 + tq * 4]);
-      bf[n][k][1] = *reinterpret_cast<const uint32_t *>(&S.q8[n * 8 + gid][k * 32 + 16 + tq * 4]);
+  if (warp == 0) {
+    // ------------------------------------------------ TMA producer
+    if (lane == 0) {
+      for (int i = kStages; i < ntiles; ++i) {
+        const int s = i % kStages;
+        if (!wait_or_abort(&S.empty[s], ((i / kStages) - 1) & 1, abort)) break;
+        issue(i);
+        S.n_issued = i + 1;
+      }
     }
-    wl[n][0] = S.wq[n * 8 + tq * 2];
-    wl[n][1] = S.wq[n * 8 + tq * 2 + 1];
+  } else if (warp == 1) {
+    // ------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(S.q8);
+      for (int i = 0; i < ntiles; ++i) {
+        const int s = i % kStages, ab = i & 1;
+        if (!wait_or_abort(&S.full[s], (i / kStages) & 1, abort)) break;
+        if (i >= 2 && !wait_or_abort(&S.tempty[ab], ((i / 2) - 1) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(S.tile[s]);
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk)
+          tc_mma_f8(tmem + ab * kHeads, smem_desc_kmajor(a_addr + kk * 32, DI),
+                    smem_desc_kmajor(q_addr + kk * 32, DI), kIdesc, kk > 0 ? 1u : 0u);
+        tc_commit(&S.empty[s]);    // stage s may be refilled once these MMAs are done
+        tc_commit(&S.tfull[ab]);   // accumulator ab is ready for the epilogue
+        S.n_mma = i + 1;
+      }
+    }
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;                    // TMEM lane quarter of this warp
+    const int r = 32 * q + lane;               // tile row = TMEM lane
+    for (int i = 0; i < ntiles; ++i) {
+      const int ab = i & 1;
+      const int tile = tile0 + i;
+      int e;
+      bool valid;
+      if (REINDEX) {
+        const int blk = pool[tile * 16 + (r >> 3)];
+        e = blk * 8 + (r & 7);
+        valid = blk >= 0 && blk < a.cap / 8 && e < n_vis;
+      } else {
+        e = tile * kTileRows + r;
+        valid = e < n_vis;
+      }
+      const float sk = valid ? a.ik_scale[(size_t)b * a.cap + e] : 0.f;
+      int ok = 1;
+      if (lane == 0) ok = wait_or_abort(&S.tfull[ab], (i / 2) & 1, abort);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t acc[kHeads];
+      const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * kHeads;
+      tmem_ld_x32(taddr, acc);
+      tmem_ld_x32(taddr + 32, acc + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.tempty[ab]);
+      float sum = 0.f;
+#pragma unroll
+      for (int h = 0; h < kHeads; ++h) sum = fmaf(S.wq[h], fmaxf(__uint_as_float(acc[h]), 0.f), sum);
+      float *out = a.scores + (size_t)row * a.ld;
+      if (REINDEX) out[tile * kTileRows + r] = valid ? sum * sk : -INFINITY;
+      else if (valid) out[e] = sum * sk;
+    }
   }
 
-  // ---- main loop over tiles
-  for (int i = 0; i < ntiles; ++i) {
-    const int s = i % kStages;
-    const int tile = tile0 + i;
-    const bool ok = mbar_wait_bounded(&S.full[s], (i / kStages) & 1, kWaitLimit);
-    if (__syncthreads_or(!ok)) {   // block-uniform decision
-      if (tid == 0) {
-        flag(a.status, CSA2_DEV_TIMEOUT);
-        // copies of tiles i .. i+kStages-1 may still be landing in this
-        // CTA's shared memory: wait for them (bounded) before exiting
-        const int end = ntiles < i + kStages ? ntiles : i + kStages;
-        for (int j = i; j < end; ++j) mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1, kWaitLimit);
-      }
-      __syncthreads();
-      return;
+  // ---- teardown: on an abort, drain in-flight copies and MMAs (bounded),
+  // then free TMEM
+  __syncthreads();
+  if (S.abort) {
+    if (tid == 0) {
+      flag(a.status, CSA2_DEV_TIMEOUT);
+      for (int j = S.n_mma; j < S.n_issued; ++j)
+        mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1, kWaitLimit);
     }
-    const uint32_t base = smem_u32(S.tile[s]);
-#pragma unroll
-    for (int ms = 0; ms < 2; ++ms) {
-      const int r0 = warp * 32 + ms * 16;
-      // entry ids and scales of the two rows this lane finishes
-      const int rl = r0 + gid, rh = rl + 8;
-      int el, eh;
-      bool vl, vh;
-      if (REINDEX) {
-        const int bl = pool[tile * 16 + (rl >> 3)], bh = pool[tile * 16 + (rh >> 3)];
-        el = bl * 8 + (rl & 7);
-        eh = bh * 8 + (rh & 7);
-        vl = bl >= 0 && bl < a.cap / 8 && el < n_vis;
-        vh = bh >= 0 && bh < a.cap / 8 && eh < n_vis;
-      } else {
-        el = tile * kTileRows + rl;
-        eh = tile * kTileRows + rh;
-        vl = el < n_vis;
-        vh = eh < n_vis;
-      }
-      const float skl = vl ? a.ik_scale[(size_t)b * a.cap + el] : 0.f;
-      const float skh = vh ? a.ik_scale[(size_t)b * a.cap + eh] : 0.f;
-
-      float acc[8][4];
-#pragma unroll
-      for (int n = 0; n < 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-#pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        // A 16x32: matrices (rows 0-7 | 8-15) x (bytes 0-15 | 16-31)
-        const int r = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-        const int ch = 2 * k + (lane >> 4);
-        uint32_t af[4];
-        ldsm_x4(base + swz<MASK>(r * DI + ch * 16), af[0], af[1], af[2], af[3]);
-#pragma unroll
-        for (int n = 0; n < 8; ++n)
-          if (n < ntn) mma_e4m3_16832(acc[n], af, bf[n][k]);
-      }
-      float sl = 0.f, sh = 0.f;
-#pragma unroll
-      for (int n = 0; n < 8; ++n) {
-        sl += wl[n][0] * fmaxf(acc[n][0], 0.f) + wl[n][1] * fmaxf(acc[n][1], 0.f);
-        sh += wl[n][0] * fmaxf(acc[n][2], 0.f) + wl[n][1] * fmaxf(acc[n][3], 0.f);
-      }
-      sl += __shfl_xor_sync(0xffffffffu, sl, 1);
-      sl += __shfl_xor_sync(0xffffffffu, sl, 2);
-      sh += __shfl_xor_sync(0xffffffffu, sh, 1);
-      sh += __shfl_xor_sync(0xffffffffu, sh, 2);
-      if (tq == 0) {
-        float *out = a.scores + (size_t)row * a.ld;
-        if (REINDEX) {
-          out[tile * kTileRows + rl] = vl ? sl * skl : -INFINITY;
-          out[tile * kTileRows + rh] = vh ? sh * skh : -INFINITY;
-        } else {
-          if (vl) out[el] = sl * skl;
-          if (vh) out[eh] = sh * skh;
-        }
-      }
+    if (tid == 32) {
+      tc_commit(&S.drain);   // arrives when every MMA issued by this thread is done
+      mbar_wait_bounded(&S.drain, 0, kWaitLimit);
     }
-    __syncthreads();  // every warp is done with stage s
-    if (tid == 0 && i + kStages < ntiles) {
-      fence_proxy_async();
-      issue(i + kStages);
-    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 

@@ -61,21 +61,51 @@ __device__ int block_sum(int v, int *red) {
 
 // Threshold of the K largest keys among keys[0..n) (0 = absent).  Leaves the
 // result in st->thr / st->take_eq.  All threads of the block must call.
+// 8-bit digits starting at the highest bit where the present keys differ
+// (the bits above are common to all of them), so no pass is spent on a
+// digit every key shares.  Histogram updates take one atomic per warp when
+// the warp's active keys share a digit (the common case in the first pass).
 template <int NT>
 __device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist, SelState *st, int *red) {
-  const int tid = threadIdx.x, lane = tid & 31;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int cnt = 0;
-  for (int i = tid; i < n; i += NT) cnt += keys[i] != 0u;
-  const int nvalid = block_sum<NT>(cnt, red);
+  uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+  for (int i = tid; i < n; i += NT) {
+    const uint32_t k = keys[i];
+    if (k) { ++cnt; kmin = min(kmin, k); kmax = max(kmax, k); }
+  }
+  cnt = __reduce_add_sync(0xffffffffu, (unsigned)cnt);
+  kmin = __reduce_min_sync(0xffffffffu, kmin);
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  __syncthreads();
+  if (lane == 0) { red[warp] = cnt; hist[warp] = kmin; hist[32 + warp] = kmax; }
+  __syncthreads();
+  int nvalid = 0;
+  kmin = 0xFFFFFFFFu;
+  kmax = 0u;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) { nvalid += red[w]; kmin = min(kmin, hist[w]); kmax = max(kmax, hist[32 + w]); }
+  __syncthreads();
   if (nvalid <= K) {   // take every present key
     if (tid == 0) { st->thr = 1u; st->take_eq = 0x7fffffff; st->nvalid = nvalid; }
     __syncthreads();
     return;
   }
-  if (tid == 0) { st->prefix = 0u; st->mask = 0u; st->krem = K; st->nvalid = nvalid; }
+  // bits above `top` are the same in every present key
+  const int top = 31 - __clz(kmin ^ kmax | 1u);   // highest differing bit (>= 0)
+  int shift = top - 7;
+  const uint32_t common = top >= 31 ? 0u : (kmin >> (top + 1)) << (top + 1);
+  if (tid == 0) {
+    st->prefix = common;
+    st->mask = top >= 31 ? 0u : ~((1u << (top + 1)) - 1u);
+    st->krem = K;
+    st->nvalid = nvalid;
+  }
   const int iters = (n + NT - 1) / NT;
 #pragma unroll 1
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  while (true) {
+    const int sh = shift < 0 ? 0 : shift;            // last digit may be narrower
+    const uint32_t dmask = shift < 0 ? (0xFFu >> (-shift)) : 0xFFu;
     for (int i = tid; i < 256; i += NT) hist[i] = 0u;
     __syncthreads();
     const uint32_t prefix = st->prefix, mask = st->mask;
@@ -83,9 +113,17 @@ __device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist,
       const int i = j * NT + tid;
       const uint32_t k = i < n ? keys[i] : 0u;
       const bool act = k != 0u && (k & mask) == prefix;
-      const uint32_t bin = (k >> shift) & 255u;
-      const unsigned peers = __match_any_sync(0xffffffffu, act ? bin : 0x100u + lane);
-      if (act && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+      const uint32_t bin = (k >> sh) & dmask;
+      const unsigned am = __ballot_sync(0xffffffffu, act);
+      if (am) {
+        const int leader = __ffs(am) - 1;
+        const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+        if (__all_sync(0xffffffffu, !act || bin == b0)) {
+          if (lane == leader) atomicAdd(&hist[b0], (uint32_t)__popc(am));
+        } else if (act) {
+          atomicAdd(&hist[bin], 1u);
+        }
+      }
     }
     __syncthreads();
     if (tid < 32) {   // warp 0: lane l owns bins 8l..8l+7; find the bin holding the krem-th largest
@@ -110,11 +148,13 @@ __device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist,
           above += h;
         }
         st->krem = krem - (int)above;
-        st->prefix = prefix | ((uint32_t)bin << shift);
-        st->mask = mask | (255u << shift);
+        st->prefix = prefix | ((uint32_t)bin << sh);
+        st->mask = mask | (dmask << sh);
       }
     }
     __syncthreads();
+    if (sh == 0) break;
+    shift -= 8;
   }
   if (tid == 0) { st->thr = st->prefix; st->take_eq = st->krem; }
   __syncthreads();
