@@ -44,8 +44,9 @@ _PM, _PS = ctypes.POINTER(MainCacheDesc), ctypes.POINTER(SwaCacheDesc)
 
 SIGNATURES = {
     "csa2_append_quant": (_I, [_PM, _P, _P, _P, _PS, _P, _P, _I, _P]),
-    "csa2_index_full": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _P]),
-    "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P]),
+    "csa2_index_full": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _P, _SZ, _P]),
+    "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
+    "csa2_index_workspace_size": (_SZ, [_I, _I]),
     "csa2_topk": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P, _SZ, _P]),
     "csa2_topk_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "csa2_topk_noalloc": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P]),
@@ -147,20 +148,35 @@ def csa2_append_quant(main: MainCache | None, kv, gate, w_ik, swa: SwaCache | No
                                    _ptr(pos0, torch.int32), int(T), _stream(stream)))
 
 
-def csa2_index_full(main: MainCache, q_idx, w, q_pos, scores, n_valid=None, stream=None):
+def csa2_index_workspace_size(rows: int, d_I: int) -> int:
+    return int(lib().csa2_index_workspace_size(rows, d_I))
+
+
+def _ws_or_alloc(ws, nbytes, device):
+    """A caller workspace, or a fresh one of the needed size (binding convenience)."""
+    if ws is None:
+        ws = workspace(nbytes, device)
+    return ws
+
+
+def csa2_index_full(main: MainCache, q_idx, w, q_pos, scores, n_valid=None, ws=None, stream=None):
     T_q = q_pos.shape[-1]
     H_I = q_idx.shape[-2]
+    ws = _ws_or_alloc(ws, csa2_index_workspace_size(main.B * T_q, main.d_I), scores.device)
     _check(lib().csa2_index_full(ctypes.byref(main.desc()), _ptr(q_idx, torch.bfloat16), _ptr(w, torch.float32),
                                  _ptr(q_pos, torch.int32), T_q, H_I, _ptr(scores, torch.float32),
-                                 scores.shape[-1], _ptr(n_valid, torch.int32), _stream(stream)))
+                                 scores.shape[-1], _ptr(n_valid, torch.int32), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)))
 
 
-def csa2_index_reindex(main: MainCache, q_idx, w, q_pos, pool_blocks, pool_scores, stream=None):
+def csa2_index_reindex(main: MainCache, q_idx, w, q_pos, pool_blocks, pool_scores, ws=None, stream=None):
     T_q = q_pos.shape[-1]
     H_I = q_idx.shape[-2]
+    ws = _ws_or_alloc(ws, csa2_index_workspace_size(main.B * T_q, main.d_I), pool_scores.device)
     _check(lib().csa2_index_reindex(ctypes.byref(main.desc()), _ptr(q_idx, torch.bfloat16), _ptr(w, torch.float32),
                                     _ptr(q_pos, torch.int32), T_q, H_I, _ptr(pool_blocks, torch.int32),
-                                    pool_blocks.shape[-1], _ptr(pool_scores, torch.float32), _stream(stream)))
+                                    pool_blocks.shape[-1], _ptr(pool_scores, torch.float32), _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def csa2_topk_workspace_size(rows: int, n_cols: int, K: int, P_out: int = 0) -> int:

@@ -81,16 +81,16 @@ csa2_status get_encoder(EncodeTiled *fn) {
   return CSA2_OK;
 }
 
-// 2D map over the indexer-key plane [B*cap][d_I] (u8), boxes of 8 rows x d_I
-// bytes, swizzled to the d_I-byte pattern the kernel's ldmatrix addressing
-// expects.
-csa2_status encode_ik_map(const csa2_main_cache *m, CUtensorMap *map) {
+// 2D map over the indexer-key plane [B*cap][d_I] (u8), boxes of `box_rows`
+// rows x d_I bytes (128: a whole Full tile per copy; 8: one pool block),
+// swizzled to the d_I-byte pattern of the MMA's shared-memory descriptors.
+csa2_status encode_ik_map(const csa2_main_cache *m, CUtensorMap *map, int box_rows) {
   EncodeTiled enc;
   csa2_status st = get_encoder(&enc);
   if (st != CSA2_OK) return st;
   cuuint64_t dims[2] = {(cuuint64_t)m->d_I, (cuuint64_t)m->B * (cuuint64_t)m->cap};
   cuuint64_t strides[1] = {(cuuint64_t)m->d_I};
-  cuuint32_t box[2] = {(cuuint32_t)m->d_I, 8};
+  cuuint32_t box[2] = {(cuuint32_t)m->d_I, (cuuint32_t)box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, m->ik, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -212,8 +212,8 @@ csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, c
 }
 
 static csa2_status index_common(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
-                                const int32_t *q_pos, int T_q, int H_I, float *scores, IndexArgs *a,
-                                CUtensorMap *map) {
+                                const int32_t *q_pos, int T_q, int H_I, float *scores, void *ws, size_t ws_bytes,
+                                IndexArgs *a, CUtensorMap *map, int box_rows) {
   csa2_status st;
   if ((st = check_main(main, false)) != CSA2_OK) return st;
   if (!q_idx || !w || !q_pos || !scores) return fail(CSA2_ERR_INVALID_ARG, "NULL argument");
@@ -222,21 +222,32 @@ static csa2_status index_common(const csa2_main_cache *main, const uint16_t *q_i
   if (T_q <= 0) return fail(CSA2_ERR_INVALID_ARG, "T_q=%d", T_q);
   if (H_I < 1 || H_I > 64) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "H_I=%d not in [1,64]", H_I);
   if ((int64_t)main->B * T_q > 65535) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "B*T_q must be <= 65535");
-  if ((st = encode_ik_map(main, map)) != CSA2_OK) return st;
+  const size_t need = index_workspace_bytes(main->B * T_q, main->d_I);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(CSA2_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  if ((st = encode_ik_map(main, map, box_rows)) != CSA2_OK) return st;
   *a = IndexArgs{};
+  a->q8 = static_cast<uint8_t *>(ws);
+  a->wq = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) +
+                                    (((size_t)main->B * T_q * 64 * main->d_I + 15) & ~size_t(15)));
   a->ik_scale = main->ik_scale; a->n_entries = main->n_entries;
   a->B = main->B; a->cap = main->cap; a->m = main->m; a->dI = main->d_I;
   a->q_idx = q_idx; a->w = w; a->q_pos = q_pos; a->T_q = T_q; a->H_I = H_I; a->scores = scores;
   return CSA2_OK;
 }
 
+size_t csa2_index_workspace_size(int rows, int d_I) {
+  if (rows <= 0 || (d_I != 64 && d_I != 128)) return 0;
+  return index_workspace_bytes(rows, d_I);
+}
+
 csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                             const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
-                            int32_t *n_valid, csa2_stream_t stream) {
+                            int32_t *n_valid, void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
   IndexArgs a;
   CUtensorMap map;
-  csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, scores, &a, &map);
+  csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, scores, ws, ws_bytes, &a, &map, 128);
   if (st != CSA2_OK) return st;
   if (ld < main->cap) return fail(CSA2_ERR_INVALID_ARG, "ld=%lld < cap=%d", (long long)ld, main->cap);
   if (n_valid && !aligned16(n_valid)) return fail(CSA2_ERR_INVALID_ARG, "n_valid must be 16-byte aligned");
@@ -257,11 +268,11 @@ csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, 
 
 csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                                const int32_t *q_pos, int T_q, int H_I, const int32_t *pool_blocks, int P,
-                               float *pool_scores, csa2_stream_t stream) {
+                               float *pool_scores, void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
   IndexArgs a;
   CUtensorMap map;
-  csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, pool_scores, &a, &map);
+  csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, pool_scores, ws, ws_bytes, &a, &map, 8);
   if (st != CSA2_OK) return st;
   if (!pool_blocks || !aligned16(pool_blocks)) return fail(CSA2_ERR_INVALID_ARG, "pool_blocks must be a 16-byte aligned device pointer");
   if (P < 16 || P > 4096 || P % 16) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "P=%d must be a multiple of 16 in [16,4096]", P);
@@ -291,7 +302,7 @@ csa2_status csa2_topk(const float *scores, int rows, int64_t ld, int n_cols, con
   if (!scores || !out_idx || !aligned16(scores) || !aligned16(out_idx))
     return fail(CSA2_ERR_INVALID_ARG, "scores/out_idx must be 16-byte aligned device pointers");
   if (rows <= 0 || rows > 65535) return fail(CSA2_ERR_INVALID_ARG, "rows=%d", rows);
-  if (n_cols < 0 || n_cols > (1 << 24) || ld < n_cols) return fail(CSA2_ERR_INVALID_ARG, "n_cols=%d ld=%lld", n_cols, (long long)ld);
+  if (n_cols < 0 || n_cols > (1 << 20) || ld < n_cols) return fail(CSA2_ERR_INVALID_ARG, "n_cols=%d ld=%lld", n_cols, (long long)ld);
   if (K < 1 || K > 2048) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "K=%d not in [1,2048]", K);
   if (P_out < 0 || P_out > 4096) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "P_out=%d not in [0,4096]", P_out);
   if (P_out > 0 && (!out_pool || !aligned16(out_pool))) return fail(CSA2_ERR_INVALID_ARG, "out_pool needed");
@@ -299,7 +310,7 @@ csa2_status csa2_topk(const float *scores, int rows, int64_t ld, int n_cols, con
   if (pool_blocks && (!aligned16(pool_blocks) || n_cols % 8)) return fail(CSA2_ERR_INVALID_ARG, "pool_blocks alignment / n_cols%%8");
   if (n_valid && !aligned16(n_valid)) return fail(CSA2_ERR_INVALID_ARG, "n_valid alignment");
   const TopkPlan p = plan_topk(rows, n_cols, K, P_out);
-  if (!ws || ws_bytes < p.bytes || !aligned16(ws))
+  if (p.bytes > 0 && (!ws || ws_bytes < p.bytes || !aligned16(ws)))
     return fail(CSA2_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", p.bytes, ws_bytes);
   TopkArgs a{scores, rows, ld, n_cols, n_valid, pool_blocks, K, out_idx, P_out, out_pool, ws};
   cudaError_t e = launch_topk(a, p, reinterpret_cast<cudaStream_t>(stream));

@@ -5,8 +5,9 @@
 //   entry with no overlap and no absolute-position term; the indexer key is
 //   projected from the main KV.  Section "3) FP4 main KV + SWA Bounded
 //   Replay": FP4 main KV, FP8 window KV.
-// One block per group of up to 8 new entries (blockDim = D/2, thread t owns
-// channels 2t, 2t+1 and writes code byte t) and one block per window row.  The quantised bytes are
+// One 512-thread block per group of up to 8 new entries (thread t < D/2 owns
+// channels 2t, 2t+1 and writes code byte t; all threads share the projection)
+// and one block per window row.  The quantised bytes are
 // decided in binary32 with IEEE division, no contraction (explicit _rn
 // intrinsics), so they are reproducible bit for bit.
 #include "common.cuh"
@@ -87,7 +88,7 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   }
 
   // ---- pool + FP4 per entry (thread t: channels 2t, 2t+1; 8 threads per group)
-  for (int jj = 0; jj < count; ++jj) {
+  for (int jj = 0; jj < count && t < D / 2; ++jj) {
     const int e = p0 / m + j0 + jj;
     float x0, x1;
     if (m == 1) {
@@ -135,7 +136,7 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   // buffer.  Block j0 == 0 is the only one that reads or writes it; it reads
   // first (above) and writes after the barrier.
   __syncthreads();
-  if (m == 2 && j0 == 0 && ((p0 + a.T) & 1)) {
+  if (m == 2 && j0 == 0 && ((p0 + a.T) & 1) && t < D / 2) {
     const size_t src = ((size_t)b * a.T + (a.T - 1)) * D;
     reinterpret_cast<uint32_t *>(a.pending_kv + (size_t)b * D)[t] = reinterpret_cast<const uint32_t *>(a.kv + src)[t];
     reinterpret_cast<uint32_t *>(a.pending_gate + (size_t)b * D)[t] = reinterpret_cast<const uint32_t *>(a.gate + src)[t];
@@ -144,23 +145,35 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
 
   // ---- indexer key: k_i = sum_c x^_c W[c][i] in a fixed order (32-channel
   // groups by fmaf in ascending channel order from +0, then pairwise sums)
-  constexpr int E = 8;
-  for (int p = t; p < G * dI; p += blockDim.x) {
-    const int i = p % dI, g = p / dI;
-    const uint16_t *wcol = ws + (32 * g) * dI + i;
-    float acc[E];
+  if (count == 1) {   // decode: one entry, one chain per (group, output)
+    for (int p = t; p < G * dI; p += blockDim.x) {
+      const int i = p % dI, g = p / dI;
+      const uint16_t *wcol = ws + (32 * g) * dI + i;
+      const float *xg = xh + 32 * g;
+      float acc = 0.0f;
 #pragma unroll
-    for (int jj = 0; jj < E; ++jj) acc[jj] = 0.0f;
+      for (int c = 0; c < 32; ++c) acc = __fmaf_rn(xg[c], bf16_to_f32(wcol[c * dI]), acc);
+      part[g * dI + i] = acc;
+    }
+  } else {            // bulk: up to 8 entries share every W_ik read
+    constexpr int E = 8;
+    for (int p = t; p < G * dI; p += blockDim.x) {
+      const int i = p % dI, g = p / dI;
+      const uint16_t *wcol = ws + (32 * g) * dI + i;
+      float acc[E];
+#pragma unroll
+      for (int jj = 0; jj < E; ++jj) acc[jj] = 0.0f;
 #pragma unroll 4
-    for (int c = 0; c < 32; ++c) {
-      const float wv = bf16_to_f32(wcol[c * dI]);
+      for (int c = 0; c < 32; ++c) {
+        const float wv = bf16_to_f32(wcol[c * dI]);
+#pragma unroll
+        for (int jj = 0; jj < E; ++jj)
+          if (jj < count) acc[jj] = __fmaf_rn(xh[jj * D + 32 * g + c], wv, acc[jj]);
+      }
 #pragma unroll
       for (int jj = 0; jj < E; ++jj)
-        if (jj < count) acc[jj] = __fmaf_rn(xh[jj * D + 32 * g + c], wv, acc[jj]);
+        if (jj < count) part[(jj * G + g) * dI + i] = acc[jj];
     }
-#pragma unroll
-    for (int jj = 0; jj < E; ++jj)
-      if (jj < count) part[(jj * G + g) * dI + i] = acc[jj];
   }
   __syncthreads();
   for (int jj = 0; jj < count; ++jj) {
@@ -190,6 +203,7 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
 
 __device__ void append_window_row(const AppendArgs &a, int b, int r) {
   const int t = threadIdx.x;
+  if (t >= a.D / 2) return;
   const int p0 = a.pos0[b];
   const int cnt = a.T < a.W_cap ? a.T : a.W_cap;
   const int tau = a.T - cnt + r;
@@ -220,7 +234,7 @@ __global__ void append_kernel(const AppendArgs a) {
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
   const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq);
   if (blocks == 0) return cudaSuccess;
-  const int threads = a.D / 2;
+  const int threads = 512;   // quantisation uses the first D/2, the projection all of them
   // [E][D] + [E][G][dI] floats, 32 floats, then W_ik [D][dI] bf16
   const size_t smem = a.codes ? sizeof(float) * ((size_t)a.entries_per_block * (a.D + (a.D / 32) * a.dI) + 32) +
                                     sizeof(uint16_t) * (size_t)a.D * a.dI

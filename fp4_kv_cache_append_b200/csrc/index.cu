@@ -7,9 +7,9 @@
 //
 // Work layout: entries on M (128-entry tiles), indexer heads on N (64, zero
 // padded), d_I on K.  Per block (one query row, a run of tiles), 6 warps:
-//   warp 0     TMA producer: each tile is 16 boxes of 8 rows x d_I bytes (a
-//              Full tile at consecutive rows, a Reindex tile at the pool's
-//              block rows), hardware 128B/64B swizzle, into a STAGES ring
+//   warp 0     TMA producer: a Full tile is one box of 128 rows x d_I bytes,
+//              a Reindex tile 16 boxes of 8 rows at the pool's block rows;
+//              hardware 128B/64B swizzle, into a STAGES ring
 //   warp 1     allocates 128 TMEM columns and issues tcgen05.mma kind::f8f6f4
 //              (M=128, N=64, K=32 per instruction) into one of two TMEM
 //              accumulators; tcgen05.commit frees the smem stage and hands
@@ -18,7 +18,9 @@
 //              its 64 head accumulators with tcgen05.ld and reduces
 //              s_k * sum_h (w_h s_q,h) * max(acc_h, 0) -> one fp32 score
 // The head reduction never leaves registers; scores are written once,
-// coalesced.  All waits are bounded: a wait that gives up sets the device
+// coalesced.  The FP8 query of each row is prepared once by
+// index_prep_kernel (into the caller's workspace, already in the MMA's
+// swizzled layout) and bulk-copied into every block of that row.  All waits are bounded: a wait that gives up sets the device
 // status bit and an abort flag that stops every role; in-flight copies and
 // MMAs are then drained (bounded) and TMEM is freed before the block exits.
 #include "common.cuh"
@@ -40,7 +42,7 @@ struct IndexSmem {
   alignas(1024) uint8_t tile[kStages][kTileRows * DI];   // A operand ring (K-major, swizzled)
   alignas(1024) uint8_t q8[kHeads * DI];                 // B operand (K-major, swizzled)
   float wq[kHeads];                                      // w_h * s_q,h
-  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain;
+  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain, qbar;
   uint32_t tmem_base;
   int abort;
   int n_issued, n_mma;
@@ -61,6 +63,40 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 }
 
 }  // namespace
+
+// Indexer query of one row: per head, E4M3 codes with scale amax/448 (the
+// rule of the keys), laid out as the MMA's B operand (64 rows x DI bytes,
+// K-major, swizzled), and the head weights w_h * s_q,h.
+// One warp per head: grid (rows, 8) x 256 threads.
+template <int DI>
+__global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
+  constexpr int MASK = DI == 128 ? 7 : 3;
+  const int row = blockIdx.x, lane = threadIdx.x & 31;
+  const uint16_t *qrow = a.q_idx + (size_t)row * a.H_I * DI;
+  const float *wrow = a.w + (size_t)row * a.H_I;
+  uint8_t *q8 = a.q8 + (size_t)row * kHeads * DI;
+  {
+    const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
+    float v[DI / 32];
+    float amax = 0.f;
+    if (h < a.H_I) {
+#pragma unroll
+      for (int i = 0; i < DI / 32; ++i) {
+        v[i] = bf16_to_f32(qrow[h * DI + lane + 32 * i]);
+        amax = fmaxf(amax, fabsf(v[i]));
+      }
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    }
+    const float sq = __fdiv_rn(amax, 448.0f);
+#pragma unroll
+    for (int i = 0; i < DI / 32; ++i) {
+      const int c = lane + 32 * i;
+      const uint32_t code = (h < a.H_I && sq != 0.f) ? f32_to_e4m3(__fdiv_rn(v[i], sq)) : 0u;
+      q8[swz<MASK>(h * DI + c)] = (uint8_t)code;
+    }
+    if (lane == 0) a.wq[(size_t)row * kHeads + h] = h < a.H_I ? wrow[h] * sq : 0.f;
+  }
+}
 
 template <int DI, bool REINDEX>
 __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constant__ CUtensorMap ik_map,
@@ -97,6 +133,7 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
     for (int s = 0; s < kStages; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
     for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 4); }
     mbar_init(&S.drain, 1);
+    mbar_init(&S.qbar, 1);
     S.abort = 0;
     S.n_issued = 0;
     S.n_mma = 0;
@@ -112,51 +149,27 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
     const int s = i % kStages;
     const int tile = tile0 + i;
     mbar_arrive_expect_tx(&S.full[s], kTileRows * DI);
+    if (REINDEX) {   // 16 boxes of 8 rows at the pool's blocks
 #pragma unroll 1
-    for (int g = 0; g < 16; ++g) {
-      int r;
-      if (REINDEX) {
+      for (int g = 0; g < 16; ++g) {
         int blk = pool[tile * 16 + g];
         if (blk < 0 || blk >= a.cap / 8) blk = 0;   // masked in the epilogue
-        r = b * a.cap + blk * 8;
-      } else {
-        r = b * a.cap + tile * kTileRows + g * 8;
+        tma_load_2d(&S.tile[s][g * 8 * DI], &ik_map, 0, b * a.cap + blk * 8, &S.full[s]);
       }
-      tma_load_2d(&S.tile[s][g * 8 * DI], &ik_map, 0, r, &S.full[s]);
+    } else {         // one 128-row box
+      tma_load_2d(&S.tile[s][0], &ik_map, 0, b * a.cap + tile * kTileRows, &S.full[s]);
     }
   };
   if (tid == 0) {
     prefetch_tmap(&ik_map);
+    // the prepared query (B operand) and head weights of this row
+    mbar_arrive_expect_tx(&S.qbar, kHeads * DI + kHeads * 4);
+    bulk_load(S.q8, a.q8 + (size_t)row * kHeads * DI, kHeads * DI, &S.qbar);
+    bulk_load(S.wq, a.wq + (size_t)row * kHeads, kHeads * 4, &S.qbar);
     const int first = ntiles < kStages ? ntiles : kStages;
     for (int i = 0; i < first; ++i) issue(i);
     S.n_issued = first;
   }
-
-  // ---- indexer query (all warps): per head FP8 with scale amax/448, stored
-  // in the swizzled K-major layout the MMA reads
-  const uint16_t *qrow = a.q_idx + (size_t)row * a.H_I * DI;
-  const float *wrow = a.w + (size_t)row * a.H_I;
-  for (int h = warp; h < kHeads; h += kThreads / 32) {
-    float v[DI / 32];
-    float amax = 0.f;
-    if (h < a.H_I) {
-#pragma unroll
-      for (int i = 0; i < DI / 32; ++i) {
-        v[i] = bf16_to_f32(qrow[h * DI + lane + 32 * i]);
-        amax = fmaxf(amax, fabsf(v[i]));
-      }
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    }
-    const float sq = __fdiv_rn(amax, 448.0f);
-#pragma unroll
-    for (int i = 0; i < DI / 32; ++i) {
-      const int c = lane + 32 * i;
-      const uint32_t code = (h < a.H_I && sq != 0.f) ? f32_to_e4m3(__fdiv_rn(v[i], sq)) : 0u;
-      S.q8[swz<MASK>(h * DI + c)] = (uint8_t)code;
-    }
-    if (lane == 0) S.wq[h] = h < a.H_I ? wrow[h] * sq : 0.f;
-  }
-  fence_proxy_async();   // generic-proxy writes of q8 -> visible to the tensor core
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -176,7 +189,8 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(S.q8);
-      for (int i = 0; i < ntiles; ++i) {
+      const bool qok = wait_or_abort(&S.qbar, 0, abort);
+      for (int i = 0; i < ntiles && qok; ++i) {
         const int s = i % kStages, ab = i & 1;
         if (!wait_or_abort(&S.full[s], (i / kStages) & 1, abort)) break;
         if (i >= 2 && !wait_or_abort(&S.tempty[ab], ((i / 2) - 1) & 1, abort)) break;
@@ -195,11 +209,9 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
     // ------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;                    // TMEM lane quarter of this warp
     const int r = 32 * q + lane;               // tile row = TMEM lane
-    for (int i = 0; i < ntiles; ++i) {
-      const int ab = i & 1;
+    // entry id, validity and key scale of this lane's row in tile i
+    auto row_of = [&](int i, int &e, bool &valid, float &sk) {
       const int tile = tile0 + i;
-      int e;
-      bool valid;
       if (REINDEX) {
         const int blk = pool[tile * 16 + (r >> 3)];
         e = blk * 8 + (r & 7);
@@ -208,7 +220,23 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
         e = tile * kTileRows + r;
         valid = e < n_vis;
       }
-      const float sk = valid ? a.ik_scale[(size_t)b * a.cap + e] : 0.f;
+      sk = valid ? a.ik_scale[(size_t)b * a.cap + e] : 0.f;
+    };
+    int e_next;
+    bool v_next;
+    float sk_next;
+    row_of(0, e_next, v_next, sk_next);
+    int qok = 1;
+    if (lane == 0) qok = wait_or_abort(&S.qbar, 0, abort);   // head weights landed in smem
+    qok = __shfl_sync(0xffffffffu, qok, 0);
+    __syncwarp();
+    for (int i = 0; i < ntiles && qok; ++i) {
+      const int ab = i & 1;
+      const int tile = tile0 + i;
+      const int e = e_next;
+      const bool valid = v_next;
+      const float sk = sk_next;
+      if (i + 1 < ntiles) row_of(i + 1, e_next, v_next, sk_next);   // prefetch one tile ahead
       int ok = 1;
       if (lane == 0) ok = wait_or_abort(&S.tfull[ab], (i / 2) & 1, abort);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -222,9 +250,10 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.tempty[ab]);
-      float sum = 0.f;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};   // independent chains
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) sum = fmaf(S.wq[h], fmaxf(__uint_as_float(acc[h]), 0.f), sum);
+      for (int h = 0; h < kHeads; ++h) s4[h & 3] = fmaf(S.wq[h], fmaxf(__uint_as_float(acc[h]), 0.f), s4[h & 3]);
+      const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       float *out = a.scores + (size_t)row * a.ld;
       if (REINDEX) out[tile * kTileRows + r] = valid ? sum * sk : -INFINITY;
       else if (valid) out[e] = sum * sk;
@@ -237,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
   if (S.abort) {
     if (tid == 0) {
       flag(a.status, CSA2_DEV_TIMEOUT);
+      mbar_wait_bounded(&S.qbar, 0, kWaitLimit);
       for (int j = S.n_mma; j < S.n_issued; ++j)
         mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1, kWaitLimit);
     }
@@ -252,8 +282,16 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
   }
 }
 
+size_t index_workspace_bytes(int rows, int dI) {
+  const size_t q = ((size_t)rows * kHeads * dI + 15) & ~size_t(15);
+  return q + (size_t)rows * kHeads * 4;
+}
+
 template <int DI, bool REINDEX>
 static cudaError_t launch_t(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
+  index_prep_kernel<DI><<<dim3(a.B * a.T_q, kHeads / 8), 256, 0, s>>>(a);
+  cudaError_t pe = cudaGetLastError();
+  if (pe != cudaSuccess) return pe;
   const size_t smem = sizeof(IndexSmem<DI>) + 1024;
   auto k = index_kernel<DI, REINDEX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

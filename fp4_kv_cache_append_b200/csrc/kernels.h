@@ -44,8 +44,11 @@ struct IndexArgs {
   const int32_t *pool;    // reindex mode: [B*T_q][P]
   int P;
   int tiles_per_row, tiles_per_cta;
+  uint8_t *q8;            // workspace: [B*T_q][64*dI] prepared FP8 query (MMA layout)
+  float *wq;              // workspace: [B*T_q][64] w_h * s_q,h
   unsigned int *status;
 };
+size_t index_workspace_bytes(int rows, int dI);
 cudaError_t launch_index(const CUtensorMap &ik_map, const IndexArgs &a, bool reindex, int sms,
                          cudaStream_t s);
 
@@ -63,14 +66,16 @@ struct TopkArgs {
   void *ws;
 };
 struct TopkPlan {
-  int chunk;      // columns per first-stage block
-  int nchunks;
-  int k1;         // candidates kept per chunk
-  int p1;         // pool candidates kept per chunk
-  size_t bytes;   // workspace bytes
+  int nchunks;        // column chunks per row (histogram / filter blocks)
+  int nb;             // blocks of 8 columns per row
+  size_t off_hist, off_histb, off_cnt, off_range, off_sel, off_cand, off_selb, off_candb;
+  size_t zero_bytes;  // [0, zero_bytes) is cleared at the start of every call
+  size_t bytes;       // workspace bytes
 };
 TopkPlan plan_topk(int rows, int n_cols, int K, int P_out);
 cudaError_t launch_topk(const TopkArgs &a, const TopkPlan &p, cudaStream_t s);
+bool topk_cluster_fits(int n_cols);                              // one cluster per row, no workspace
+cudaError_t launch_topk_cluster(const TopkArgs &a, cudaStream_t s);
 
 struct AttnArgs {
   const uint8_t *codes, *scales;

@@ -88,7 +88,7 @@ extern "C" CSA2_API csa2_status csa2_topk_noalloc(const float *scores, int rows,
   if (!scores || !out_idx || !noalloc_aligned16(scores) || !noalloc_aligned16(out_idx))
     return noalloc_fail(CSA2_ERR_INVALID_ARG, "scores/out_idx must be 16-byte aligned device pointers");
   if (rows <= 0 || rows > 65535) return noalloc_fail(CSA2_ERR_INVALID_ARG, "rows=%d", rows);
-  if (n_cols < 0 || n_cols > (1 << 24) || ld < n_cols)
+  if (n_cols < 0 || n_cols > (1 << 20) || ld < n_cols)
     return noalloc_fail(CSA2_ERR_INVALID_ARG, "n_cols=%d ld=%lld", n_cols, (long long)ld);
   if (K < 1 || K > 2048) return noalloc_fail(CSA2_ERR_UNSUPPORTED_SHAPE, "K=%d not in [1,2048]", K);
   if (P_out < 0 || P_out > 4096) return noalloc_fail(CSA2_ERR_UNSUPPORTED_SHAPE, "P_out=%d not in [0,4096]", P_out);

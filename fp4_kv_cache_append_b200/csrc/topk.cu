@@ -1,21 +1,33 @@
-// Top-K selection and the hierarchical candidate pool.
+// Top-K selection and the hierarchical candidate pool (rows of more than
+// 65,536 columns; shorter rows use the single-launch cluster kernel of
+// topk_cluster.cu).
 //   DeepSeek-V4.1-Flash (jaehun.me review), section "2) CSA2": each Full or
 //   Reindex layer keeps the Top-512 entries; the first Full layer of the
 //   decoder also builds the pool of <= 2,048 blocks x 8 positions that the
 //   Reindex layers rescore (paper sec. 2.3.2, 4.2.1, Fig. 5).
 // Order: score descending, ties -> smaller column; absent = non-finite.  The
-// result lists the chosen columns in ascending order, -1 padded.
+// result lists the chosen columns in ascending order, -1 padded.  A block's
+// score is the maximum of its present columns.
 //
-// Two launches, no cross-block waiting:
-//  1. topk_chunk_kernel: one block per (row, chunk of columns) keeps the
-//     chunk's best k1 columns (and best p1 blocks of 8) with a 4-pass 8-bit
-//     radix select over order-preserving 32-bit keys held in shared memory,
-//     then an order-preserving compaction (ballots) into the workspace.
-//  2. topk_merge_kernel: one block per row repeats the select over the
-//     concatenated candidates (already in column order) and writes the
-//     result, mapping columns through the pool for Reindex rows.
-// The global Top-K is inside the union of the chunks' Top-Ks because the
-// (key, -column) order is total.
+// Scores become order-preserving 32-bit keys (0 = absent).  Four kernels
+// after a memset of the per-row counters, none of them waiting on another
+// block:
+//  0. topk_range_kernel  (rows x column chunks): the row's smallest and
+//     largest present key (atomic max of key and of ~key).
+//  1. topk_hist_kernel   (same grid): 2048-bin histogram of the digit
+//     (key - min) >> shift, the shift chosen so the bins span the row's key
+//     range, for entries and for block maxima.
+//  2. topk_filter_kernel (same grid): every block derives the threshold bin
+//     T (the bin holding the K-th key) from the histogram, and appends the
+//     columns above T to the row's "selected" list and the columns in T to
+//     its "candidates" list (one atomic per warp and list).
+//  3. topk_select_kernel (one block per row): exact radix select among the
+//     candidates (a second select on the column among keys equal to the
+//     threshold, so ties go to smaller columns); the chosen columns are
+//     marked in a bitmap and written in ascending order by a prefix popcount
+//     (mapped through the pool for Reindex rows).
+// Binning over the actual range keeps the threshold bin small even when a
+// row's scores sit within a few percent of each other.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -23,9 +35,11 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kT1 = 512;
-constexpr int kT2 = 1024;
-constexpr int kMergeSmemCands = 16384;
+constexpr int kBins = 2048;          // digit = (key - kmin) >> shift, 11 bits
+constexpr int kColsPerBlock = 4096;  // columns per hist/filter block
+constexpr int kTF = 256;             // hist/filter threads: 16 columns each
+constexpr int kTS = 1024;            // select threads
+constexpr int kSmemCands = 12288;    // candidates staged in shared memory by the select kernel
 
 // Order-preserving key of a score: larger score -> larger key; -0 == +0;
 // non-finite -> 0 (absent).
@@ -36,42 +50,140 @@ __device__ __forceinline__ uint32_t score_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-struct SelState {
-  uint32_t thr;     // keys > thr are taken; keys == thr are taken ...
-  int take_eq;      // ... for the first take_eq of them in column order
-  uint32_t prefix, mask;
-  int krem;
-  int nvalid;
-  int found_bin;
-  int warp_gt[32], warp_eq[32];
+struct Ws {
+  uint32_t *hist, *histb;   // [rows][kBins]
+  uint32_t *cnt;            // [rows][4]: selected, candidates, selected blocks, candidate blocks
+  uint32_t *range;          // [rows][2]: max key, max of ~key (both start at 0)
+  int32_t *sel, *cand, *selb, *candb;
 };
 
-template <int NT>
-__device__ int block_sum(int v, int *red) {
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int s = 0;
-#pragma unroll
-  for (int w = 0; w < NT / 32; ++w) s += red[w];
-  return s;
+// Digit of a present key within the row's key range [kmin, kmax].
+struct Binning {
+  uint32_t kmin;
+  int shift;
+  __device__ __forceinline__ int digit(uint32_t key) const { return (int)((key - kmin) >> shift); }
+};
+
+__device__ __forceinline__ Ws ws_view(const TopkArgs &a, const TopkPlan &p) {
+  uint8_t *q = reinterpret_cast<uint8_t *>(a.ws);
+  Ws w;
+  w.hist = reinterpret_cast<uint32_t *>(q + p.off_hist);
+  w.histb = reinterpret_cast<uint32_t *>(q + p.off_histb);
+  w.cnt = reinterpret_cast<uint32_t *>(q + p.off_cnt);
+  w.range = reinterpret_cast<uint32_t *>(q + p.off_range);
+  w.sel = reinterpret_cast<int32_t *>(q + p.off_sel);
+  w.cand = reinterpret_cast<int32_t *>(q + p.off_cand);
+  w.selb = reinterpret_cast<int32_t *>(q + p.off_selb);
+  w.candb = reinterpret_cast<int32_t *>(q + p.off_candb);
+  return w;
 }
 
-// Threshold of the K largest keys among keys[0..n) (0 = absent).  Leaves the
-// result in st->thr / st->take_eq.  All threads of the block must call.
-// 8-bit digits starting at the highest bit where the present keys differ
-// (the bits above are common to all of them), so no pass is spent on a
-// digit every key shares.  Histogram updates take one atomic per warp when
-// the warp's active keys share a digit (the common case in the first pass).
+__device__ __forceinline__ int row_cols(const TopkArgs &a, int row) {
+  int n = a.n_cols;
+  if (a.n_valid) {
+    const int v = a.n_valid[row];
+    if (v < n) n = v < 0 ? 0 : v;
+  }
+  return n;
+}
+
+__device__ __forceinline__ Binning row_binning(const Ws &w, int row) {
+  const uint32_t kmax = w.range[2 * row], kmin = ~w.range[2 * row + 1];
+  Binning b;
+  b.kmin = kmin;
+  const uint32_t span = kmax > kmin ? kmax - kmin : 0u;
+  b.shift = span >= (uint32_t)kBins ? (32 - __clz(span)) - 11 : 0;
+  return b;
+}
+
+// Histogram update, one atomic per warp when the warp's present keys share a bin.
+__device__ __forceinline__ void hist_add(uint32_t *h, uint32_t key, const Binning &bn, int lane) {
+  const bool act = key != 0u;
+  const uint32_t bin = act ? (uint32_t)bn.digit(key) : 0u;
+  const unsigned am = __ballot_sync(0xffffffffu, act);
+  if (!am) return;
+  const int leader = __ffs(am) - 1;
+  const uint32_t b0 = __shfl_sync(0xffffffffu, bin, leader);
+  if (__all_sync(0xffffffffu, !act || bin == b0)) {
+    if (lane == leader) atomicAdd(&h[b0], (uint32_t)__popc(am));
+  } else if (act) {
+    atomicAdd(&h[bin], 1u);
+  }
+}
+
+// Append `val` to list[] for the lanes with flag set; one atomic per warp.
+__device__ __forceinline__ void warp_append(bool flag, int32_t val, uint32_t *counter, int32_t *list, int lane) {
+  const unsigned m = __ballot_sync(0xffffffffu, flag);
+  if (!m) return;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(counter, (uint32_t)__popc(m));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  if (flag) list[base + __popc(m & ((1u << lane) - 1u))] = val;
+}
+
+// Threshold bin of the K-th largest key from a row histogram: the bin T whose
+// keys, with all keys of higher bins (`above` of them), reach K.  Fewer than
+// K present keys: T = -1 and above = their number.  All threads call; every
+// thread gets the result.
 template <int NT>
-__device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist, SelState *st, int *red) {
+__device__ void find_threshold(const uint32_t *hist, int K, int &T, int &above, int *sm_ws) {
+  constexpr int BPT = kBins / NT;   // bins per thread
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t h[BPT];
+  uint32_t local = 0;
+#pragma unroll
+  for (int i = 0; i < BPT; ++i) { h[i] = hist[tid * BPT + i]; local += h[i]; }
+  uint32_t v = local;   // inclusive suffix over lanes >= lane
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, v, o);
+    if (lane + o < 32) v += y;
+  }
+  __syncthreads();
+  if (lane == 0) sm_ws[warp] = (int)v;
+  __syncthreads();
+  uint32_t higher = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < NT / 32; ++w) {
+    const uint32_t s = (uint32_t)sm_ws[w];
+    total += s;
+    if (w > warp) higher += s;
+  }
+  const uint32_t excl = v - local + higher;   // keys in bins above this thread's
+  if (total <= (uint32_t)K) {
+    if (tid == 0) { sm_ws[32] = -1; sm_ws[33] = (int)total; }
+  } else if (excl < (uint32_t)K && excl + local >= (uint32_t)K) {
+    uint32_t ab = excl;
+    int t_bin = tid * BPT;
+    for (int i = BPT - 1; i >= 0; --i) {
+      if (ab + h[i] >= (uint32_t)K) { t_bin = tid * BPT + i; break; }
+      ab += h[i];
+    }
+    sm_ws[32] = t_bin;
+    sm_ws[33] = (int)ab;
+  }
+  __syncthreads();
+  T = sm_ws[32];
+  above = sm_ws[33];
+  __syncthreads();
+}
+
+// Threshold of the K largest keys key(0..n-1) (0 = absent): keys > thr are
+// taken, and take_eq of the keys == thr.  8-bit digits from the highest bit
+// where present keys differ.
+struct SelState {
+  uint32_t thr, prefix, mask;
+  int take_eq, krem;
+};
+
+template <int NT, class KeyF>
+__device__ void radix_select(KeyF key, int n, int K, uint32_t *hist, SelState *st, int *red) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   int cnt = 0;
   uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
   for (int i = tid; i < n; i += NT) {
-    const uint32_t k = keys[i];
+    const uint32_t k = key(i);
     if (k) { ++cnt; kmin = min(kmin, k); kmax = max(kmax, k); }
   }
   cnt = __reduce_add_sync(0xffffffffu, (unsigned)cnt);
@@ -86,32 +198,29 @@ __device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist,
 #pragma unroll
   for (int w = 0; w < NT / 32; ++w) { nvalid += red[w]; kmin = min(kmin, hist[w]); kmax = max(kmax, hist[32 + w]); }
   __syncthreads();
-  if (nvalid <= K) {   // take every present key
-    if (tid == 0) { st->thr = 1u; st->take_eq = 0x7fffffff; st->nvalid = nvalid; }
+  if (nvalid <= K) {
+    if (tid == 0) { st->thr = 1u; st->take_eq = 0x7fffffff; }
     __syncthreads();
     return;
   }
-  // bits above `top` are the same in every present key
-  const int top = 31 - __clz(kmin ^ kmax | 1u);   // highest differing bit (>= 0)
+  const int top = 31 - __clz((kmin ^ kmax) | 1u);   // highest differing bit
   int shift = top - 7;
-  const uint32_t common = top >= 31 ? 0u : (kmin >> (top + 1)) << (top + 1);
   if (tid == 0) {
-    st->prefix = common;
+    st->prefix = top >= 31 ? 0u : (kmin >> (top + 1)) << (top + 1);
     st->mask = top >= 31 ? 0u : ~((1u << (top + 1)) - 1u);
     st->krem = K;
-    st->nvalid = nvalid;
   }
   const int iters = (n + NT - 1) / NT;
 #pragma unroll 1
   while (true) {
-    const int sh = shift < 0 ? 0 : shift;            // last digit may be narrower
+    const int sh = shift < 0 ? 0 : shift;
     const uint32_t dmask = shift < 0 ? (0xFFu >> (-shift)) : 0xFFu;
     for (int i = tid; i < 256; i += NT) hist[i] = 0u;
     __syncthreads();
     const uint32_t prefix = st->prefix, mask = st->mask;
     for (int j = 0; j < iters; ++j) {
       const int i = j * NT + tid;
-      const uint32_t k = i < n ? keys[i] : 0u;
+      const uint32_t k = i < n ? key(i) : 0u;
       const bool act = k != 0u && (k & mask) == prefix;
       const uint32_t bin = (k >> sh) & dmask;
       const unsigned am = __ballot_sync(0xffffffffu, act);
@@ -126,20 +235,19 @@ __device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist,
       }
     }
     __syncthreads();
-    if (tid < 32) {   // warp 0: lane l owns bins 8l..8l+7; find the bin holding the krem-th largest
+    if (tid < 32) {   // lane l owns bins 8l..8l+7: find the bin holding the krem-th largest
       const int krem = st->krem;
       uint32_t own = 0;
 #pragma unroll
       for (int q = 0; q < 8; ++q) own += hist[8 * lane + q];
-      uint32_t suf = own;   // inclusive suffix over lanes >= lane
+      uint32_t suf = own;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const uint32_t v = __shfl_down_sync(0xffffffffu, suf, o);
         if (lane + o < 32) suf += v;
       }
-      const uint32_t above_lane = suf - own;   // keys in bins of higher lanes
-      const bool here = suf >= (uint32_t)krem && above_lane < (uint32_t)krem;
-      if (here) {
+      const uint32_t above_lane = suf - own;
+      if (suf >= (uint32_t)krem && above_lane < (uint32_t)krem) {
         uint32_t above = above_lane;
         int bin = 8 * lane;
         for (int q = 7; q >= 0; --q) {
@@ -160,201 +268,289 @@ __device__ void radix_select(const uint32_t *keys, int n, int K, uint32_t *hist,
   __syncthreads();
 }
 
-// Column-ordered compaction of the selected keys: emit(pos, i, key) for each
-// taken i in increasing i.  Returns the number taken.  All threads call.
-template <int NT, class Emit>
-__device__ int ordered_emit(const uint32_t *keys, int n, SelState *st, Emit emit) {
-  constexpr int NW = NT / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const uint32_t thr = st->thr;
-  const int take_eq = st->take_eq;
-  const int per = ((n + NW - 1) / NW + 31) & ~31;
-  const int lo = warp * per;
-  const int hi = lo + per < n ? lo + per : n;
-  int gt = 0, eq = 0;
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t k = i < hi ? keys[i] : 0u;
-    gt += __popc(__ballot_sync(0xffffffffu, k > thr));
-    eq += __popc(__ballot_sync(0xffffffffu, k == thr));
-  }
-  __syncthreads();
-  if (lane == 0) { st->warp_gt[warp] = gt; st->warp_eq[warp] = eq; }
-  __syncthreads();
-  int gt_before = 0, eq_before = 0, gt_all = 0, eq_all = 0;
-  for (int w = 0; w < NW; ++w) {
-    if (w < warp) { gt_before += st->warp_gt[w]; eq_before += st->warp_eq[w]; }
-    gt_all += st->warp_gt[w];
-    eq_all += st->warp_eq[w];
-  }
-  int out = gt_before + (eq_before < take_eq ? eq_before : take_eq);
-  const unsigned lt = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += 32) {
-    const int i = base + lane;
-    const uint32_t k = i < hi ? keys[i] : 0u;
-    const unsigned eqb = __ballot_sync(0xffffffffu, k == thr);
-    const int rank = eq_before + __popc(eqb & lt);
-    const bool take = k > thr || (k == thr && rank < take_eq);
-    const unsigned tb = __ballot_sync(0xffffffffu, take);
-    if (take) emit(out + __popc(tb & lt), i, k);
-    out += __popc(tb);
-    eq_before += __popc(eqb);
-  }
-  return gt_all + (eq_all < take_eq ? eq_all : take_eq);
-}
-
-struct WsView {
-  uint32_t *ckey;   // [rows][nchunks][k1]
-  int32_t *ccol;
-  uint32_t *pkey;   // [rows][nchunks][p1]
-  int32_t *pblk;
-};
-
-__host__ __device__ inline WsView ws_view(void *ws, int rows, const TopkPlan &p) {
-  WsView v;
-  const size_t nk = (size_t)rows * p.nchunks * p.k1, np = (size_t)rows * p.nchunks * p.p1;
-  uint8_t *q = reinterpret_cast<uint8_t *>(ws);
-  v.ckey = reinterpret_cast<uint32_t *>(q);
-  q += nk * 4;
-  v.ccol = reinterpret_cast<int32_t *>(q);
-  q += nk * 4;
-  v.pkey = reinterpret_cast<uint32_t *>(q);
-  q += np * 4;
-  v.pblk = reinterpret_cast<int32_t *>(q);
-  return v;
-}
-
-__global__ void __launch_bounds__(kT1) topk_chunk_kernel(const TopkArgs a, const TopkPlan p) {
-  extern __shared__ uint32_t sm1[];
-  __shared__ uint32_t hist[256];
-  __shared__ SelState st;
-  __shared__ int red[32];
-  uint32_t *keys = sm1;                 // [chunk]
-  uint32_t *bkeys = sm1 + p.chunk;      // [chunk/8]
-  const int row = blockIdx.y, chunk = blockIdx.x, tid = threadIdx.x;
-  const int c0 = chunk * p.chunk;
-  int ncol = a.n_cols;
-  if (a.n_valid) {
-    const int nv = a.n_valid[row];
-    if (nv < ncol) ncol = nv < 0 ? 0 : nv;
-  }
-  int cnt = ncol - c0;
-  cnt = cnt < 0 ? 0 : (cnt > p.chunk ? p.chunk : cnt);
-  const float *srow = a.scores + (size_t)row * a.ld + c0;
-  for (int i = tid; i < p.chunk; i += kT1) keys[i] = i < cnt ? score_key(srow[i]) : 0u;
-  __syncthreads();
-
-  WsView v = ws_view(a.ws, a.rows, p);
-  const size_t base = ((size_t)row * p.nchunks + chunk) * p.k1;
-  radix_select<kT1>(keys, p.chunk, p.k1, hist, &st, red);
-  const int taken = ordered_emit<kT1>(keys, p.chunk, &st, [&](int pos, int i, uint32_t k) {
-    v.ckey[base + pos] = k;
-    v.ccol[base + pos] = c0 + i;
-  });
-  for (int i = taken + tid; i < p.k1; i += kT1) { v.ckey[base + i] = 0u; v.ccol[base + i] = -1; }
-
-  if (a.P_out > 0) {
-    const int nb = p.chunk / 8;
-    for (int j = tid; j < nb; j += kT1) {
-      uint32_t m = 0u;
+__global__ void __launch_bounds__(kTF) topk_range_kernel(const TopkArgs a, const TopkPlan p) {
+  __shared__ uint32_t wmax[kTF / 32], wnmin[kTF / 32];
+  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c0 = blockIdx.x * kColsPerBlock;
+  const int ncol = row_cols(a, row);
+  const float *srow = a.scores + (size_t)row * a.ld;
+  uint32_t kmax = 0u, nmin = 0u;   // max key, max of ~key over present keys
 #pragma unroll
-      for (int q = 0; q < 8; ++q) m = max(m, keys[8 * j + q]);
-      bkeys[j] = m;
+  for (int j = 0; j < kColsPerBlock / kTF; ++j) {
+    const int col = c0 + j * kTF + tid;
+    const uint32_t key = col < ncol ? score_key(srow[col]) : 0u;
+    if (key) { kmax = max(kmax, key); nmin = max(nmin, ~key); }
+  }
+  kmax = __reduce_max_sync(0xffffffffu, kmax);
+  nmin = __reduce_max_sync(0xffffffffu, nmin);
+  if (lane == 0) { wmax[warp] = kmax; wnmin[warp] = nmin; }
+  __syncthreads();
+  if (tid == 0) {
+    for (int w = 1; w < kTF / 32; ++w) { kmax = max(kmax, wmax[w]); nmin = max(nmin, wnmin[w]); }
+    if (kmax) {
+      const Ws w = ws_view(a, p);
+      atomicMax(&w.range[2 * row], kmax);
+      atomicMax(&w.range[2 * row + 1], nmin);
     }
-    __syncthreads();
-    const size_t pb = ((size_t)row * p.nchunks + chunk) * p.p1;
-    radix_select<kT1>(bkeys, nb, p.p1, hist, &st, red);
-    const int pt = ordered_emit<kT1>(bkeys, nb, &st, [&](int pos, int j, uint32_t k) {
-      v.pkey[pb + pos] = k;
-      v.pblk[pb + pos] = c0 / 8 + j;
-    });
-    for (int i = pt + tid; i < p.p1; i += kT1) { v.pkey[pb + i] = 0u; v.pblk[pb + i] = -1; }
   }
 }
 
-__global__ void __launch_bounds__(kT2) topk_merge_kernel(const TopkArgs a, const TopkPlan p) {
-  extern __shared__ uint32_t sm2[];
-  __shared__ uint32_t hist[256];
+__global__ void __launch_bounds__(kTF) topk_hist_kernel(const TopkArgs a, const TopkPlan p) {
+  __shared__ uint32_t h[kBins], hb[kBins];
+  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int c0 = blockIdx.x * kColsPerBlock;
+  const int ncol = row_cols(a, row);
+  for (int i = tid; i < kBins; i += kTF) { h[i] = 0u; hb[i] = 0u; }
+  __syncthreads();
+  const float *srow = a.scores + (size_t)row * a.ld;
+  const Ws w = ws_view(a, p);
+  const Binning bn = row_binning(w, row);
+  float v[kColsPerBlock / kTF];
+#pragma unroll
+  for (int j = 0; j < kColsPerBlock / kTF; ++j) {
+    const int col = c0 + j * kTF + tid;
+    v[j] = col < ncol ? srow[col] : -INFINITY;
+  }
+#pragma unroll
+  for (int j = 0; j < kColsPerBlock / kTF; ++j) {
+    const uint32_t key = score_key(v[j]);
+    hist_add(h, key, bn, lane);
+    if (a.P_out > 0) {   // block of 8 consecutive columns = 8 consecutive lanes
+      uint32_t bk = key;
+      bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 1));
+      bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 2));
+      bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 4));
+      hist_add(hb, (lane & 7) == 0 ? bk : 0u, bn, lane);
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < kBins; i += kTF) {
+    if (h[i]) atomicAdd(&w.hist[(size_t)row * kBins + i], h[i]);
+    if (a.P_out > 0 && hb[i]) atomicAdd(&w.histb[(size_t)row * kBins + i], hb[i]);
+  }
+}
+
+__global__ void __launch_bounds__(kTF) topk_filter_kernel(const TopkArgs a, const TopkPlan p) {
+  __shared__ int sm_ws[40];
+  const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
+  const int c0 = blockIdx.x * kColsPerBlock;
+  const int ncol = row_cols(a, row);
+  const Ws w = ws_view(a, p);
+  const Binning bn = row_binning(w, row);
+  int T, above, Tb = -1, aboveb = 0;
+  find_threshold<kTF>(w.hist + (size_t)row * kBins, a.K, T, above, sm_ws);
+  if (a.P_out > 0) find_threshold<kTF>(w.histb + (size_t)row * kBins, a.P_out, Tb, aboveb, sm_ws);
+  (void)above;
+  (void)aboveb;
+  const float *srow = a.scores + (size_t)row * a.ld;
+  uint32_t *cnt = w.cnt + (size_t)row * 4;
+  float v[kColsPerBlock / kTF];
+#pragma unroll
+  for (int j = 0; j < kColsPerBlock / kTF; ++j) {
+    const int col = c0 + j * kTF + tid;
+    v[j] = col < ncol ? srow[col] : -INFINITY;
+  }
+#pragma unroll
+  for (int j = 0; j < kColsPerBlock / kTF; ++j) {
+    const int col = c0 + j * kTF + tid;
+    const uint32_t key = score_key(v[j]);
+    const int bin = key ? bn.digit(key) : -2;
+    warp_append(key && bin > T, col, &cnt[0], w.sel + (size_t)row * a.K, lane);
+    warp_append(key && bin == T, col, &cnt[1], w.cand + (size_t)row * a.n_cols, lane);
+    if (a.P_out > 0) {
+      uint32_t bk = key;
+      bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 1));
+      bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 2));
+      bk = max(bk, __shfl_xor_sync(0xffffffffu, bk, 4));
+      const bool lead = (lane & 7) == 0 && bk != 0u;
+      const int bbin = bk ? bn.digit(bk) : -2;
+      warp_append(lead && bbin > Tb, col >> 3, &cnt[2], w.selb + (size_t)row * a.P_out, lane);
+      warp_append(lead && bbin == Tb, col >> 3, &cnt[3], w.candb + (size_t)row * p.nb, lane);
+    }
+  }
+}
+
+// One part (entries or blocks) of the select kernel: out[0..K) = the K best
+// columns in ascending order (-1 padded), from the selected list, the
+// candidate list and the key of each candidate column.  The chosen columns
+// are marked in a bitmap of the row's columns; a prefix popcount over the
+// bitmap gives each one its output position (no sort).
+template <class KeyOfCol>
+__device__ void select_part(const uint32_t *hist, const int32_t *sel, const int32_t *cand, uint32_t n_cand,
+                            int K, int n_cols, KeyOfCol key_of, const int32_t *pool_blocks, int32_t *out,
+                            uint32_t *cand_key, int32_t *cand_col, uint32_t *bitmap, uint32_t *hist256,
+                            SelState *st, int *red) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nwords = (n_cols + 31) >> 5;
+  for (int i = tid; i < nwords; i += kTS) bitmap[i] = 0u;
+  int T, above;
+  find_threshold<kTS>(hist, K, T, above, red);   // (synchronises: bitmap cleared)
+  for (int i = tid; i < above; i += kTS) {
+    const int32_t c = sel[i];
+    atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+  }
+  const int need = T < 0 ? 0 : K - above;
+  if (need > 0) {
+    const int n = (int)n_cand;
+    const bool staged = n <= kSmemCands;
+    if (staged) {
+      for (int i = tid; i < n; i += kTS) {
+        const int32_t c = cand[i];
+        cand_col[i] = c;
+        cand_key[i] = key_of(c);
+      }
+      __syncthreads();
+    }
+    auto kf = [&](int i) -> uint32_t { return staged ? cand_key[i] : key_of(cand[i]); };
+    auto cf = [&](int i) -> int32_t { return staged ? cand_col[i] : cand[i]; };
+    radix_select<kTS>(kf, n, need, hist256, st, red);
+    const uint32_t thr = st->thr;
+    const int take_eq = st->take_eq;
+    // ties at thr: the take_eq smallest columns (skipped when all ties fit)
+    int n_eq = 0;
+    for (int i = tid; i < n; i += kTS) n_eq += kf(i) == thr;
+    n_eq = __reduce_add_sync(0xffffffffu, (unsigned)n_eq);
+    if (lane == 0) red[warp] = n_eq;
+    __syncthreads();
+    n_eq = 0;
+#pragma unroll
+    for (int w = 0; w < kTS / 32; ++w) n_eq += red[w];
+    __syncthreads();
+    uint32_t thr2 = 0u;
+    auto tf = [&](int i) -> uint32_t { return kf(i) == thr ? 0xFFFFFFFFu - (uint32_t)cf(i) : 0u; };
+    if (n_eq > take_eq) {
+      radix_select<kTS>(tf, n, take_eq, hist256, st, red);
+      thr2 = st->thr;
+    }
+    for (int i = tid; i < n; i += kTS) {
+      const uint32_t k = kf(i);
+      if (k > thr || (k == thr && tf(i) >= thr2)) {
+        const int32_t c = cf(i);
+        atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+      }
+    }
+  }
+  __syncthreads();
+  // exclusive prefix popcount over the bitmap words (each thread a run of words)
+  const int per = (nwords + kTS - 1) / kTS;
+  const int w0 = tid * per, w1 = min(w0 + per, nwords);
+  int mine = 0;
+  for (int wi = w0; wi < w1; ++wi) mine += __popc(bitmap[wi]);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) red[warp] = incl;
+  __syncthreads();
+  int before = incl - mine, total = 0;
+#pragma unroll
+  for (int w = 0; w < kTS / 32; ++w) {
+    const int v = red[w];
+    if (w < warp) before += v;
+    total += v;
+  }
+  for (int wi = w0; wi < w1; ++wi) {
+    uint32_t bits = bitmap[wi];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int c = wi * 32 + bpos;
+      if (before < K) out[before] = pool_blocks ? pool_blocks[c >> 3] * 8 + (c & 7) : c;
+      ++before;
+    }
+  }
+  for (int i = total + tid; i < K; i += kTS) out[i] = -1;
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kTS) topk_select_kernel(const TopkArgs a, const TopkPlan p) {
+  extern __shared__ uint32_t sm3[];
+  __shared__ uint32_t hist256[256];
   __shared__ SelState st;
-  __shared__ int red[32];
-  const int row = blockIdx.x, tid = threadIdx.x;
-  WsView v = ws_view(a.ws, a.rows, p);
+  __shared__ int red[40];
+  uint32_t *cand_key = sm3;                                           // [kSmemCands]
+  int32_t *cand_col = reinterpret_cast<int32_t *>(sm3 + kSmemCands);  // [kSmemCands]
+  uint32_t *bitmap = sm3 + 2 * kSmemCands;                            // [n_cols / 32]
+  const int row = blockIdx.x;
+  const Ws w = ws_view(a, p);
+  const float *srow = a.scores + (size_t)row * a.ld;
+  const int ncol = row_cols(a, row);
+  const uint32_t *cnt = w.cnt + (size_t)row * 4;
+  const int32_t *pb = a.pool_blocks ? a.pool_blocks + (size_t)row * (a.n_cols / 8) : nullptr;
 
-  // ---- entries
-  {
-    const int n = p.nchunks * p.k1;
-    const size_t base = (size_t)row * n;
-    const uint32_t *keys = v.ckey + base;
-    const int32_t *cols = v.ccol + base;
-    if (n <= kMergeSmemCands) {
-      uint32_t *k_s = sm2;
-      int32_t *c_s = reinterpret_cast<int32_t *>(sm2 + n);
-      for (int i = tid; i < n; i += kT2) { k_s[i] = keys[i]; c_s[i] = cols[i]; }
-      __syncthreads();
-      keys = k_s;
-      cols = c_s;
-    }
-    radix_select<kT2>(keys, n, a.K, hist, &st, red);
-    int32_t *out = a.out_idx + (size_t)row * a.K;
-    const int32_t *pb = a.pool_blocks ? a.pool_blocks + (size_t)row * (a.n_cols / 8) : nullptr;
-    const int taken = ordered_emit<kT2>(keys, n, &st, [&](int pos, int i, uint32_t) {
-      const int c = cols[i];
-      out[pos] = pb ? pb[c >> 3] * 8 + (c & 7) : c;
-    });
-    for (int i = taken + tid; i < a.K; i += kT2) out[i] = -1;
-    __syncthreads();
-  }
-  // ---- pool
+  auto entry_key = [&](int32_t c) -> uint32_t { return c < ncol ? score_key(srow[c]) : 0u; };
+  select_part(w.hist + (size_t)row * kBins, w.sel + (size_t)row * a.K, w.cand + (size_t)row * a.n_cols, cnt[1],
+              a.K, a.n_cols, entry_key, pb, a.out_idx + (size_t)row * a.K, cand_key, cand_col, bitmap, hist256,
+              &st, red);
   if (a.P_out > 0) {
-    const int n = p.nchunks * p.p1;
-    const size_t base = (size_t)row * n;
-    const uint32_t *keys = v.pkey + base;
-    const int32_t *blks = v.pblk + base;
-    if (n <= kMergeSmemCands) {
-      uint32_t *k_s = sm2;
-      int32_t *b_s = reinterpret_cast<int32_t *>(sm2 + n);
-      for (int i = tid; i < n; i += kT2) { k_s[i] = keys[i]; b_s[i] = blks[i]; }
-      __syncthreads();
-      keys = k_s;
-      blks = b_s;
-    }
-    radix_select<kT2>(keys, n, a.P_out, hist, &st, red);
-    int32_t *out = a.out_pool + (size_t)row * a.P_out;
-    const int taken = ordered_emit<kT2>(keys, n, &st, [&](int pos, int i, uint32_t) { out[pos] = blks[i]; });
-    for (int i = taken + tid; i < a.P_out; i += kT2) out[i] = -1;
+    auto block_key = [&](int32_t blk) -> uint32_t {
+      uint32_t m = 0u;
+      for (int q = 0; q < 8; ++q) {
+        const int c = blk * 8 + q;
+        if (c < ncol) m = max(m, score_key(srow[c]));
+      }
+      return m;
+    };
+    select_part(w.histb + (size_t)row * kBins, w.selb + (size_t)row * a.P_out, w.candb + (size_t)row * p.nb,
+                cnt[3], a.P_out, p.nb, block_key, nullptr, a.out_pool + (size_t)row * a.P_out, cand_key, cand_col,
+                bitmap, hist256, &st, red);
   }
 }
+
+size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
 }  // namespace
 
 TopkPlan plan_topk(int rows, int n_cols, int K, int P_out) {
-  TopkPlan p;
-  int chunk = 4096;
-  auto kk = [&](int c) { return K < c ? K : c; };
-  while (chunk < 32768 && (size_t)((n_cols + chunk - 1) / chunk) * kk(chunk) > 8192) chunk *= 2;
-  p.chunk = chunk;
-  p.nchunks = n_cols > 0 ? (n_cols + chunk - 1) / chunk : 1;
-  p.k1 = kk(chunk);
-  p.p1 = P_out > 0 ? (P_out < chunk / 8 ? P_out : chunk / 8) : 0;
-  p.bytes = (size_t)rows * p.nchunks * ((size_t)p.k1 + p.p1) * 8;
+  TopkPlan p{};
+  if (topk_cluster_fits(n_cols)) return p;   // the cluster kernel needs no workspace
+  p.nchunks = n_cols > 0 ? (n_cols + kColsPerBlock - 1) / kColsPerBlock : 1;
+  p.nb = (n_cols + 7) / 8;
+  const size_t R = (size_t)(rows > 0 ? rows : 0);
+  size_t o = 0;
+  p.off_hist = o;
+  o += R * kBins * 4;
+  p.off_histb = o;
+  if (P_out > 0) o += R * kBins * 4;
+  p.off_cnt = o;
+  o += R * 4 * 4;
+  p.off_range = o;
+  o += R * 2 * 4;
+  p.zero_bytes = o;
+  o = align16(o);
+  p.off_sel = o;
+  o = align16(o + R * K * 4);
+  p.off_cand = o;
+  o = align16(o + R * (size_t)n_cols * 4);
+  p.off_selb = o;
+  if (P_out > 0) o = align16(o + R * P_out * 4);
+  p.off_candb = o;
+  if (P_out > 0) o = align16(o + R * (size_t)p.nb * 4);
+  p.bytes = o;
   return p;
 }
 
 cudaError_t launch_topk(const TopkArgs &a, const TopkPlan &p, cudaStream_t s) {
-  const size_t sm1 = sizeof(uint32_t) * ((size_t)p.chunk + p.chunk / 8);
-  cudaError_t e = cudaFuncSetAttribute(topk_chunk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm1);
+  if (topk_cluster_fits(a.n_cols)) return launch_topk_cluster(a, s);
+  cudaError_t e = cudaMemsetAsync(a.ws, 0, p.zero_bytes, s);
   if (e != cudaSuccess) return e;
-  topk_chunk_kernel<<<dim3(p.nchunks, a.rows), kT1, sm1, s>>>(a, p);
-  e = cudaGetLastError();
+  if (a.n_cols > 0) {
+    const dim3 grid(p.nchunks, a.rows);
+    topk_range_kernel<<<grid, kTF, 0, s>>>(a, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    topk_hist_kernel<<<grid, kTF, 0, s>>>(a, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    topk_filter_kernel<<<grid, kTF, 0, s>>>(a, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // candidates staged + a bitmap of the row's columns (bits)
+  const size_t sm = sizeof(uint32_t) * (2 * (size_t)kSmemCands + ((size_t)a.n_cols + 31) / 32 + 1);
+  if (sm > 227 * 1024) return cudaErrorInvalidValue;
+  e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
   if (e != cudaSuccess) return e;
-  // shared memory holds whichever candidate list fits (the other is read from
-  // the workspace directly)
-  const int nk = p.nchunks * p.k1, np = p.nchunks * p.p1;
-  const int sk = nk <= kMergeSmemCands ? nk : 0, sp = np <= kMergeSmemCands ? np : 0;
-  const size_t sm2 = (size_t)(sk > sp ? sk : sp) * 8;
-  e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm2);
-  if (e != cudaSuccess) return e;
-  topk_merge_kernel<<<a.rows, kT2, sm2, s>>>(a, p);
+  topk_select_kernel<<<a.rows, kTS, sm, s>>>(a, p);
   return cudaGetLastError();
 }
 

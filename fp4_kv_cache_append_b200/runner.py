@@ -101,6 +101,7 @@ class Step:
         ws_at = C.csa2_attn_workspace_size(B, self.T_q, wl.H, D, wl.K, wl.window)
         self.ws_topk = C.workspace(max(ws_full, ws_re), dev)
         self.ws_attn = C.workspace(ws_at, dev)
+        self.ws_index = C.workspace(C.csa2_index_workspace_size(self.rows, wl.dI), dev)
 
     # ------------------------------------------------------------------ set-up (untimed)
 
@@ -136,7 +137,8 @@ class Step:
         m = self.main[0]
         # the step's token must be in the cache for the scan: append it first
         C.csa2_append_quant(m, self.kv_new, self.gate_new, self.w_ik, None, None, self.pos0, wl.T)
-        C.csa2_index_full(m, self.q_idx[POOL_LAYER], self.w[POOL_LAYER], self.q_pos, self.scores, self.n_valid)
+        C.csa2_index_full(m, self.q_idx[POOL_LAYER], self.w[POOL_LAYER], self.q_pos, self.scores, self.n_valid,
+                          ws=self.ws_index)
         C.csa2_topk(self.scores, self.cap, wl.K, self.idx, n_valid=self.n_valid, P_out=wl.P, out_pool=self.pool,
                     ws=self.ws_topk)
         self.group_pool = self.pool.clone()
@@ -170,7 +172,7 @@ class Step:
                 timed("append", lambda: C.csa2_append_quant(main, self.kv_new, self.gate_new, self.w_ik, swa[l],
                                                             self.kv_swa_new[l], self.pos0, wl.T))
                 timed("index_full", lambda: C.csa2_index_full(main, self.q_idx[l], self.w[l], self.q_pos,
-                                                              self.scores, self.n_valid))
+                                                              self.scores, self.n_valid, ws=self.ws_index))
                 timed("topk", lambda: C.csa2_topk(self.scores, self.cap, wl.K, self.idx, n_valid=self.n_valid,
                                                   P_out=wl.P, out_pool=self.pool if wl.P else None,
                                                   ws=self.ws_topk))
@@ -179,7 +181,7 @@ class Step:
                                                             self.pos0, wl.T))
                 pool = self.group_pool if wl.mode == "group" else self.pool
                 timed("index_reindex", lambda: C.csa2_index_reindex(main, self.q_idx[l], self.w[l], self.q_pos,
-                                                                    pool, self.pool_scores))
+                                                                    pool, self.pool_scores, ws=self.ws_index))
                 timed("topk", lambda: C.csa2_topk(self.pool_scores, wl.P * 8, wl.K, self.idx, pool_blocks=pool,
                                                   ws=self.ws_topk))
             else:  # reuse: own window rows and query, inherited KV and indices

@@ -135,12 +135,15 @@ CSA2_API csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16
  *         n_vis = min(n_entries[b], floor((q_pos+1)/m)); columns >= n_vis are
  *         not written
  *  n_valid [B*T_q] i32 out (may be NULL): n_vis of each row
+ *  ws, ws_bytes: workspace of csa2_index_workspace_size(B*T_q, d_I) bytes
+ *         (holds each row's prepared FP8 query)
  * Supported: 1 <= H_I <= 64, ld >= cap.
  */
 CSA2_API csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx,
                             const float *w, const int32_t *q_pos, int T_q, int H_I,
                             float *scores, int64_t ld, int32_t *n_valid,
-                            csa2_stream_t stream);
+                            void *ws, size_t ws_bytes, csa2_stream_t stream);
+CSA2_API size_t csa2_index_workspace_size(int rows, int d_I);
 
 /*
  * 3. Reindex scoring  [jaehun "2) CSA2": later Reindex layers rescore only the
@@ -149,12 +152,13 @@ CSA2_API csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t
  *  pool_blocks [B*T_q][P] i32 block ids (block g = entries 8g..8g+7), -1 = none
  *  pool_scores [B*T_q][P*8] f32 out: column c scores entry pool[c/8]*8 + c%8,
  *              -inf when the block is -1 or the entry is not visible
+ *  ws, ws_bytes: as for csa2_index_full
  * Supported: P a multiple of 16, 16 <= P <= 4096.
  */
 CSA2_API csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_idx,
                                const float *w, const int32_t *q_pos, int T_q, int H_I,
                                const int32_t *pool_blocks, int P, float *pool_scores,
-                               csa2_stream_t stream);
+                               void *ws, size_t ws_bytes, csa2_stream_t stream);
 
 /*
  * 4. Top-K selection and the hierarchical candidate pool  [jaehun "2) CSA2":
@@ -170,7 +174,7 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint1
  *         blocks of 8 columns with the largest block maximum (ties -> smaller
  *         block), ascending, -1 padded
  *  ws, ws_bytes: workspace of csa2_topk_workspace_size(rows, n_cols, K, P_out)
- * Supported: 1 <= K <= 2048, 0 <= P_out <= 4096, n_cols <= 2^24.
+ * Supported: 1 <= K <= 2048, 0 <= P_out <= 4096, n_cols <= 2^20.
  */
 CSA2_API csa2_status csa2_topk(const float *scores, int rows, int64_t ld, int n_cols,
                       const int32_t *n_valid, const int32_t *pool_blocks, int K,

@@ -45,21 +45,22 @@ def test_host_validation_rejects_bad_arguments_without_a_gpu():
     # no main and no window cache
     assert L.csa2_append_quant(None, p, None, p, None, p, p, 1, None) == 1
     # misaligned pointer
-    assert L.csa2_index_full(ctypes.byref(d), ctypes.c_void_p(18), p, p, 1, 64, p, 128, None, None) == 1
+    assert L.csa2_index_full(ctypes.byref(d), ctypes.c_void_p(18), p, p, 1, 64, p, 128, None, p, 1 << 20, None) == 1
     # unsupported D
     bad = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 1, 128, 384, 128, 1)
-    assert L.csa2_index_full(ctypes.byref(bad), p, p, p, 1, 64, p, 128, None, None) == 2
+    assert L.csa2_index_full(ctypes.byref(bad), p, p, p, 1, 64, p, 128, None, p, 1 << 20, None) == 2
     # cap not a multiple of 128
     bad = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 1, 100, 512, 128, 1)
-    assert L.csa2_index_full(ctypes.byref(bad), p, p, p, 1, 64, p, 128, None, None) == 2
+    assert L.csa2_index_full(ctypes.byref(bad), p, p, p, 1, 64, p, 128, None, p, 1 << 20, None) == 2
     # H_I out of range
-    assert L.csa2_index_full(ctypes.byref(d), p, p, p, 1, 65, p, 128, None, None) == 2
+    assert L.csa2_index_full(ctypes.byref(d), p, p, p, 1, 65, p, 128, None, p, 1 << 20, None) == 2
     # ld < cap
-    assert L.csa2_index_full(ctypes.byref(d), p, p, p, 1, 64, p, 64, None, None) in (1, 3)
+    assert L.csa2_index_full(ctypes.byref(d), p, p, p, 1, 64, p, 64, None, p, 1 << 20, None) in (1, 3, 5)
     # K out of range, P not a multiple of 16, workspace too small
     assert L.csa2_topk(p, 1, 128, 128, None, None, 0, p, 0, None, p, 1 << 20, None) == 2
-    assert L.csa2_index_reindex(ctypes.byref(d), p, p, p, 1, 64, p, 20, p, None) in (2, 3)
-    assert L.csa2_topk(p, 1, 128, 128, None, None, 64, p, 0, None, p, 0, None) == 5
+    assert L.csa2_index_reindex(ctypes.byref(d), p, p, p, 1, 64, p, 20, p, p, 1 << 20, None) in (2, 3, 5)
+    # rows over 65,536 columns need a workspace (shorter rows need none)
+    assert L.csa2_topk(p, 1, 100000, 100000, None, None, 64, p, 0, None, p, 0, None) == 5
     assert "workspace" in L.csa2_last_error().decode()
     # m = 2 without pending buffers
     m2 = C.MainCacheDesc(16, 16, 16, 16, 16, None, None, 1, 128, 512, 128, 2)
@@ -67,5 +68,6 @@ def test_host_validation_rejects_bad_arguments_without_a_gpu():
 
 
 def test_workspace_sizes_are_pure_host_functions():
-    assert C.csa2_topk_workspace_size(8, 65536, 512, 2048) > 0
+    assert C.csa2_topk_workspace_size(8, 100000, 512, 2048) > 0
+    assert C.csa2_topk_workspace_size(8, 65536, 512, 2048) == 0   # single-launch cluster path
     assert C.csa2_topk_workspace_size(0, 65536, 512, 2048) == 0
