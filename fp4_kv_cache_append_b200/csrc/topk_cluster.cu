@@ -5,21 +5,27 @@
 //   x 8 positions (paper sec. 2.3.2, 4.2.1, Fig. 5).
 // Same contract as the multi-kernel path in topk.cu (score descending, ties
 // -> smaller column, non-finite = absent, ascending output, -1 padding,
-// block score = max of its present columns), without a workspace:
-//   * block r of the cluster owns columns [r*S, (r+1)*S); each thread keeps
-//     32 consecutive columns' order-preserving keys (and their 4 block
-//     maxima) in registers;
-//   * the cluster-wide key range comes from every block's min/max read
-//     through distributed shared memory;
-//   * rounds of a 2048-bin histogram over the remaining key range, summed
-//     across the cluster (block r reduces bins [256r, 256r+256)), narrow
-//     the range to the bin holding the K-th key until that bin is either
-//     taken whole or is a single key value (at most 3 rounds for 32-bit keys);
-//   * ties at that value are shared out in column order from per-block
-//     counts, and every block writes its chosen columns, in order, at the
-//     offset given by the counts of the blocks before it.
-// Entries (K) and blocks (P_out) are selected together in the same rounds.
-// Only cluster barriers are used; no block waits on a flag.
+// block score = max of its present columns), without a workspace.
+//
+// Block r of the cluster owns columns [8192r, 8192(r+1)); thread t keeps the
+// order-preserving keys of columns 8t..8t+7 of that slice in registers, and
+// their maximum, the key of one 8-column pool block.  The K-th largest key is
+// found by levels of 512-bin histograms:
+//   * level 0 bins by VALUE, linearly between the row's smallest and largest
+//     score, so scores concentrated in a few binades still spread over many
+//     bins; the bin holding the K-th key is then turned into an exact key
+//     interval by a 32-way search over keys (bins are monotone in the key);
+//   * further levels bin by key bits inside that interval;
+//   * a bin holding the K-th key with at most 256 keys is resolved exactly:
+//     its keys are collected in block 0 and ranked (score desc, column asc);
+//   * a single-valued bin with more keys shares its ties out in column order.
+// Per level the block histograms are pushed into the owning block's slice
+// (block r owns bins [64r, 64r+64)) with distributed-shared-memory atomics
+// and read back after ONE cluster barrier; slices rotate over 3 buffers so no
+// second barrier is needed before they are reused.  The two selections
+// (entries, pool blocks) run side by side in the two halves of the block.
+// Loops stay rolled and the state lives in shared memory: the kernel runs
+// once per row, so the code it fetches is as much a cost as what it executes.
 #include <cooperative_groups.h>
 
 #include "common.cuh"
@@ -31,64 +37,120 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kCl = 8;        // blocks per row
-constexpr int kT = 256;       // threads per block
-constexpr int kN = 32;        // columns per thread
-constexpr int kNB = kN / 8;   // blocks of 8 columns per thread
-constexpr int kBins = 2048;
+constexpr int kCl = 8;            // blocks per row
+constexpr int kT = 1024;          // threads per block
+constexpr int kN = 8;             // columns per thread (= one pool block)
+constexpr int kSpan = kT * kN;    // columns per block
+constexpr int kBins = 512;        // bins per selection (kT = 2 * kBins)
+constexpr int kSeg = kBins / kCl; // bins owned by one block
+constexpr int kCand = 256;        // largest bin resolved by exact ranking
+
+static_assert(kT == 2 * kBins, "one thread per (selection, bin)");
 
 __device__ __forceinline__ uint32_t ckey(float f) {
-  if (!isfinite(f)) return 0u;
-  if (f == 0.0f) f = 0.0f;
+  if (!isfinite(f)) return 0u;   // absent
+  if (f == 0.0f) f = 0.0f;       // -0 == +0
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
-
-// Exclusive scan of one int per thread over the block; returns the total.
-__device__ __forceinline__ int block_excl_scan(int v, int &excl, int *red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int incl = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, incl, o);
-    if (lane >= o) incl += y;
-  }
-  __syncthreads();
-  if (lane == 31) red[warp] = incl;
-  __syncthreads();
-  int before = 0, total = 0;
-#pragma unroll
-  for (int w = 0; w < kT / 32; ++w) {
-    if (w < warp) before += red[w];
-    total += red[w];
-  }
-  excl = before + incl - v;
-  return total;
+__device__ __forceinline__ float kval(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-struct Sel {          // state of one selection (entries or blocks), identical in every block
-  uint32_t lo, hi;    // key range still undecided
-  int need;           // keys still to take inside [lo, hi]
-  int shift;
-  bool done;
-  uint32_t thr_gt;    // final: keys > thr_gt are taken ...
-  uint32_t thr_eq;    // ... and `take_eq` of the keys == thr_eq (in column order)
+enum : int { kActive = 0, kCollect = 1, kDone = 2 };
+
+// State of one selection, kept in shared memory and written by one thread.
+struct Sel {
+  int state;
+  bool vs;            // the current level bins by value (level 0)
+  float v_lo, inv;    // value bin = clamp((v - v_lo) * inv)
+  uint32_t g_lo, g_hi;
+  uint32_t lo, hi;    // key interval of the current level's region
+  int shift;          // key bin = (key - lo) >> shift
+  int need;           // keys still to take inside the region
+  int cnt;            // keys in the region (when collecting)
+  // final rule: key > kthr, or key == kthr and (cmode ? column <= cthr : tie rank < take_eq)
+  uint32_t kthr;
+  int cthr;
+  bool cmode;
   int take_eq;
 };
 
+__device__ __forceinline__ int vbin(float v_lo, float inv, uint32_t k) {
+  const int b = (int)((kval(k) - v_lo) * inv);
+  return b < 0 ? 0 : (b > kBins - 1 ? kBins - 1 : b);
+}
+__device__ __forceinline__ int key_shift(uint32_t lo, uint32_t hi) {
+  const uint32_t span = hi - lo;
+  return span >= (uint32_t)kBins ? (32 - __clz(span)) - 9 : 0;
+}
+
+// Smallest key in (lo, hi] whose value bin is >= T, given vbin(lo) < T <= vbin(hi);
+// one 32-way step per iteration, every lane of the warp takes part.
+__device__ uint32_t first_key_of_bin(float v_lo, float inv, uint32_t lo, uint32_t hi, int T, int lane) {
+#pragma unroll 1
+  while (hi - lo > 1u) {
+    const uint32_t step = (uint32_t)(((uint64_t)(hi - lo) + 31u) >> 5);
+    const uint64_t p = (uint64_t)lo + (uint64_t)step * (uint32_t)(lane + 1);
+    const bool ge = p >= hi || vbin(v_lo, inv, (uint32_t)p) >= T;
+    const int j = __ffs(__ballot_sync(0xffffffffu, ge)) - 1;   // lane 31 always probes >= hi
+    const uint64_t pj = __shfl_sync(0xffffffffu, p, j);
+    const uint64_t pp = __shfl_sync(0xffffffffu, p, j > 0 ? j - 1 : 0);
+    const uint32_t nhi = pj >= hi ? hi : (uint32_t)pj;
+    lo = j > 0 ? (uint32_t)pp : lo;
+    hi = nhi;
+  }
+  return hi;
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_incl_scan(T v, int lane) {
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const T y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  return v;
+}
+
+// Exclusive block scan; afterwards red[w] holds the inclusive sum of warps 0..w
+// (valid until the next scan).
+template <typename T>
+__device__ __forceinline__ T block_scan(T v, T *red, int lane, int warp) {
+  const T incl = warp_incl_scan(v, lane);
+  __syncthreads();   // the previous scan's readers of red are done
+  if (lane == 31) red[warp] = incl;
+  __syncthreads();
+  if (warp == 0) red[lane] = warp_incl_scan(red[lane], lane);
+  __syncthreads();
+  return (warp ? red[warp - 1] : T(0)) + incl - v;
+}
+
 struct Shared {
-  uint32_t hist[2][kBins];
-  uint32_t hsum[2][kBins / kCl];
-  uint32_t stat[2][3];       // this block: min, max, count of present keys
-  int cnt[2][2];             // this block: ties, chosen
-  int red[kT / 32];
-  uint32_t g[2][3];          // cluster: min, max, count
-  int th[2][3];              // threshold bin, keys above it in the range, keys in it
+  uint32_t hist[2][kBins];        // this block's histogram of the current level
+  uint32_t hsum[3][2][kSeg];      // cluster histogram, the bins this block owns
+  uint2 cand[2][kCand];           // collected (key, column) pairs (block 0's are used)
+  uint2 loc[2][kCand];            // local copy of block 0's pairs
+  unsigned long long red[32];
+  uint32_t wst[2][3][32];         // per-warp min, max, count
+  uint32_t stat[2][3];            // this block: min key, max key, present count
+  uint32_t cand_n[2];
+  int cnt[4];                     // this block: ties / strict (entries), ties / strict (blocks)
+  int th[2][3];                   // threshold bin, keys above it, keys in it
+  int base[2], allow[2], total[2];
+  Sel sel[2];
 };
+
+__device__ __forceinline__ void cluster_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
 
 }  // namespace
 
-__global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT) topk_cluster_kernel(const TopkArgs a, int S) {
+__global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluster_kernel(const TopkArgs a) {
   __shared__ Shared sh;
   cg::cluster_group cl = cg::this_cluster();
   const int r = (int)cl.block_rank();
@@ -98,296 +160,345 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT) topk_cluster_k
     const int v = a.n_valid[row];
     if (v < ncol) ncol = v < 0 ? 0 : v;
   }
-  const int npt = S / kT;                   // columns per thread (a multiple of 8, <= kN)
-  const int c0 = r * S + tid * npt;         // this thread's first column
-  const float *srow = a.scores + (size_t)row * a.ld;
+  const int c0 = r * kSpan + tid * kN;   // this thread's first column
+  const int blk = c0 >> 3;               // its pool block
   const int nsel = a.P_out > 0 ? 2 : 1;
-  const int Kt[2] = {a.K, a.P_out};
 
-  // ---- keys in registers (column order within the thread)
-  uint32_t key[kN], bkey[kNB];
-  // c0 is a multiple of 8, so 16-byte loads are aligned when the row is
-  const bool vec = (a.ld & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0;
-#pragma unroll
-  for (int k = 0; k < kN; k += 4) {
-    const int col = c0 + k;
-    if (vec && k < npt && col + 4 <= ncol) {
-      const float4 v = __ldcs(reinterpret_cast<const float4 *>(srow + col));
-      key[k] = ckey(v.x);
-      key[k + 1] = ckey(v.y);
-      key[k + 2] = ckey(v.z);
-      key[k + 3] = ckey(v.w);
+  // ---- keys (both 16-byte loads are issued before either is used)
+  uint32_t key[kN];
+  {
+    const float *src = a.scores + (size_t)row * a.ld + c0;
+    float v[kN];
+    if (c0 + kN <= ncol && (a.ld & 3) == 0 && (reinterpret_cast<uintptr_t>(a.scores) & 15u) == 0) {
+      const float4 x = __ldcs(reinterpret_cast<const float4 *>(src));
+      const float4 y = __ldcs(reinterpret_cast<const float4 *>(src) + 1);
+      v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w; v[4] = y.x; v[5] = y.y; v[6] = y.z; v[7] = y.w;
     } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) key[k + j] = (k + j < npt && col + j < ncol) ? ckey(srow[col + j]) : 0u;
+      for (int k = 0; k < kN; ++k) v[k] = c0 + k < ncol ? src[k] : __int_as_float(0x7fc00000);
+    }
+#pragma unroll
+    for (int k = 0; k < kN; ++k) key[k] = ckey(v[k]);
+  }
+  uint32_t bkey = 0u;
+#pragma unroll
+  for (int k = 0; k < kN; ++k) bkey = max(bkey, key[k]);
+
+  // ---- zero the histograms, the round-0 slices and the collect counters
+  (&sh.hist[0][0])[tid] = 0u;
+  if (tid < 2 * kSeg) (&sh.hsum[0][0][0])[tid] = 0u;
+  if (tid < 2) sh.cand_n[tid] = 0u;
+
+  // ---- key range and count: warp, block, cluster
+  {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u, c = 0u;
+#pragma unroll
+    for (int k = 0; k < kN; ++k)
+      if (key[k]) { mn = min(mn, key[k]); mx = max(mx, key[k]); ++c; }
+    const uint32_t bmn = bkey ? bkey : 0xFFFFFFFFu, bc = bkey ? 1u : 0u;
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    c = __reduce_add_sync(0xffffffffu, c);
+    const uint32_t bmn2 = __reduce_min_sync(0xffffffffu, bmn);
+    const uint32_t bc2 = __reduce_add_sync(0xffffffffu, bc);
+    if (lane == 0) {
+      sh.wst[0][0][warp] = mn; sh.wst[0][1][warp] = mx; sh.wst[0][2][warp] = c;
+      sh.wst[1][0][warp] = bmn2; sh.wst[1][1][warp] = mx; sh.wst[1][2][warp] = bc2;
     }
   }
-#pragma unroll
-  for (int g = 0; g < kNB; ++g) {
-    uint32_t m = 0u;
-#pragma unroll
-    for (int k = 0; k < 8; ++k) m = max(m, key[8 * g + k]);
-    bkey[g] = m;
+  __syncthreads();
+  if (warp < 2) {   // warp s combines selection s
+    const uint32_t mn = __reduce_min_sync(0xffffffffu, sh.wst[warp][0][lane]);
+    const uint32_t mx = __reduce_max_sync(0xffffffffu, sh.wst[warp][1][lane]);
+    const uint32_t c = __reduce_add_sync(0xffffffffu, sh.wst[warp][2][lane]);
+    if (lane == 0) { sh.stat[warp][0] = mn; sh.stat[warp][1] = mx; sh.stat[warp][2] = c; }
   }
-
-  // ---- local and cluster-wide key range and count
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    if (s >= nsel) break;
+  cl.sync();
+  if (warp < 2) {
+    const int s = warp;
     uint32_t mn = 0xFFFFFFFFu, mx = 0u, c = 0u;
-    if (s == 0) {
-#pragma unroll
-      for (int k = 0; k < kN; ++k) if (key[k]) { mn = min(mn, key[k]); mx = max(mx, key[k]); ++c; }
-    } else {
-#pragma unroll
-      for (int g = 0; g < kNB; ++g) if (bkey[g]) { mn = min(mn, bkey[g]); mx = max(mx, bkey[g]); ++c; }
+    if (lane < kCl) {
+      const uint32_t *rs = cl.map_shared_rank(&sh.stat[s][0], lane);
+      mn = rs[0];
+      mx = rs[1];
+      c = rs[2];
     }
     mn = __reduce_min_sync(0xffffffffu, mn);
     mx = __reduce_max_sync(0xffffffffu, mx);
     c = __reduce_add_sync(0xffffffffu, c);
-    if (lane == 0) { sh.hsum[s][warp] = mn; sh.hsum[s][8 + warp] = mx; sh.hsum[s][16 + warp] = c; }
-  }
-  __syncthreads();
-  if (tid < nsel) {
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u, c = 0u;
-    for (int w = 0; w < kT / 32; ++w) {
-      mn = min(mn, sh.hsum[tid][w]);
-      mx = max(mx, sh.hsum[tid][8 + w]);
-      c += sh.hsum[tid][16 + w];
-    }
-    sh.stat[tid][0] = mn;
-    sh.stat[tid][1] = mx;
-    sh.stat[tid][2] = c;
-  }
-  cl.sync();
-  if (warp == 0) {
-    for (int s = 0; s < nsel; ++s) {
-      uint32_t mn = 0xFFFFFFFFu, mx = 0u, c = 0u;
-      if (lane < kCl) {
-        const uint32_t *rs = cl.map_shared_rank(&sh.stat[s][0], lane);
-        mn = rs[0];
-        mx = rs[1];
-        c = rs[2];
+    if (lane == 0) {
+      Sel &l = sh.sel[s];
+      const int Kt = s == 0 ? a.K : a.P_out;
+      l.g_lo = l.lo = mn;
+      l.g_hi = l.hi = mx;
+      l.need = Kt;
+      l.cnt = 0;
+      l.kthr = 0u;   // with cmode and cthr = -1: every present key
+      l.cthr = -1;
+      l.cmode = true;
+      l.take_eq = 0;
+      l.vs = false;
+      l.v_lo = 0.f;
+      l.inv = 0.f;
+      l.shift = 0;
+      if (s >= nsel || (int)c <= Kt) {
+        l.state = kDone;
+      } else {
+        l.state = kActive;
+        const float vlo = kval(mn), vhi = kval(mx);
+        const float span = vhi - vlo;
+        const float inv = (float)kBins / span;
+        if (span > 0.f && isfinite(span) && isfinite(inv)) {
+          l.vs = true;
+          l.v_lo = vlo;
+          l.inv = inv;
+        } else {
+          l.shift = key_shift(mn, mx);
+        }
       }
-      mn = __reduce_min_sync(0xffffffffu, mn);
-      mx = __reduce_max_sync(0xffffffffu, mx);
-      c = __reduce_add_sync(0xffffffffu, c);
-      if (lane == 0) { sh.g[s][0] = mn; sh.g[s][1] = mx; sh.g[s][2] = c; }
     }
   }
   __syncthreads();
 
-  Sel sel[2];
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    sel[s].lo = sh.g[s][0];
-    sel[s].hi = sh.g[s][1];
-    sel[s].need = Kt[s];
-    sel[s].shift = 0;
-    sel[s].take_eq = 0;
-    sel[s].thr_eq = 0u;
-    sel[s].thr_gt = 0u;
-    // every present key fits: take them all
-    sel[s].done = s >= nsel || (int)sh.g[s][2] <= Kt[s];
-  }
-
-  // ---- rounds: histogram of the undecided range, cluster-reduced
+  // ---- levels
 #pragma unroll 1
-  while (!(sel[0].done && sel[1].done)) {
-#pragma unroll
+  for (int round = 0;; ++round) {
+    if (sh.sel[0].state == kDone && sh.sel[1].state == kDone) break;   // cluster-uniform
+    const int buf = round % 3;
+    // 1. this block's histogram; zero the owned slices of round + 1
+#pragma unroll 1
     for (int s = 0; s < 2; ++s) {
-      const uint32_t span = sel[s].hi - sel[s].lo;
-      sel[s].shift = span >= (uint32_t)kBins ? (32 - __clz(span)) - 11 : 0;
-      for (int i = tid; i < kBins; i += kT) sh.hist[s][i] = 0u;
+      const Sel &l = sh.sel[s];
+      if (l.state != kActive) continue;
+      const bool vs = l.vs;
+      const float v_lo = l.v_lo, inv = l.inv;
+      const uint32_t lo = l.lo, hi = l.hi;
+      const int shift = l.shift;
+#pragma unroll
+      for (int k = 0; k < kN; ++k) {
+        const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
+        if (kk && (vs || (kk >= lo && kk <= hi)))
+          atomicAdd(&sh.hist[s][vs ? vbin(v_lo, inv, kk) : (int)((kk - lo) >> shift)], 1u);
+      }
+    }
+    if (tid < 2 * kSeg) (&sh.hsum[(round + 1) % 3][0][0])[tid] = 0u;
+    __syncthreads();
+    // 2. thread (s, bin) pushes its bin into the owner's slice and re-zeroes it
+    {
+      const int s = tid / kBins, b = tid % kBins;
+      const uint32_t h = sh.hist[s][b];
+      if (h) {
+        sh.hist[s][b] = 0u;
+        atomicAdd(cl.map_shared_rank(&sh.hsum[buf][s][b % kSeg], b / kSeg), h);
+      }
+    }
+    cl.sync();
+    // 3. thread (s, bin) reads the bin's cluster count; a scan over the bins
+    // finds the one holding the need-th largest key
+    {
+      const int s = tid / kBins, b = tid % kBins;
+      const bool act = sh.sel[s].state == kActive;
+      const int h = act ? (int)*cl.map_shared_rank(&sh.hsum[buf][s][b % kSeg], b / kSeg) : 0;
+      const int pre = (int)block_scan<unsigned long long>((unsigned long long)h, sh.red, lane, warp);
+      const int h0 = (int)sh.red[kBins / 32 - 1], tot = (int)sh.red[31];
+      const int above = s == 0 ? h0 - pre - h : tot - pre - h;   // keys in higher bins
+      const int need = sh.sel[s].need;
+      if (act && above < need && above + h >= need) {
+        sh.th[s][0] = b;
+        sh.th[s][1] = above;
+        sh.th[s][2] = h;
+      }
     }
     __syncthreads();
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      if (sel[s].done) continue;
-      const uint32_t lo = sel[s].lo, hi = sel[s].hi;
-      const int shf = sel[s].shift;
-      if (s == 0) {
-#pragma unroll
-        for (int k = 0; k < kN; ++k)
-          if (key[k] && key[k] >= lo && key[k] <= hi) atomicAdd(&sh.hist[0][(key[k] - lo) >> shf], 1u);
+    // 4. warp s decides the next level of selection s
+    if (warp < 2 && sh.sel[warp].state == kActive) {
+      Sel &l = sh.sel[warp];
+      const int T = sh.th[warp][0], cntT = sh.th[warp][2];
+      const int need2 = l.need - sh.th[warp][1];   // 1 <= need2 <= cntT
+      uint32_t lo_T, hi_T;
+      if (l.vs) {   // exact key interval of value bin T
+        lo_T = T == 0 ? l.g_lo : first_key_of_bin(l.v_lo, l.inv, l.g_lo, l.g_hi, T, lane);
+        hi_T = T == kBins - 1 ? l.g_hi : first_key_of_bin(l.v_lo, l.inv, l.g_lo, l.g_hi, T + 1, lane) - 1u;
       } else {
-#pragma unroll
-        for (int g = 0; g < kNB; ++g)
-          if (bkey[g] && bkey[g] >= lo && bkey[g] <= hi) atomicAdd(&sh.hist[1][(bkey[g] - lo) >> shf], 1u);
+        lo_T = l.lo + ((uint32_t)T << l.shift);
+        const uint32_t w1 = (1u << l.shift) - 1u;
+        hi_T = (l.hi - lo_T > w1) ? lo_T + w1 : l.hi;
       }
-    }
-    cl.sync();   // every block's histogram is complete
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      if (sel[s].done) continue;
-      const int bin = r * (kBins / kCl) + tid;   // this block reduces 256 bins
-      uint32_t v = 0u;
-#pragma unroll
-      for (int c = 0; c < kCl; ++c) v += cl.map_shared_rank(&sh.hist[s][0], c)[bin];
-      sh.hsum[s][tid] = v;
-    }
-    cl.sync();   // every segment is reduced
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      if (sel[s].done) continue;   // cluster-uniform
-      // thread t reads bins [8t, 8t+8) of the reduced histogram
-      uint32_t h[8], local = 0u;
-      const uint32_t *seg = cl.map_shared_rank(&sh.hsum[s][0], (8 * tid) / (kBins / kCl));
-#pragma unroll
-      for (int i = 0; i < 8; ++i) { h[i] = seg[(8 * tid) % (kBins / kCl) + i]; local += h[i]; }
-      int lower;   // keys in the bins of lower threads
-      const int total = block_excl_scan((int)local, lower, sh.red);
-      const int above_me = total - lower - (int)local;   // keys in the bins of higher threads
-      const int need = sel[s].need;
-      if (above_me < need && above_me + (int)local >= need) {   // exactly one thread
-        int ab = above_me, t_bin = 8 * tid, cnt_t = (int)h[0];
-        for (int i = 7; i >= 0; --i) {
-          if (ab + (int)h[i] >= need) { t_bin = 8 * tid + i; cnt_t = (int)h[i]; break; }
-          ab += (int)h[i];
+      if (lane == 0) {
+        if (cntT == need2) {                 // every key of the bin is taken
+          l.kthr = lo_T - 1u; l.cthr = -1; l.cmode = true; l.state = kDone;
+        } else if (cntT <= kCand) {          // rank the bin's keys exactly
+          l.lo = lo_T; l.hi = hi_T; l.need = need2; l.cnt = cntT; l.vs = false; l.state = kCollect;
+        } else if (!l.vs && l.shift == 0) {  // one key value: need2 of its ties, in column order
+          l.kthr = lo_T; l.cmode = false; l.take_eq = need2; l.state = kDone;
+        } else {                             // next level inside the bin
+          l.lo = lo_T; l.hi = hi_T; l.shift = key_shift(lo_T, hi_T); l.need = need2; l.vs = false;
         }
-        sh.th[s][0] = t_bin;
-        sh.th[s][1] = ab;
-        sh.th[s][2] = cnt_t;
-      }
-      __syncthreads();
-      const int T = sh.th[s][0], above = sh.th[s][1], cntT = sh.th[s][2];
-      const uint32_t lo_T = sel[s].lo + ((uint32_t)T << sel[s].shift);
-      const uint32_t w1 = (1u << sel[s].shift) - 1u;
-      const uint32_t hi_T = (sel[s].hi - lo_T > w1) ? lo_T + w1 : sel[s].hi;
-      const int need2 = need - above;
-      if (cntT == need2) {            // bin T is taken whole: every key >= lo_T
-        sel[s].thr_gt = lo_T - 1u;
-        sel[s].take_eq = 0;
-        sel[s].done = true;
-      } else if (sel[s].shift == 0) { // bin T is one key value: need2 of its ties
-        sel[s].thr_gt = lo_T;
-        sel[s].thr_eq = lo_T;
-        sel[s].take_eq = need2;
-        sel[s].done = true;
-      } else {                        // refine inside bin T
-        sel[s].lo = lo_T;
-        sel[s].hi = hi_T;
-        sel[s].need = need2;
       }
     }
-    cl.sync();   // reduced segments are no longer read; the next round may overwrite them
+    __syncthreads();
+    if (sh.sel[0].state != kCollect && sh.sel[1].state != kCollect) continue;   // cluster-uniform
+
+    // 5. collect the region's keys in block 0 and rank them
+#pragma unroll 1
+    for (int s = 0; s < 2; ++s) {
+      const Sel &l = sh.sel[s];
+      if (l.state != kCollect) continue;
+      const uint32_t lo = l.lo, hi = l.hi;
+      int m = 0;
+#pragma unroll
+      for (int k = 0; k < kN; ++k) {
+        const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
+        m += kk && kk >= lo && kk <= hi;
+      }
+      const int incl = warp_incl_scan(m, lane);
+      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
+      uint32_t wbase = 0u;
+      if (lane == 31 && wtot > 0) wbase = atomicAdd(cl.map_shared_rank(&sh.cand_n[s], 0), (uint32_t)wtot);
+      int pos = (int)__shfl_sync(0xffffffffu, wbase, 31) + incl - m;
+      uint2 *dst = cl.map_shared_rank(&sh.cand[s][0], 0);
+#pragma unroll
+      for (int k = 0; k < kN; ++k) {
+        const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
+        if (kk && kk >= lo && kk <= hi) {
+          if (pos < kCand) dst[pos] = make_uint2(kk, (uint32_t)(s == 0 ? c0 + k : blk));
+          ++pos;
+        }
+      }
+    }
+    cl.sync();
+    {
+      const int s = tid / kBins, i = tid % kBins;
+      if (sh.sel[s].state == kCollect && i < sh.sel[s].cnt) sh.loc[s][i] = cl.map_shared_rank(&sh.cand[s][0], 0)[i];
+    }
+    __syncthreads();
+    {
+      const int s = tid / kBins, i = tid % kBins;
+      const int n = sh.sel[s].cnt;
+      if (sh.sel[s].state == kCollect && i < n) {
+        const uint2 me = sh.loc[s][i];
+        int rank = 0;
+#pragma unroll 1
+        for (int j = 0; j < n; ++j) {
+          const uint2 o = sh.loc[s][j];
+          rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        }
+        if (rank == sh.sel[s].need - 1) {   // exactly one pair
+          sh.sel[s].kthr = me.x;
+          sh.sel[s].cthr = (int)me.y;
+        }
+      }
+    }
+    __syncthreads();
+    if (tid < 2 && sh.sel[tid].state == kCollect) {
+      sh.sel[tid].cmode = true;
+      sh.sel[tid].state = kDone;
+    }
+    __syncthreads();
   }
 
-  // ---- ties (column order across the cluster) and output offsets
-  int my_ties[2] = {0, 0}, my_chosen[2] = {0, 0}, tie_base[2] = {0, 0};
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    int t = 0;
-    if (s < nsel && sel[s].take_eq > 0) {
-      if (s == 0) {
-#pragma unroll
-        for (int k = 0; k < kN; ++k) t += key[k] && key[k] == sel[s].thr_eq;
-      } else {
-#pragma unroll
-        for (int g = 0; g < kNB; ++g) t += bkey[g] && bkey[g] == sel[s].thr_eq;
-      }
-    }
-    my_ties[s] = t;
-    const int tot = block_excl_scan(t, tie_base[s], sh.red);
-    if (tid == 0) sh.cnt[s][0] = tot;
-  }
-  cl.sync();
-  int ties_before[2] = {0, 0}, allow[2] = {0, 0};
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    for (int c = 0; c < r; ++c) ties_before[s] += cl.map_shared_rank(&sh.cnt[s][0], c)[0];
-    allow[s] = sel[s].take_eq - ties_before[s];   // ties this block may still take
-  }
-  // chosen per thread (ties in column order: block prefix + thread prefix)
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    int c = 0, tr = tie_base[s];
-    if (s < nsel) {
-      if (s == 0) {
-#pragma unroll
-        for (int k = 0; k < kN; ++k) {
-          const uint32_t kk = key[k];
-          const bool tie = kk && kk == sel[s].thr_eq && sel[s].take_eq > 0;
-          c += (kk && kk > sel[s].thr_gt) || (tie && tr < allow[s]);
-          tr += tie;
-        }
-      } else {
-#pragma unroll
-        for (int g = 0; g < kNB; ++g) {
-          const uint32_t kk = bkey[g];
-          const bool tie = kk && kk == sel[s].thr_eq && sel[s].take_eq > 0;
-          c += (kk && kk > sel[s].thr_gt) || (tie && tr < allow[s]);
-          tr += tie;
-        }
-      }
-    }
-    my_chosen[s] = c;
-  }
-  int pos[2];
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int tot = block_excl_scan(my_chosen[s], pos[s], sh.red);
-    if (tid == 0) sh.cnt[s][1] = tot;
-  }
-  cl.sync();
-  int base[2] = {0, 0}, total[2] = {0, 0};
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    for (int c = 0; c < kCl; ++c) {
-      const int v = cl.map_shared_rank(&sh.cnt[s][1], c)[0];
-      if (c < r) base[s] += v;
-      total[s] += v;
-    }
-  }
-  // ---- write the chosen columns in order
+  // ---- per-block counts -> output offsets (one exchange)
+  const uint32_t kthr0 = sh.sel[0].kthr, kthr1 = sh.sel[1].kthr;
+  const int cthr0 = sh.sel[0].cthr, cthr1 = sh.sel[1].cthr;
+  const bool cm0 = sh.sel[0].cmode, cm1 = sh.sel[1].cmode;
+  int tie_base0, tie_base1;
   {
-    int o = base[0] + pos[0], tr = tie_base[0];
-    int32_t *out = a.out_idx + (size_t)row * a.K;
-    const int32_t *pb = a.pool_blocks ? a.pool_blocks + (size_t)row * (a.n_cols / 8) : nullptr;
+    int t0 = 0, s0 = 0;
 #pragma unroll
     for (int k = 0; k < kN; ++k) {
       const uint32_t kk = key[k];
-      const bool tie = kk && kk == sel[0].thr_eq && sel[0].take_eq > 0;
-      const bool take = (kk && kk > sel[0].thr_gt) || (tie && tr < allow[0]);
-      tr += tie;
-      if (take) {
-        const int col = c0 + k;
-        if (o < a.K) out[o] = pb ? pb[col >> 3] * 8 + (col & 7) : col;
-        ++o;
-      }
+      s0 += kk && (kk > kthr0 || (cm0 && kk == kthr0 && c0 + k <= cthr0));
+      t0 += kk && !cm0 && kk == kthr0;
     }
-    if (r == kCl - 1)
-      for (int i = total[0] + tid; i < a.K; i += kT) out[i] = -1;
+    const int t1 = nsel > 1 && bkey && !cm1 && bkey == kthr1;
+    const int s1 = nsel > 1 && bkey && (bkey > kthr1 || (cm1 && bkey == kthr1 && blk <= cthr1));
+    const unsigned long long v = (unsigned long long)t0 | ((unsigned long long)s0 << 16) |
+                                 ((unsigned long long)t1 << 32) | ((unsigned long long)s1 << 48);
+    const unsigned long long ex = block_scan<unsigned long long>(v, sh.red, lane, warp);
+    tie_base0 = (int)(ex & 0xFFFFu);
+    tie_base1 = (int)((ex >> 32) & 0xFFFFu);
+    if (tid == 0) {
+      const unsigned long long tot = sh.red[31];
+      sh.cnt[0] = (int)(tot & 0xFFFFu);
+      sh.cnt[1] = (int)((tot >> 16) & 0xFFFFu);
+      sh.cnt[2] = (int)((tot >> 32) & 0xFFFFu);
+      sh.cnt[3] = (int)((tot >> 48) & 0xFFFFu);
+    }
   }
-  if (nsel == 2) {
-    int o = base[1] + pos[1], tr = tie_base[1];
-    int32_t *out = a.out_pool + (size_t)row * a.P_out;
+  cl.sync();
+  if (warp < 2) {   // warp s: offsets of selection s
+    const int s = warp;
+    int tt = 0, st = 0;
+    if (lane < kCl) {
+      const int *rc = cl.map_shared_rank(&sh.cnt[0], lane);
+      tt = rc[2 * s];
+      st = rc[2 * s + 1];
+    }
+    const int ties_before = warp_incl_scan(tt, lane) - tt;
+    const int take_eq = sh.sel[s].take_eq;
+    int al = take_eq - ties_before;
+    al = al < 0 ? 0 : (al > tt ? tt : al);
+    const int chosen = st + al;
+    const int cinc = warp_incl_scan(chosen, lane);
+    const int ctot = __shfl_sync(0xffffffffu, cinc, kCl - 1);
+    if (lane == r) {
+      sh.base[s] = cinc - chosen;
+      sh.allow[s] = take_eq - ties_before;
+      sh.total[s] = ctot;
+    }
+  }
+  cluster_arrive();   // no remote shared memory is read after this point
+  __syncthreads();
+
+  // ---- write the chosen columns in order
+  {
+    const int allow0 = sh.allow[0], allow1 = sh.allow[1];
+    int n0 = 0, tr = tie_base0;
 #pragma unroll
-    for (int g = 0; g < kNB; ++g) {
-      const uint32_t kk = bkey[g];
-      const bool tie = kk && kk == sel[1].thr_eq && sel[1].take_eq > 0;
-      const bool take = (kk && kk > sel[1].thr_gt) || (tie && tr < allow[1]);
+    for (int k = 0; k < kN; ++k) {
+      const uint32_t kk = key[k];
+      const bool tie = kk && !cm0 && kk == kthr0;
+      n0 += (kk && (kk > kthr0 || (cm0 && kk == kthr0 && c0 + k <= cthr0))) || (tie && tr < allow0);
+      tr += tie;
+    }
+    const bool tie1 = nsel > 1 && bkey && !cm1 && bkey == kthr1;
+    const bool take1 = (nsel > 1 && bkey && (bkey > kthr1 || (cm1 && bkey == kthr1 && blk <= cthr1))) ||
+                       (tie1 && tie_base1 < allow1);
+    const uint32_t ex = block_scan<uint32_t>((uint32_t)n0 | ((uint32_t)take1 << 16), reinterpret_cast<uint32_t *>(sh.red),
+                                             lane, warp);
+    int o = sh.base[0] + (int)(ex & 0xFFFFu);
+    int32_t *out = a.out_idx + (size_t)row * a.K;
+    const int32_t *pb = a.pool_blocks ? a.pool_blocks + (size_t)row * (a.n_cols / 8) : nullptr;
+    tr = tie_base0;
+#pragma unroll
+    for (int k = 0; k < kN; ++k) {
+      const uint32_t kk = key[k];
+      const bool tie = kk && !cm0 && kk == kthr0;
+      const bool take = (kk && (kk > kthr0 || (cm0 && kk == kthr0 && c0 + k <= cthr0))) || (tie && tr < allow0);
       tr += tie;
       if (take) {
-        if (o < a.P_out) out[o] = (c0 >> 3) + g;
+        if (o < a.K) out[o] = pb ? pb[blk] * 8 + k : c0 + k;
         ++o;
       }
     }
-    if (r == kCl - 1)
-      for (int i = total[1] + tid; i < a.P_out; i += kT) out[i] = -1;
+    if (take1) {
+      const int o1 = sh.base[1] + (int)(ex >> 16);
+      if (o1 < a.P_out) a.out_pool[(size_t)row * a.P_out + o1] = blk;
+    }
+    if (r == kCl - 1) {
+      for (int i = sh.total[0] + tid; i < a.K; i += kT) out[i] = -1;
+      if (nsel > 1)
+        for (int i = sh.total[1] + tid; i < a.P_out; i += kT) a.out_pool[(size_t)row * a.P_out + i] = -1;
+    }
   }
-  cl.sync();   // no block leaves while another may still read its shared memory
+  cluster_wait();   // no block leaves while another may still read its shared memory
 }
 
-// Rows of up to kCl * kT * kN columns go through the cluster kernel.
-bool topk_cluster_fits(int n_cols) { return n_cols <= kCl * kT * kN; }
+// Rows of up to kCl * kSpan columns go through the cluster kernel.
+bool topk_cluster_fits(int n_cols) { return n_cols <= kCl * kSpan; }
 
 cudaError_t launch_topk_cluster(const TopkArgs &a, cudaStream_t s) {
-  // slice per block: a multiple of 8 columns per thread
-  int npt = (a.n_cols + kCl * kT - 1) / (kCl * kT);
-  npt = (npt + 7) / 8 * 8;
-  if (npt < 8) npt = 8;
-  topk_cluster_kernel<<<dim3(kCl, a.rows), kT, 0, s>>>(a, npt * kT);
+  topk_cluster_kernel<<<dim3(kCl, a.rows), kT, 0, s>>>(a);
   return cudaGetLastError();
 }
 

@@ -10,6 +10,7 @@ accumulation of exact FP8 products over <= 64 heads: ~64 * 2^-24 relative,
 with headroom for the tensor-core accumulation order).
 """
 import math
+import zlib
 
 import numpy as np
 import pytest
@@ -205,6 +206,43 @@ def test_topk_exact_on_same_scores(rows, n, K, P, levels):
     if P:
         refp = np.stack([oracle.block_pool(s[r, :n_valid[r]].astype(np.float64), P) for r in range(rows)])
         np.testing.assert_array_equal(pool.cpu().numpy(), refp)
+
+
+def _hard_scores(kind, rows, n, rng):
+    s = rng.standard_normal((rows, n)).astype(np.float32)
+    if kind == "outlier":            # one huge score: every other score shares the first value bin
+        s[:, n // 3] = 1e30
+    elif kind == "constant":         # a single value: ties decided by column only
+        s[:] = 0.75
+    elif kind == "huge_range":       # the value range overflows binary32
+        s[:, 1] = -3e38
+        s[:, 2] = 3e38
+    elif kind == "two_clusters":     # two narrow groups far apart, the K-th inside the upper one
+        s = np.where(rng.random((rows, n)) < 0.02, 1000.0 + 1e-3 * s, 1e-3 * s).astype(np.float32)
+    elif kind == "tiny":             # subnormal and tiny normal magnitudes
+        s = (s * np.float32(1e-39)).astype(np.float32)
+    elif kind == "few_values":       # 5 distinct values, many ties at the K-th
+        s = np.round(s).astype(np.float32)
+    return s
+
+
+@pytest.mark.parametrize("kind", ["outlier", "constant", "huge_range", "two_clusters", "tiny", "few_values"])
+@pytest.mark.parametrize("n", [65536, 20000])
+def test_topk_exact_on_hard_distributions(kind, n):
+    rows, K, P = 2, 512, 2048
+    rng = np.random.default_rng(zlib.crc32(f"{kind}/{n}".encode()))
+    s = _hard_scores(kind, rows, n, rng)
+    s[1, rng.choice(n, n // 10, replace=False)] = -np.inf
+    n_valid = np.array([n, n - 5], np.int32)
+    out = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    pool = torch.empty(rows, P, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_topk_workspace_size(rows, n, K, P))
+    C.csa2_topk(torch.from_numpy(s).cuda(), n, K, out, n_valid=torch.from_numpy(n_valid).cuda(), P_out=P,
+                out_pool=pool, ws=ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy(), _ref_topk_rows(s, n_valid, K))
+    refp = np.stack([oracle.block_pool(s[r, :n_valid[r]].astype(np.float64), P) for r in range(rows)])
+    np.testing.assert_array_equal(pool.cpu().numpy(), refp)
 
 
 def test_topk_pool_mapping_for_reindex_rows():
