@@ -343,10 +343,9 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   DeviceState *d;
   if ((st = device_state(&d)) != CSA2_OK) return st;
   AttnPlan p = plan_attn(main->B, T_q, H, main->D, K, swa->window, d->sms);
-  if (p.nsplit > 1 && (!ws || ws_bytes < p.bytes || !aligned16(ws))) {
-    const int nc = (K + 63) / 64 + (swa->window + 63) / 64;
+  if (p.nsplit > 1 && (!ws || ws_bytes < p.bytes || !aligned16(ws))) {   // no workspace: one block per row
     p.nsplit = 1;
-    p.chunks_per_split = nc;
+    p.chunks_per_split = 1 << 20;
   }
   AttnArgs a{};
   a.codes = main->codes; a.scales = main->scales; a.cap = main->cap; a.D = main->D;

@@ -6,14 +6,16 @@
 //
 // One block per (query row, key split); keys in tiles of 128 (the selected
 // entries first, then the window rows).  Per tile:
-//   1. all 8 warps gather the tile's rows (FP4 codes + scales, or E4M3 rows)
-//      and dequantise them exactly into fp16 in shared memory, laid out as a
-//      K-major 128B-swizzled operand (E2M1 x E4M3 and E4M3 are exact in fp16);
+//   1. every thread issues all of its gather loads at once (FP4 codes +
+//      scales, or E4M3 rows) and dequantises them exactly into fp16 with the
+//      hardware E2M1/E4M3 -> f16x2 converts (E2M1 x E4M3 products and E4M3
+//      values are exact in fp16), laid out in shared memory as a K-major
+//      128B-swizzled operand;
 //   2. S^T = K^ Q^T on tcgen05 (kind::f16, M = 128 keys, N = 64 heads,
 //      K = D): TMEM lane = key, column = head;
-//   3. warps 0-3 (one TMEM lane quarter each) read S^T, reduce the per-head
-//      maximum and sum across the 128 lanes with a reduce-scatter butterfly,
-//      exponentiate (base 2) and write P^T (fp16) as the next B operand;
+//   3. all 8 warps (TMEM lane quarter x 32-head half) form the per-head
+//      maxima and sums over the 128 keys and write P (fp16) row by row as an
+//      MN-major operand [key][head];
 //   4. O^T += V^T P^T on tcgen05 (M = 128 channels per TMEM block, N = 64
 //      heads, K = 128 keys).  V^T is the same shared-memory tile as K^, read
 //      as an MN-major operand, so the tile is dequantised once.
@@ -21,8 +23,12 @@
 // than 2^8 (then O^T and the running sum are rescaled in place), so P stays
 // within fp16 range and rescaling is rare.  Window rows keep their raw E4M3
 // values; the layer's window scale multiplies their logits and their P.
-// With several splits per row each writes (m, l, O) partials that
-// attn_combine_kernel merges.
+// The splits of one row form a thread-block cluster: each writes its
+// unnormalised O^T and (max, sum) per head to the workspace, and after one
+// cluster barrier each split merges a slice of the channels from all splits
+// and writes the bf16 output.  Straight-line code is kept short (rolled
+// loops): each block runs it about once, so fetching it costs as much as
+// executing it.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -37,29 +43,15 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;      // log2 headroom before the reference max moves
 constexpr uint32_t kWaitLimit = 1u << 22;
 
-// fp16 bits of the 16 E2M1 codes (0, .5, 1, 1.5, 2, 3, 4, 6 and negatives).
-__constant__ uint16_t kE2m1Half[16] = {0x0000, 0x3800, 0x3C00, 0x3E00, 0x4000, 0x4200, 0x4400, 0x4600,
-                                       0x8000, 0xB800, 0xBC00, 0xBE00, 0xC000, 0xC200, 0xC400, 0xC600};
-
-// E4M3 byte -> fp16 bits (exact): normal e>0 maps to fp16 exponent e+8,
-// subnormal m*2^-9 is an fp16 normal.
-__device__ __forceinline__ uint32_t e4m3_to_half_bits(uint32_t b) {
-  const uint32_t s = (b & 0x80u) << 8, e = (b >> 3) & 15u, m = b & 7u;
-  if (e) return s | ((e + 8u) << 10) | (m << 7);
-  if (m == 0) return s;
-  const uint32_t p = 31u - __clz(m);   // m * 2^-9 = 2^(p-9) * (m / 2^p)
-  return s | ((p - 9u + 15u) << 10) | (((m << (3u - p)) & 7u) << 7);
-}
-
 template <int D>
 struct AttnSmem {
   alignas(1024) uint8_t kh[(D / 64) * kTile * 128];   // K^ tile: D/64 chunks of [128 keys x 128 B]
   alignas(1024) uint8_t q[(D / 64) * kHeads * 128];   // Q: D/64 chunks of [64 heads x 128 B]
-  alignas(1024) uint8_t p[2 * kHeads * 128];          // P^T: 2 chunks of [64 heads x 128 B]
-  uint32_t lut[256];                                  // code byte -> fp16 pair (low nibble first)
-  int key_ent[kTile];                                 // entry id or window slot, -1 = masked
+  alignas(1024) uint8_t p[kTile * 128];               // P: [128 keys][64 heads] fp16, MN-major
+  int key_ent[2][kTile];                              // entry id or window slot, -1 = masked
   float red[4][kHeads];
   float m_ref[kHeads], l_run[kHeads], alpha[kHeads];
+  float wgt[8][kHeads];                               // merge weights of the splits
   uint64_t sbar, obar;
   uint32_t tmem_base;
   int rescale;
@@ -71,42 +63,68 @@ __device__ __forceinline__ uint32_t sw_off(int r, int pc, int rows) {
   return (uint32_t)((pc >> 3) * rows * 128 + r * 128 + (((pc & 7) ^ (r & 7)) << 4));
 }
 
-// Reduce-scatter of 64 values across the 32 lanes of a warp: afterwards
-// t[0], t[1] hold the reduction over the warp of columns c, c+1 with
-// c = the lane's column base (returned).
-template <bool MAX>
-__device__ __forceinline__ int reduce_scatter64(float *t, int lane) {
-  int base = 0;
+// After the call, lane l holds in t[0] the sum over the warp of column l.
+__device__ __forceinline__ void reduce_scatter32(float *t, int lane) {
 #pragma unroll
-  for (int o = 16, n = 32; o >= 1; o >>= 1, n >>= 1) {
+  for (int o = 16; o >= 1; o >>= 1) {
     const bool up = (lane & o) != 0;
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      if (j < n) {
-        const float lo = t[j], hi = t[j + n];
-        const float send = up ? lo : hi, keep = up ? hi : lo;
-        const float recv = __shfl_xor_sync(0xffffffffu, send, o);
-        t[j] = MAX ? fmaxf(keep, recv) : keep + recv;
+    for (int j = 0; j < 16; ++j) {
+      if (j < o) {
+        const float lo = t[j], hi = t[j + o];
+        const float recv = __shfl_xor_sync(0xffffffffu, up ? lo : hi, o);
+        t[j] = (up ? hi : lo) + recv;
       }
     }
-    if (up) base += n;
   }
-  return base;
+}
+
+__device__ __forceinline__ int ordered(float f) {
+  const int b = __float_as_int(f);
+  return b >= 0 ? b : (b ^ 0x7FFFFFFF);
+}
+__device__ __forceinline__ float unordered(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7FFFFFFF)); }
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Key ids of tile c (threads 0..127): entry ids of the selected entries, or
+// ring slots of the window rows; -1 = masked.
+__device__ __forceinline__ void load_key_ids(const AttnArgs &a, int row, int c, int n_fp4_tiles, int wlo, int nwin,
+                                             int *dst, int tid) {
+  if (tid >= kTile) return;
+  int id = -1;
+  if (c < n_fp4_tiles) {
+    const int k = c * kTile + tid;
+    if (k < a.K) {
+      const int e = a.idx[(size_t)row * a.K + k];
+      if (e >= a.cap) flag(a.status, CSA2_DEV_INDEX_RANGE);
+      id = (e >= 0 && e < a.cap) ? e : -1;
+    }
+  } else {
+    const int j = (c - n_fp4_tiles) * kTile + tid;
+    id = j < nwin ? (wlo + j) % a.W_cap : -1;
+  }
+  dst[tid] = id;
 }
 
 }  // namespace
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
-  constexpr int NCH = D / 64;                      // 64-channel chunks
   constexpr int MT = D / 128;                      // O^T TMEM blocks of 128 channels
+  constexpr int QI = kHeads * (D / 8) / kThreads;  // 16-byte pieces of Q per thread
+  constexpr int GF = D / 64;                       // FP4 items (32 channels) per thread and tile
+  constexpr int GW = D / 32;                       // window items (16 channels) per thread and tile
   constexpr uint32_t kCols = D == 128 ? 128u : (D == 256 ? 256u : 512u);
   constexpr uint32_t kIdS = mma_idesc(128, kHeads, 0u /*f16*/, 0u /*f16*/);
-  constexpr uint32_t kIdO = kIdS | (1u << 15);     // A (V^T) MN-major
+  constexpr uint32_t kIdO = kIdS | (1u << 15) | (1u << 16);   // A (V^T) and B (P^T) MN-major
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D> &S = *reinterpret_cast<AttnSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                    ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int quarter = warp & 3, half = warp >> 2;   // TMEM lane quarter, 32-head half
   const int row = blockIdx.x;   // b * T_q + query
   const int split = blockIdx.y;
   const int b = row / a.T_q;
@@ -122,7 +140,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   int c_end = c_begin + a.chunks_per_split;
   if (c_end > total) c_end = total;
 
-  // ---- set-up
+  // ---- set-up; Q loads and the first tile's key ids are issued together
   if (tid == 0) {
     mbar_init(&S.sbar, 1);
     mbar_init(&S.obar, 1);
@@ -133,28 +151,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     tmem_alloc(&S.tmem_base, kCols);
     tmem_relinquish();
   }
-  for (int i = tid; i < 256; i += kThreads)
-    S.lut[i] = (uint32_t)kE2m1Half[i & 15] | ((uint32_t)kE2m1Half[i >> 4] << 16);
-  if (tid < kHeads) { S.m_ref[tid] = -INFINITY; S.l_run[tid] = 0.f; S.alpha[tid] = 1.f; }
-  // Q: bf16 -> fp16 into the B-operand layout (heads >= H are zero), in
-  // batches of 4 items whose loads are all issued before they are used
+  uint4 qraw[QI];
   {
-    constexpr int QI = kHeads * (D / 8) / kThreads;   // 16-byte items per thread
     const uint16_t *qrow = a.q + (size_t)row * a.H * D;
+#pragma unroll
+    for (int u = 0; u < QI; ++u) {
+      const int i = tid + u * kThreads;
+      const int h = i / (D / 8), pc = i % (D / 8);
+      qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  if (c_begin < c_end) load_key_ids(a, row, c_begin, n_fp4_tiles, wlo, nwin, S.key_ent[c_begin & 1], tid);
+  if (tid < kHeads) { S.m_ref[tid] = -INFINITY; S.l_run[tid] = 0.f; S.alpha[tid] = 1.f; }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  const uint32_t kh_base = smem_u32(S.kh), q_base = smem_u32(S.q), p_base = smem_u32(S.p);
+
+  bool aborted = false;
+  int n_done = 0;   // tiles whose O^T MMAs were issued
 #pragma unroll 1
-    for (int j0 = 0; j0 < QI; j0 += 4) {
-      uint4 raw[4];
+  for (int c = c_begin; c < c_end; ++c) {
+    const bool is_win = c >= n_fp4_tiles;
+    const int *ids = S.key_ent[c & 1];
+    // ---- 1a. gather loads, all issued before any is used: FP4 item = 32
+    // channels (16 code bytes + 2 scale bytes), window item = 16 E4M3 bytes
+    uint4 raw[GW];
+    uint32_t sc[GF];
+    if (!is_win) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = tid + (j0 + u) * kThreads;
-        const int h = i / (D / 8), pc = i % (D / 8);
-        raw[u] = h < a.H ? *reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < GF; ++u) {
+        const int i = tid + u * kThreads;
+        const int r = i / (D / 32), g = i % (D / 32);
+        const int id = ids[r];
+        raw[u] = make_uint4(0, 0, 0, 0);
+        sc[u] = 0u;
+        if (id >= 0) {
+          const size_t er = (size_t)b * a.cap + id;
+          raw[u] = __ldg(reinterpret_cast<const uint4 *>(a.codes + er * (D / 2)) + g);
+          sc[u] = __ldg(reinterpret_cast<const uint16_t *>(a.scales + er * (D / 16)) + g);
+        }
       }
+    } else {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int i = tid + (j0 + u) * kThreads;
+      for (int u = 0; u < GW; ++u) {
+        const int i = tid + u * kThreads;
+        const int r = i / (D / 16), g = i % (D / 16);
+        const int id = ids[r];
+        raw[u] = id >= 0 ? __ldg(reinterpret_cast<const uint4 *>(a.swa_rows + ((size_t)b * a.W_cap + id) * D) + g)
+                         : make_uint4(0, 0, 0, 0);
+      }
+    }
+    // ---- Q: bf16 -> fp16 into the B-operand layout (first tile only)
+    if (c == c_begin) {
+#pragma unroll
+      for (int u = 0; u < QI; ++u) {
+        const int i = tid + u * kThreads;
         const int h = i / (D / 8), pc = i % (D / 8);
-        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+        const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
         uint32_t o[4];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -164,88 +219,46 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
         *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
-  const uint32_t kh_base = smem_u32(S.kh), q_base = smem_u32(S.q), p_base = smem_u32(S.p);
-
-  bool aborted = false;
-  int n_done = 0;   // tiles whose O^T MMAs were issued
-  for (int c = c_begin; c < c_end && !aborted; ++c) {
-    const bool is_win = c >= n_fp4_tiles;
-    // ---- key ids
-    if (tid < kTile) {
-      int id = -1;
-      if (!is_win) {
-        const int k = c * kTile + tid;
-        if (k < a.K) {
-          const int e = a.idx[(size_t)row * a.K + k];
-          if (e >= a.cap) flag(a.status, CSA2_DEV_INDEX_RANGE);
-          id = (e >= 0 && e < a.cap) ? e : -1;
-        }
-      } else {
-        const int j = (c - n_fp4_tiles) * kTile + tid;
-        id = j < nwin ? (wlo + j) % a.W_cap : -1;
-      }
-      S.key_ent[tid] = id;
-    }
-    // the previous tile's O^T MMAs read K^ and P^T: wait before overwriting
+    // the previous tile's O^T MMAs read K^ and P: wait before overwriting
     bool ok = true;
     if (n_done > 0) ok = mbar_wait_bounded(&S.obar, (n_done - 1) & 1, kWaitLimit);
     if (__syncthreads_or(!ok)) { aborted = true; break; }
 
-    // ---- 1. gather + dequantise: item = 16 channels of one row -> 2 pieces,
-    // in batches of 4 items whose loads are issued before they are decoded
-    {
-      constexpr int GI = kTile * (D / 16) / kThreads;   // items per thread
-#pragma unroll 1
-      for (int j0 = 0; j0 < GI; j0 += 4) {
-        uint4 raw[4];   // FP4: codes in .x/.y, scale byte in .z; window: 16 E4M3 bytes
+    // ---- 1b. dequantise (hardware converts, exact) into the swizzled K^ tile
+    if (!is_win) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = tid + (j0 + u) * kThreads;
-          const int r = i / (D / 16), g = i % (D / 16);
-          const int id = S.key_ent[r];
-          raw[u] = make_uint4(0, 0, 0, 0);
-          if (id >= 0) {
-            if (!is_win) {
-              const size_t er = (size_t)b * a.cap + id;
-              const uint2 cb = *reinterpret_cast<const uint2 *>(a.codes + er * (D / 2) + g * 8);
-              raw[u] = make_uint4(cb.x, cb.y, a.scales[er * (D / 16) + g], 0);
-            } else {
-              raw[u] = *reinterpret_cast<const uint4 *>(a.swa_rows + ((size_t)b * a.W_cap + id) * D + g * 16);
-            }
+      for (int u = 0; u < GF; ++u) {
+        const int i = tid + u * kThreads;
+        const int r = i / (D / 32), g = i % (D / 32);
+        const uint32_t s2 = e4m3x2_to_f16x2(sc[u]);   // scales of channels 32g.. and 32g+16..
+        const __half2 slo = __low2half2(*reinterpret_cast<const __half2 *>(&s2));
+        const __half2 shi = __high2half2(*reinterpret_cast<const __half2 *>(&s2));
+        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {   // 8 channels -> one 16-byte piece
+          uint32_t h[4];
+          e2m1x8_to_f16x2(w[k], h);
+          const __half2 sk = k < 2 ? slo : shi;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h[e]), sk);
+            h[e] = *reinterpret_cast<const uint32_t *>(&v);
           }
+          *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 4 * g + k, kTile)) = make_uint4(h[0], h[1], h[2], h[3]);
         }
+      }
+    } else {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int i = tid + (j0 + u) * kThreads;
-          const int r = i / (D / 16), g = i % (D / 16);
-          uint32_t out[8];
-          if (!is_win) {
-            const uint32_t sh = e4m3_to_half_bits(raw[u].z);
-            const __half2 s2 = __halves2half2(__ushort_as_half((unsigned short)sh), __ushort_as_half((unsigned short)sh));
-            const uint32_t bytes[2] = {raw[u].x, raw[u].y};
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t pr = S.lut[(bytes[k >> 2] >> (8 * (k & 3))) & 0xFFu];
-              const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&pr), s2);
-              out[k] = *reinterpret_cast<const uint32_t *>(&v);
-            }
-          } else {
-            const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-              const uint32_t b0 = (w[k >> 1] >> (16 * (k & 1))) & 0xFFu;
-              const uint32_t b1 = (w[k >> 1] >> (16 * (k & 1) + 8)) & 0xFFu;
-              out[k] = e4m3_to_half_bits(b0) | (e4m3_to_half_bits(b1) << 16);
-            }
-          }
-          *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 2 * g, kTile)) = make_uint4(out[0], out[1], out[2], out[3]);
-          *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 2 * g + 1, kTile)) = make_uint4(out[4], out[5], out[6], out[7]);
-        }
+      for (int u = 0; u < GW; ++u) {
+        const int i = tid + u * kThreads;
+        const int r = i / (D / 16), g = i % (D / 16);
+        uint32_t h[8];
+        e4m3x4_to_f16x2(raw[u].x, h);
+        e4m3x4_to_f16x2(raw[u].y, h + 2);
+        e4m3x4_to_f16x2(raw[u].z, h + 4);
+        e4m3x4_to_f16x2(raw[u].w, h + 6);
+        *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 2 * g, kTile)) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 2 * g + 1, kTile)) = make_uint4(h[4], h[5], h[6], h[7]);
       }
     }
     fence_proxy_async();
@@ -254,117 +267,120 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
 
     // ---- 2. S^T = K^ Q^T
     if (tid == 128) {
+      // descriptors advance by (byte offset >> 4) in their start-address field
       tc_fence_after();
-#pragma unroll 1
+      const uint64_t da = smem_desc_kmajor(kh_base, 128), db = smem_desc_kmajor(q_base, 128);
+#pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (uint32_t)((ks >> 2) * 0 + (ks & 3) * 32);
-        const uint32_t a_addr = kh_base + (ks >> 2) * (kTile * 128) + off;
-        const uint32_t b_addr = q_base + (ks >> 2) * (kHeads * 128) + off;
-        tc_mma_f16(tmem, smem_desc_kmajor(a_addr, 128), smem_desc_kmajor(b_addr, 128), kIdS, ks > 0 ? 1u : 0u);
+        const uint32_t off = (uint32_t)((ks & 3) * 32);
+        tc_mma_f16(tmem, da + (((ks >> 2) * (kTile * 128) + off) >> 4), db + (((ks >> 2) * (kHeads * 128) + off) >> 4),
+                   kIdS, ks > 0 ? 1u : 0u);
       }
       tc_commit(&S.sbar);
     }
+    // the next tile's key ids (the other buffer) while the MMAs run
+    if (c + 1 < c_end) load_key_ids(a, row, c + 1, n_fp4_tiles, wlo, nwin, S.key_ent[(c + 1) & 1], tid);
     ok = mbar_wait_bounded(&S.sbar, (c - c_begin) & 1, kWaitLimit);
     if (__syncthreads_or(!ok)) { aborted = true; break; }
     tc_fence_after();
 
-    // ---- 3. softmax (warps 0-3: TMEM lane = key)
+    // ---- 3. softmax: warp (quarter, half) holds keys 32*quarter + lane,
+    // heads 32*half .. 32*half + 31
     const float lsc = a.scale * (is_win ? a.s_swa : 1.0f) * kLog2e;
     const float psc = is_win ? a.s_swa : 1.0f;
     const bool first = (c == c_begin);
-    if (warp < 4) {
-      const int r = 32 * warp + lane;
-      float sv[kHeads], tt[kHeads];
-      {
-        uint32_t raw[kHeads];
-        tmem_ld_x32(tmem + ((uint32_t)(32 * warp) << 16), raw);
-        tmem_ld_x32(tmem + ((uint32_t)(32 * warp) << 16) + 32, raw + 32);
-        tmem_wait_ld();
-        const bool valid = S.key_ent[r] >= 0;
+    const int r = 32 * quarter + lane;
+    float sv[32];
+    {
+      uint32_t rv[32];
+      tmem_ld_x32(tmem + ((uint32_t)(32 * quarter) << 16) + 32 * half, rv);
+      tmem_wait_ld();
+      const bool valid = ids[r] >= 0;
+      int mine = 0;
 #pragma unroll
-        for (int h = 0; h < kHeads; ++h) {
-          sv[h] = valid ? __uint_as_float(raw[h]) * lsc : -INFINITY;
-          tt[h] = sv[h];
-        }
+      for (int j = 0; j < 32; ++j) {
+        sv[j] = valid ? __uint_as_float(rv[j]) * lsc : -INFINITY;
+        const int m = __reduce_max_sync(0xffffffffu, ordered(sv[j]));
+        mine = lane == j ? m : mine;
       }
-      // per-head max over the warp's 32 keys: integer max of order-preserving bits
-#pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
-        const int bits = __float_as_int(tt[h]);
-        const int key = bits >= 0 ? bits : (bits ^ 0x7FFFFFFF);
-        const int mk = __reduce_max_sync(0xffffffffu, key);
-        if (lane == (h & 31)) S.red[warp][h] = __int_as_float(mk >= 0 ? mk : (mk ^ 0x7FFFFFFF));
-      }
-      named_bar(1, 128);
-      int cb;
-      if (tid < kHeads) {   // new reference max of head tid
-        const float m_old = S.m_ref[tid];
-        const float mt = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]), fmaxf(S.red[2][tid], S.red[3][tid]));
-        float al = 1.f;
-        if (mt != -INFINITY) {
-          if (m_old == -INFINITY) {
-            S.m_ref[tid] = mt;
-            al = 0.f;
-          } else if (mt > m_old + kLazy) {
-            S.m_ref[tid] = mt;
-            al = exp2f(m_old - mt);
-            if (!first) S.rescale = 1;
-          }
-        }
-        S.alpha[tid] = al;
-        S.l_run[tid] *= al;
-      }
-      named_bar(1, 128);
-      // P = 2^(s - m_ref), written as P^T[head][key] (fp16, window rows scaled)
-#pragma unroll
-      for (int h = 0; h < kHeads; ++h) {
-        const float m = S.m_ref[h];
-        const float pv = (sv[h] == -INFINITY || m == -INFINITY) ? 0.f : exp2f(sv[h] - m);
-        tt[h] = pv;
-        const __half hp = __float2half_rn(pv * psc);
-        *reinterpret_cast<__half *>(S.p + sw_off(h, r >> 3, kHeads) + (r & 7) * 2) = hp;
-      }
-      cb = reduce_scatter64<false>(tt, lane);
-      S.red[warp][cb] = tt[0];
-      S.red[warp][cb + 1] = tt[1];
-      named_bar(1, 128);
-      if (tid < kHeads) S.l_run[tid] += (S.red[0][tid] + S.red[1][tid]) + (S.red[2][tid] + S.red[3][tid]);
-      named_bar(1, 128);
-      // rare: a head's reference max moved -> rescale its O^T column
-      if (S.rescale) {
-#pragma unroll 1
-        for (int mt = 0; mt < MT; ++mt) {
-          const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + kHeads + mt * kHeads;
-          uint32_t o[kHeads];
-          tmem_ld_x32(taddr, o);
-          tmem_ld_x32(taddr + 32, o + 32);
-          tmem_wait_ld();
-#pragma unroll
-          for (int h = 0; h < kHeads; ++h) o[h] = __float_as_uint(__uint_as_float(o[h]) * S.alpha[h]);
-          tmem_st_x32(taddr, o);
-          tmem_st_x32(taddr + 32, o + 32);
-        }
-        tmem_wait_st();
-        named_bar(1, 128);
-        if (tid == 0) S.rescale = 0;
-      }
+      S.red[quarter][32 * half + lane] = unordered(mine);
     }
-    fence_proxy_async();   // P^T (generic stores) -> visible to the tensor core
+    __syncthreads();
+    if (tid < kHeads) {   // new reference max of head tid
+      const float m_old = S.m_ref[tid];
+      const float mt = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]), fmaxf(S.red[2][tid], S.red[3][tid]));
+      float al = 1.f;
+      if (mt != -INFINITY) {
+        if (m_old == -INFINITY) {
+          S.m_ref[tid] = mt;
+          al = 0.f;
+        } else if (mt > m_old + kLazy) {
+          S.m_ref[tid] = mt;
+          al = exp2f(m_old - mt);
+          if (!first) S.rescale = 1;
+        }
+      }
+      S.alpha[tid] = al;
+      S.l_run[tid] *= al;
+    }
+    __syncthreads();
+    // P = 2^(s - m_ref): row r of the P operand (fp16, window rows scaled)
+    {
+      const float4 *mp = reinterpret_cast<const float4 *>(&S.m_ref[32 * half]);
+      uint32_t ph[16];
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 m4 = mp[j4];
+        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int j = 4 * j4 + k;
+          sv[j] = (sv[j] == -INFINITY || mm[k] == -INFINITY) ? 0.f : exp2f(sv[j] - mm[k]);
+        }
+        const __half2 h0 = __floats2half2_rn(sv[4 * j4] * psc, sv[4 * j4 + 1] * psc);
+        const __half2 h1 = __floats2half2_rn(sv[4 * j4 + 2] * psc, sv[4 * j4 + 3] * psc);
+        ph[2 * j4] = *reinterpret_cast<const uint32_t *>(&h0);
+        ph[2 * j4 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        *reinterpret_cast<uint4 *>(S.p + r * 128 + (((4 * half + i) ^ (r & 7)) << 4)) =
+            make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
+      reduce_scatter32(sv, lane);   // sv[0] = sum over this warp's keys of head 32*half + lane
+    }
+    S.red[quarter][32 * half + lane] = sv[0];   // the max readers finished before the last barrier
+    __syncthreads();
+    if (tid < kHeads) S.l_run[tid] += (S.red[0][tid] + S.red[1][tid]) + (S.red[2][tid] + S.red[3][tid]);
+    // rare: a head's reference max moved -> rescale its O^T column
+    if (S.rescale) {
+#pragma unroll 1
+      for (int mt = 0; mt < MT; ++mt) {
+        const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + kHeads + mt * kHeads + 32 * half;
+        uint32_t o[32];
+        tmem_ld_x32(taddr, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * S.alpha[32 * half + j]);
+        tmem_st_x32(taddr, o);
+      }
+      tmem_wait_st();
+    }
+    fence_proxy_async();   // P (generic stores) -> visible to the tensor core
     tc_fence_before();
     __syncthreads();
+    if (tid == 0) S.rescale = 0;
 
     // ---- 4. O^T += V^T P^T
     if (tid == 128) {
       tc_fence_after();
-#pragma unroll 1
+      const uint64_t da = smem_desc_mnmajor_sw128(kh_base, kTile * 128, 1024);
+      const uint64_t db = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
+#pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-#pragma unroll 1
-        for (int ks = 0; ks < kTile / 16; ++ks) {
-          const uint32_t a_addr = kh_base + (2 * mt) * (kTile * 128) + (2 * ks) * 1024;
-          const uint32_t b_addr = p_base + (ks >> 2) * (kHeads * 128) + (ks & 3) * 32;
-          tc_mma_f16(tmem + kHeads + mt * kHeads, smem_desc_mnmajor_sw128(a_addr, kTile * 128, 1024),
-                     smem_desc_kmajor(b_addr, 128), kIdO, (ks > 0 || !first) ? 1u : 0u);
-        }
+#pragma unroll
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          tc_mma_f16(tmem + kHeads + mt * kHeads, da + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
+                     db + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0 || !first) ? 1u : 0u);
       }
       tc_commit(&S.obar);
     }
@@ -374,7 +390,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   // ---- epilogue: O^T (TMEM lane = channel within a 128-channel block)
   bool ok = !aborted;
   if (ok && n_done > 0) ok = mbar_wait_bounded(&S.obar, (n_done - 1) & 1, kWaitLimit);
-  if (__syncthreads_or(!ok)) {
+  const bool failed = __syncthreads_or(!ok);
+  if (failed) {
     if (tid == 0) flag(a.status, CSA2_DEV_TIMEOUT);
     if (tid == 128 && n_done > 0) {   // let every issued MMA finish before TMEM is freed
       mbar_init(&S.sbar, 1);
@@ -382,88 +399,118 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       tc_commit(&S.sbar);
       mbar_wait_bounded(&S.sbar, 0, kWaitLimit);
     }
-    __syncthreads();
   } else {
     tc_fence_after();
-    if (warp < 4) {
-      const size_t nrows = (size_t)a.B * a.T_q;
+    const size_t nrows = (size_t)a.B * a.T_q;
 #pragma unroll 1
-      for (int mt = 0; mt < MT; ++mt) {
-        const int ch = mt * 128 + 32 * warp + lane;
-        uint32_t o[kHeads];
-        if (n_done > 0) {
-          const uint32_t taddr = tmem + ((uint32_t)(32 * warp) << 16) + kHeads + mt * kHeads;
-          tmem_ld_x32(taddr, o);
-          tmem_ld_x32(taddr + 32, o + 32);
-          tmem_wait_ld();
-        } else {
+    for (int mt = 0; mt < MT; ++mt) {
+      const int ch = mt * 128 + 32 * quarter + lane;
+      uint32_t o[32];
+      if (n_done > 0) {
+        tmem_ld_x32(tmem + ((uint32_t)(32 * quarter) << 16) + kHeads + mt * kHeads + 32 * half, o);
+        tmem_wait_ld();
+      } else {
 #pragma unroll
-          for (int h = 0; h < kHeads; ++h) o[h] = 0u;
-        }
-        if (a.nsplit == 1) {
-          uint16_t *orow = a.out + (size_t)row * a.H * D;
-#pragma unroll
-          for (int h = 0; h < kHeads; ++h) {
-            if (h < a.H) {
-              const float l = S.l_run[h];
-              const float v = l > 0.f ? __uint_as_float(o[h]) / l : 0.f;
-              const __nv_bfloat16 bv = __float2bfloat16_rn(v);
-              orow[(size_t)h * D + ch] = *reinterpret_cast<const uint16_t *>(&bv);
-            }
-          }
-        } else {
-          float *po = a.ws + ((size_t)row * a.nsplit + split) * kHeads * D;
-#pragma unroll
-          for (int h = 0; h < kHeads; ++h) po[(size_t)h * D + ch] = __uint_as_float(o[h]);
-        }
+        for (int j = 0; j < 32; ++j) o[j] = 0u;
       }
-      if (a.nsplit > 1 && tid < kHeads) {
-        float *pm = a.ws + nrows * a.nsplit * kHeads * D + ((size_t)row * a.nsplit + split) * kHeads;
-        float *pl = pm + nrows * a.nsplit * kHeads;
-        pm[tid] = S.m_ref[tid];
-        pl[tid] = S.l_run[tid];
+      if (a.nsplit == 1) {
+        uint16_t *orow = a.out + (size_t)row * a.H * D;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int h = 32 * half + j;
+          if (h < a.H) {
+            const float l = S.l_run[h];
+            const __nv_bfloat16 bv = __float2bfloat16_rn(l > 0.f ? __uint_as_float(o[j]) / l : 0.f);
+            orow[(size_t)h * D + ch] = *reinterpret_cast<const uint16_t *>(&bv);
+          }
+        }
+      } else {
+        float *po = a.ws + ((size_t)row * a.nsplit + split) * kHeads * D;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) po[(size_t)(32 * half + j) * D + ch] = __uint_as_float(o[j]);
       }
     }
-    tc_fence_before();
-    __syncthreads();
+    if (a.nsplit > 1 && tid < kHeads) {
+      float *pm = a.ws + nrows * a.nsplit * kHeads * D + ((size_t)row * a.nsplit + split) * kHeads;
+      float *pl = pm + nrows * a.nsplit * kHeads;
+      pm[tid] = S.m_ref[tid];
+      pl[tid] = S.l_run[tid];
+    }
   }
+  tc_fence_before();
+  __syncthreads();
   if (warp == 4) {
     tc_fence_after();
     tmem_dealloc(tmem, kCols);
   }
-}
 
-// out = sum_s 2^(m_s - M) O_s / sum_s 2^(m_s - M) l_s, per (row, head).
-template <int D>
-__global__ void attn_combine_kernel(const AttnArgs a) {
-  const int row = blockIdx.x, h = blockIdx.y;
-  const size_t nrows = (size_t)a.B * a.T_q;
-  const float *pm = a.ws + nrows * a.nsplit * kHeads * D + (size_t)row * a.nsplit * kHeads;
-  const float *pl = pm + nrows * a.nsplit * kHeads;
-  float M = -INFINITY;
-  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, pm[s * kHeads + h]);
-  float L = 0.f;
-  for (int s = 0; s < a.nsplit; ++s) {
-    const float ms = pm[s * kHeads + h];
-    if (ms != -INFINITY) L += exp2f(ms - M) * pl[s * kHeads + h];
-  }
-  const float inv = L > 0.f ? 1.f / L : 0.f;
-  for (int c = threadIdx.x * 4; c < D; c += blockDim.x * 4) {
-    float4 acc = make_float4(0, 0, 0, 0);
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float ms = pm[s * kHeads + h];
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      const float4 v = *reinterpret_cast<const float4 *>(a.ws + (((size_t)row * a.nsplit + s) * kHeads + h) * D + c);
-      acc.x += w * v.x; acc.y += w * v.y; acc.z += w * v.z; acc.w += w * v.w;
+  // ---- merge of the splits (the row's blocks form one cluster)
+  if (a.nsplit > 1) {
+    cluster_sync_all();   // every split's partials are written
+    const size_t nrows = (size_t)a.B * a.T_q;
+    const float *pm = a.ws + nrows * a.nsplit * kHeads * D + (size_t)row * a.nsplit * kHeads;
+    const float *pl = pm + nrows * a.nsplit * kHeads;
+    if (tid < kHeads) {   // all 2 x nsplit loads in flight together
+      float ms[8], ls[8];
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        ms[s] = s < a.nsplit ? __ldcg(pm + s * kHeads + tid) : -INFINITY;
+        ls[s] = s < a.nsplit ? __ldcg(pl + s * kHeads + tid) : 0.f;
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) M = fmaxf(M, ms[s]);
+      float L = 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) {
+        ms[s] = ms[s] == -INFINITY ? 0.f : exp2f(ms[s] - M);
+        L += ms[s] * ls[s];
+      }
+      const float inv = L > 0.f ? 1.f / L : 0.f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s) S.wgt[s][tid] = ms[s] * inv;
     }
-    uint16_t *dst = a.out + ((size_t)row * a.H + h) * D + c;
-    const __nv_bfloat162 v0 = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
-    const __nv_bfloat162 v1 = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
-    uint2 pk;
-    pk.x = *reinterpret_cast<const uint32_t *>(&v0);
-    pk.y = *reinterpret_cast<const uint32_t *>(&v1);
-    *reinterpret_cast<uint2 *>(dst) = pk;
+    __syncthreads();
+    // this split's channel slice, in 4-channel groups
+    const int cs = ((D / a.nsplit) + 7) / 8 * 8;
+    const int c_lo = split * cs;
+    const int c_hi = c_lo + cs < D ? c_lo + cs : D;
+    const int ng = c_hi > c_lo ? (c_hi - c_lo) / 4 : 0;
+    const float *base = a.ws + (size_t)row * a.nsplit * kHeads * D;
+    const int n_items = a.H * ng;
+#pragma unroll 1
+    for (int it0 = tid; it0 < n_items; it0 += 4 * kThreads) {   // 4 items' loads in flight
+      float4 acc[4];
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        const int it = it0 + v * kThreads;
+        if (it < n_items) {
+          const int h = it / ng, ch = c_lo + 4 * (it % ng);
+#pragma unroll
+          for (int s = 0; s < 8; ++s) {
+            if (s < a.nsplit) {
+              const float w = S.wgt[s][h];
+              const float4 x = __ldcg(reinterpret_cast<const float4 *>(base + ((size_t)s * kHeads + h) * D + ch));
+              acc[v].x += w * x.x; acc[v].y += w * x.y; acc[v].z += w * x.z; acc[v].w += w * x.w;
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int it = it0 + v * kThreads;
+        if (it < n_items) {
+          const int h = it / ng, ch = c_lo + 4 * (it % ng);
+          const __nv_bfloat162 v0 = __floats2bfloat162_rn(acc[v].x, acc[v].y);
+          const __nv_bfloat162 v1 = __floats2bfloat162_rn(acc[v].z, acc[v].w);
+          uint2 pk;
+          pk.x = *reinterpret_cast<const uint32_t *>(&v0);
+          pk.y = *reinterpret_cast<const uint32_t *>(&v1);
+          *reinterpret_cast<uint2 *>(a.out + ((size_t)row * a.H + h) * D + ch) = pk;
+        }
+      }
+    }
   }
 }
 
@@ -476,6 +523,7 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   if (rows < sms) {
     nsplit = (2 * sms + rows - 1) / rows;
     if (nsplit > nc) nsplit = nc;
+    if (nsplit > 8) nsplit = 8;   // one cluster per row
   }
   const int cps = (nc + nsplit - 1) / nsplit;
   nsplit = (nc + cps - 1) / cps;
@@ -490,11 +538,19 @@ static cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s) {
   const size_t smem = sizeof(AttnSmem<D>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  attn_kernel<D><<<dim3(a.B * a.T_q, a.nsplit), kThreads, smem, s>>>(a);
-  e = cudaGetLastError();
-  if (e != cudaSuccess || a.nsplit == 1) return e;
-  attn_combine_kernel<D><<<dim3(a.B * a.T_q, a.H), D / 4 < 128 ? D / 4 : 128, 0, s>>>(a);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(a.B * a.T_q, a.nsplit);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)a.nsplit;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = a.nsplit > 1 ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, attn_kernel<D>, a);
 }
 
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s) {

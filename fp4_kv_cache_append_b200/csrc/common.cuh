@@ -61,6 +61,31 @@ __device__ __forceinline__ float e2m1_to_f32(uint32_t c) {
   return (c & 8u) ? -mag : mag;
 }
 
+// ------------------------------------------------------------------ hardware converts (exact)
+
+// Eight E2M1 codes (one 32-bit word; each byte holds a channel pair, low
+// nibble = even channel) -> four f16x2 (low half = even channel).
+__device__ __forceinline__ void e2m1x8_to_f16x2(uint32_t w, uint32_t *h) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\tmov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\tcvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\tcvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(w));
+}
+// Four E4M3 bytes (one 32-bit word, low byte first) -> two f16x2.
+__device__ __forceinline__ void e4m3x4_to_f16x2(uint32_t w, uint32_t *h) {
+  asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+      : "=r"(h[0]), "=r"(h[1])
+      : "r"(w));
+}
+// Two E4M3 bytes (low 16 bits) -> one f16x2.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
+  uint32_t h;
+  asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}" : "=r"(h) : "r"(w));
+  return h;
+}
+
 // ------------------------------------------------------------------ status
 
 __device__ __forceinline__ void flag(unsigned int *status, unsigned int bit) {

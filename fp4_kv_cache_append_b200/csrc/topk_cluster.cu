@@ -13,11 +13,13 @@
 // found by levels of 512-bin histograms:
 //   * level 0 bins by VALUE, linearly between the row's smallest and largest
 //     score, so scores concentrated in a few binades still spread over many
-//     bins; the bin holding the K-th key is then turned into an exact key
-//     interval by a 32-way search over keys (bins are monotone in the key);
-//   * further levels bin by key bits inside that interval;
+//     bins;
 //   * a bin holding the K-th key with at most 256 keys is resolved exactly:
 //     its keys are collected in block 0 and ranked (score desc, column asc);
+//     as the bins are monotone in the key, that key and its column decide
+//     every column of the row;
+//   * a larger level-0 bin is turned into an exact key interval by a 32-way
+//     search over keys, and further levels bin by key bits inside it;
 //   * a single-valued bin with more keys shares its ties out in column order.
 // Per level the block histograms are pushed into the owning block's slice
 // (block r owns bins [64r, 64r+64)) with distributed-shared-memory atomics
@@ -63,6 +65,8 @@ enum : int { kActive = 0, kCollect = 1, kDone = 2 };
 struct Sel {
   int state;
   bool vs;            // the current level bins by value (level 0)
+  bool vreg;          // the region is value bin T0 (else the key interval [lo, hi])
+  int T0;
   float v_lo, inv;    // value bin = clamp((v - v_lo) * inv)
   uint32_t g_lo, g_hi;
   uint32_t lo, hi;    // key interval of the current level's region
@@ -238,6 +242,8 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
       l.cmode = true;
       l.take_eq = 0;
       l.vs = false;
+      l.vreg = false;
+      l.T0 = 0;
       l.v_lo = 0.f;
       l.inv = 0.f;
       l.shift = 0;
@@ -315,24 +321,31 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
       Sel &l = sh.sel[warp];
       const int T = sh.th[warp][0], cntT = sh.th[warp][2];
       const int need2 = l.need - sh.th[warp][1];   // 1 <= need2 <= cntT
-      uint32_t lo_T, hi_T;
-      if (l.vs) {   // exact key interval of value bin T
-        lo_T = T == 0 ? l.g_lo : first_key_of_bin(l.v_lo, l.inv, l.g_lo, l.g_hi, T, lane);
-        hi_T = T == kBins - 1 ? l.g_hi : first_key_of_bin(l.v_lo, l.inv, l.g_lo, l.g_hi, T + 1, lane) - 1u;
+      if (l.vs && cntT <= kCand) {
+        // rank the keys of value bin T exactly (no key interval needed: the
+        // bins are monotone in the key, so the need2-th key of the bin and its
+        // column decide every key of the row)
+        if (lane == 0) { l.vreg = true; l.T0 = T; l.need = need2; l.cnt = cntT; l.state = kCollect; }
       } else {
-        lo_T = l.lo + ((uint32_t)T << l.shift);
-        const uint32_t w1 = (1u << l.shift) - 1u;
-        hi_T = (l.hi - lo_T > w1) ? lo_T + w1 : l.hi;
-      }
-      if (lane == 0) {
-        if (cntT == need2) {                 // every key of the bin is taken
-          l.kthr = lo_T - 1u; l.cthr = -1; l.cmode = true; l.state = kDone;
-        } else if (cntT <= kCand) {          // rank the bin's keys exactly
-          l.lo = lo_T; l.hi = hi_T; l.need = need2; l.cnt = cntT; l.vs = false; l.state = kCollect;
-        } else if (!l.vs && l.shift == 0) {  // one key value: need2 of its ties, in column order
-          l.kthr = lo_T; l.cmode = false; l.take_eq = need2; l.state = kDone;
-        } else {                             // next level inside the bin
-          l.lo = lo_T; l.hi = hi_T; l.shift = key_shift(lo_T, hi_T); l.need = need2; l.vs = false;
+        uint32_t lo_T, hi_T;
+        if (l.vs) {   // exact key interval of value bin T
+          lo_T = T == 0 ? l.g_lo : first_key_of_bin(l.v_lo, l.inv, l.g_lo, l.g_hi, T, lane);
+          hi_T = T == kBins - 1 ? l.g_hi : first_key_of_bin(l.v_lo, l.inv, l.g_lo, l.g_hi, T + 1, lane) - 1u;
+        } else {
+          lo_T = l.lo + ((uint32_t)T << l.shift);
+          const uint32_t w1 = (1u << l.shift) - 1u;
+          hi_T = (l.hi - lo_T > w1) ? lo_T + w1 : l.hi;
+        }
+        if (lane == 0) {
+          if (cntT == need2) {                 // every key of the bin is taken
+            l.kthr = lo_T - 1u; l.cthr = -1; l.cmode = true; l.state = kDone;
+          } else if (cntT <= kCand) {          // rank the bin's keys exactly
+            l.lo = lo_T; l.hi = hi_T; l.need = need2; l.cnt = cntT; l.vs = false; l.state = kCollect;
+          } else if (!l.vs && l.shift == 0) {  // one key value: need2 of its ties, in column order
+            l.kthr = lo_T; l.cmode = false; l.take_eq = need2; l.state = kDone;
+          } else {                             // next level inside the bin
+            l.lo = lo_T; l.hi = hi_T; l.shift = key_shift(lo_T, hi_T); l.need = need2; l.vs = false;
+          }
         }
       }
     }
@@ -345,11 +358,16 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
       const Sel &l = sh.sel[s];
       if (l.state != kCollect) continue;
       const uint32_t lo = l.lo, hi = l.hi;
+      const bool vreg = l.vreg;
+      const int T0 = l.T0;
+      const float v_lo = l.v_lo, inv = l.inv;
+      bool in[kN];
       int m = 0;
 #pragma unroll
       for (int k = 0; k < kN; ++k) {
         const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
-        m += kk && kk >= lo && kk <= hi;
+        in[k] = kk && (vreg ? vbin(v_lo, inv, kk) == T0 : (kk >= lo && kk <= hi));
+        m += in[k];
       }
       const int incl = warp_incl_scan(m, lane);
       const int wtot = __shfl_sync(0xffffffffu, incl, 31);
@@ -360,7 +378,7 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
 #pragma unroll
       for (int k = 0; k < kN; ++k) {
         const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
-        if (kk && kk >= lo && kk <= hi) {
+        if (in[k]) {
           if (pos < kCand) dst[pos] = make_uint2(kk, (uint32_t)(s == 0 ? c0 + k : blk));
           ++pos;
         }
@@ -401,7 +419,7 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
   const uint32_t kthr0 = sh.sel[0].kthr, kthr1 = sh.sel[1].kthr;
   const int cthr0 = sh.sel[0].cthr, cthr1 = sh.sel[1].cthr;
   const bool cm0 = sh.sel[0].cmode, cm1 = sh.sel[1].cmode;
-  int tie_base0, tie_base1;
+  int tie_base0, tie_base1, pos0, pos1;
   {
     int t0 = 0, s0 = 0;
 #pragma unroll
@@ -417,6 +435,8 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
     const unsigned long long ex = block_scan<unsigned long long>(v, sh.red, lane, warp);
     tie_base0 = (int)(ex & 0xFFFFu);
     tie_base1 = (int)((ex >> 32) & 0xFFFFu);
+    pos0 = (int)((ex >> 16) & 0xFFFFu);   // the output positions when no tie is shared by count
+    pos1 = (int)((ex >> 48) & 0xFFFFu);
     if (tid == 0) {
       const unsigned long long tot = sh.red[31];
       sh.cnt[0] = (int)(tot & 0xFFFFu);
@@ -464,9 +484,13 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
     const bool tie1 = nsel > 1 && bkey && !cm1 && bkey == kthr1;
     const bool take1 = (nsel > 1 && bkey && (bkey > kthr1 || (cm1 && bkey == kthr1 && blk <= cthr1))) ||
                        (tie1 && tie_base1 < allow1);
-    const uint32_t ex = block_scan<uint32_t>((uint32_t)n0 | ((uint32_t)take1 << 16), reinterpret_cast<uint32_t *>(sh.red),
-                                             lane, warp);
-    int o = sh.base[0] + (int)(ex & 0xFFFFu);
+    if (!(cm0 && cm1)) {   // ties shared by count: positions from the final counts (block-uniform)
+      const uint32_t ex = block_scan<uint32_t>((uint32_t)n0 | ((uint32_t)take1 << 16),
+                                               reinterpret_cast<uint32_t *>(sh.red), lane, warp);
+      pos0 = (int)(ex & 0xFFFFu);
+      pos1 = (int)(ex >> 16);
+    }
+    int o = sh.base[0] + pos0;
     int32_t *out = a.out_idx + (size_t)row * a.K;
     const int32_t *pb = a.pool_blocks ? a.pool_blocks + (size_t)row * (a.n_cols / 8) : nullptr;
     tr = tie_base0;
@@ -482,7 +506,7 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
       }
     }
     if (take1) {
-      const int o1 = sh.base[1] + (int)(ex >> 16);
+      const int o1 = sh.base[1] + pos1;
       if (o1 < a.P_out) a.out_pool[(size_t)row * a.P_out + o1] = blk;
     }
     if (r == kCl - 1) {
