@@ -195,18 +195,26 @@ def run_ours(args, rank, world, dist):
     torch.cuda.synchronize()
     assert C.csa2_device_status() == 0
 
-    # ---- graph of `rot` rotations over the cache copies, events around each call
+    # ---- graphs of `rot` rotations over the cache copies: the headline graph
+    # has nothing between the calls (consecutive kernels overlap their launch
+    # with the previous kernel's tail); the breakdown graph records events
+    # around every call for the per-kernel durations and the roofline.
     rot = max(1, args.graph_rotations)
     steps_per_graph = rot * args.copies
-    events = {}
-    g = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(side):
         st.run(copy=0)   # one more eager call on the capture stream
     torch.cuda.current_stream().wait_stream(side)
     torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
+        for r in range(rot):
+            for cp in range(args.copies):
+                st.run(copy=cp)
+    events = {}
+    g_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ev):
         for r in range(rot):
             for cp in range(args.copies):
                 st.run(copy=cp, events=events, external_events=True)
@@ -214,6 +222,7 @@ def run_ours(args, rank, world, dist):
     K = n_graph * steps_per_graph
     for _ in range(max(3, args.warmup)):
         g.replay()
+        g_ev.replay()
     torch.cuda.synchronize()
 
     gpu_id = None
@@ -228,7 +237,7 @@ def run_ours(args, rank, world, dist):
         if dist is not None:
             dist.barrier()
 
-    # ---- timed region
+    # ---- timed region (headline)
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     sampler = ClockSampler(gpu_id) if rank == 0 else None
     if sampler:
@@ -246,7 +255,19 @@ def run_ours(args, rank, world, dist):
     ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
     assert C.csa2_device_status() == 0, "device status flagged during the timed region"
 
-    # per-entry-point durations: the event pairs of the last replay of the timed region
+    # ---- timed region (breakdown): same steps with events around every call;
+    # per-entry-point durations are the event pairs of its last replay
+    n_ev = max(1, n_graph // 4)
+    barrier()
+    torch.cuda.synchronize()
+    t2, t3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t2.record()
+    for _ in range(n_ev):
+        g_ev.replay()
+    t3.record()
+    torch.cuda.synchronize()
+    barrier()
+    ms_ev = t2.elapsed_time(t3) / (n_ev * steps_per_graph)
     kern_us = {k: statistics.mean(s.elapsed_time(e) for s, e in v) * 1e3 for k, v in events.items()}
     calls_per_step = {k: len(v) / steps_per_graph for k, v in events.items()}
 
@@ -261,11 +282,13 @@ def run_ours(args, rank, world, dist):
     step_bytes = sum(alg.values()) + B * (wl.D + wl.D) * 2 + B * (wl.D // 2 + wl.D // 16 + wl.dI + 4)
     idx_bytes = B * n * (wl.dI + 4)                        # 132 B per visible entry
     hbm, hbm_kind = peaks()
-    dom = max(kern_us, key=lambda k: kern_us[k] * calls_per_step[k])
-    dom_bytes = {"index_full": idx_bytes, "attn": alg.get("attn", 0)}.get(dom)
-    achieved = dom_bytes / (kern_us[dom] * 1e-6) / 1e9 if dom_bytes else None
-    traffic = ncu_traffic(f"index_full_{WORKLOAD}") if dom == "index_full" else None
-    launches_per_step = 6 if st.ws_attn is not None else 5
+    # dominant kernel = the one that moves the step's bytes (the Full scan:
+    # 132 B per visible entry, ~96% of the step's algorithmic bytes)
+    dom = "index_full"
+    dom_bytes = idx_bytes
+    achieved = dom_bytes / (kern_us[dom] * 1e-6) / 1e9
+    traffic = ncu_traffic(f"index_full_{WORKLOAD}")
+    launches_per_step = st.launches_per_step()
     clocks = sampler.summary() if sampler else None
     return {
         "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world, "steps": K,
@@ -279,6 +302,7 @@ def run_ours(args, rank, world, dist):
         "step_bytes": step_bytes, "step_gbs": step_bytes * steps_per_s / world / 1e9,
         "step_frac_hbm": step_bytes * steps_per_s / world / 1e9 / hbm,
         "kernels_us": {k: round(v, 3) for k, v in kern_us.items()},
+        "ms_per_step_with_events": ms_ev,
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm,
                      "peak_kind": hbm_kind, "unit": "GB/s", "frac": achieved / hbm if achieved else None,
                      "traffic": traffic, "bytes_per_launch": dom_bytes,

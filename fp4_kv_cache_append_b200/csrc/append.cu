@@ -221,6 +221,8 @@ __device__ void append_window_row(const AppendArgs &a, int b, int r) {
 
 __global__ void append_kernel(const AppendArgs a) {
   extern __shared__ float sm[];
+  pdl_launch_dependents();
+  pdl_wait();
   const int nm = a.B * a.main_blocks_per_seq;
   if ((int)blockIdx.x < nm) {
     append_entries(a, blockIdx.x / a.main_blocks_per_seq,
@@ -241,8 +243,7 @@ cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
                               : 0;
   cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  append_kernel<<<blocks, threads, smem, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(append_kernel, dim3(blocks), dim3(threads), smem, s, dim3(1, 1, 1), a);
 }
 
 }  // namespace csa2

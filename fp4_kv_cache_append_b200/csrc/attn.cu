@@ -128,6 +128,20 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   const int row = blockIdx.x;   // b * T_q + query
   const int split = blockIdx.y;
   const int b = row / a.T_q;
+  pdl_launch_dependents();
+
+  // ---- set-up that touches no global memory overlaps the previous kernel
+  if (tid == 0) {
+    mbar_init(&S.sbar, 1);
+    mbar_init(&S.obar, 1);
+    S.rescale = 0;
+    fence_barrier_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(&S.tmem_base, kCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
   const int t = a.q_pos[row];
 
   // ---- keys of this split
@@ -140,17 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   int c_end = c_begin + a.chunks_per_split;
   if (c_end > total) c_end = total;
 
-  // ---- set-up; Q loads and the first tile's key ids are issued together
-  if (tid == 0) {
-    mbar_init(&S.sbar, 1);
-    mbar_init(&S.obar, 1);
-    S.rescale = 0;
-    fence_barrier_init();
-  }
-  if (warp == 4) {
-    tmem_alloc(&S.tmem_base, kCols);
-    tmem_relinquish();
-  }
+  // ---- Q loads and the first tile's key ids are issued together
   uint4 qraw[QI];
   {
     const uint16_t *qrow = a.q + (size_t)row * a.H * D;
@@ -538,19 +542,8 @@ static cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s) {
   const size_t smem = sizeof(AttnSmem<D>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(a.B * a.T_q, a.nsplit);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = (unsigned)a.nsplit;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = a.nsplit > 1 ? 1 : 0;
-  return cudaLaunchKernelEx(&cfg, attn_kernel<D>, a);
+  return launch_pdl(attn_kernel<D>, dim3(a.B * a.T_q, a.nsplit), dim3(kThreads), smem, s, dim3(1, (unsigned)a.nsplit, 1),
+                    a);
 }
 
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s) {

@@ -86,6 +86,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w) {
   return h;
 }
 
+// ------------------------------------------------------------------ programmatic dependent launch
+// Kernels launched with programmatic stream serialisation start while the
+// previous kernel of the stream drains: pdl_wait() returns once that grid has
+// completed and its memory is visible (a no-op without the attribute), and
+// pdl_launch_dependents() lets the next kernel of the stream launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------------ status
 
 __device__ __forceinline__ void flag(unsigned int *status, unsigned int bit) {

@@ -72,6 +72,8 @@ template <int DI>
 __global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
   constexpr int MASK = DI == 128 ? 7 : 3;
   const int row = blockIdx.x, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  pdl_wait();
   const uint16_t *qrow = a.q_idx + (size_t)row * a.H_I * DI;
   const float *wrow = a.w + (size_t)row * a.H_I;
   uint8_t *q8 = a.q8 + (size_t)row * kHeads * DI;
@@ -112,6 +114,7 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.y;   // b * T_q + query
   const int b = row / a.T_q;
+  pdl_wait();
   const int t = a.q_pos[row];
   int n_vis = (t + 1) / a.m;
   const int ne = a.n_entries[b];
@@ -262,6 +265,7 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
 
   // ---- teardown: on an abort, drain in-flight copies and MMAs (bounded),
   // then free TMEM
+  pdl_launch_dependents();
   __syncthreads();
   if (S.abort) {
     if (tid == 0) {
@@ -289,16 +293,14 @@ size_t index_workspace_bytes(int rows, int dI) {
 
 template <int DI, bool REINDEX>
 static cudaError_t launch_t(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
-  index_prep_kernel<DI><<<dim3(a.B * a.T_q, kHeads / 8), 256, 0, s>>>(a);
-  cudaError_t pe = cudaGetLastError();
+  cudaError_t pe = launch_pdl(index_prep_kernel<DI>, dim3(a.B * a.T_q, kHeads / 8), dim3(256), 0, s, dim3(1, 1, 1), a);
   if (pe != cudaSuccess) return pe;
   const size_t smem = sizeof(IndexSmem<DI>) + 1024;
   auto k = index_kernel<DI, REINDEX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((a.tiles_per_row + a.tiles_per_cta - 1) / a.tiles_per_cta, a.B * a.T_q);
-  k<<<grid, kThreads, smem, s>>>(map, a);
-  return cudaGetLastError();
+  return launch_pdl(k, grid, dim3(kThreads), smem, s, dim3(1, 1, 1), map, a);
 }
 
 cudaError_t launch_index(const CUtensorMap &map, const IndexArgs &a, bool reindex, int sms, cudaStream_t s) {

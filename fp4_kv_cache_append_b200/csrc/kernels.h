@@ -1,6 +1,7 @@
 // Host-side launchers of the libcsa2 kernels (internal; the public ABI is
 // include/csa2.h).  Each returns the cudaError_t of its launch.
 #pragma once
+#include <utility>
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -51,6 +52,33 @@ struct IndexArgs {
 size_t index_workspace_bytes(int rows, int dI);
 cudaError_t launch_index(const CUtensorMap &ik_map, const IndexArgs &a, bool reindex, int sms,
                          cudaStream_t s);
+
+// Launch with programmatic stream serialisation (and an optional cluster
+// shape): the kernel may start while the stream's previous kernel drains and
+// synchronises with it through pdl_wait().
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              dim3 cluster, Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster.x * cluster.y * cluster.z > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster.x;
+    attr[1].val.clusterDim.y = cluster.y;
+    attr[1].val.clusterDim.z = cluster.z;
+    n = 2;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 struct TopkArgs {
   const float *scores;

@@ -159,14 +159,16 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
   cg::cluster_group cl = cg::this_cluster();
   const int r = (int)cl.block_rank();
   const int row = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int c0 = r * kSpan + tid * kN;   // this thread's first column
+  const int blk = c0 >> 3;               // its pool block
+  const int nsel = a.P_out > 0 ? 2 : 1;
+  pdl_launch_dependents();
+  pdl_wait();
   int ncol = a.n_cols;
   if (a.n_valid) {
     const int v = a.n_valid[row];
     if (v < ncol) ncol = v < 0 ? 0 : v;
   }
-  const int c0 = r * kSpan + tid * kN;   // this thread's first column
-  const int blk = c0 >> 3;               // its pool block
-  const int nsel = a.P_out > 0 ? 2 : 1;
 
   // ---- keys (both 16-byte loads are issued before either is used)
   uint32_t key[kN];
@@ -522,8 +524,7 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
 bool topk_cluster_fits(int n_cols) { return n_cols <= kCl * kSpan; }
 
 cudaError_t launch_topk_cluster(const TopkArgs &a, cudaStream_t s) {
-  topk_cluster_kernel<<<dim3(kCl, a.rows), kT, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_pdl(topk_cluster_kernel, dim3(kCl, a.rows), dim3(kT), 0, s, dim3(1, 1, 1), a);
 }
 
 }  // namespace csa2

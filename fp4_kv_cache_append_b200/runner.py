@@ -192,6 +192,21 @@ class Step:
 
     # ------------------------------------------------------------------ accounting
 
+    def launches_per_step(self) -> int:
+        """libcsa2 kernel launches one step enqueues (append 1, index 2 =
+        query prep + scan, Top-K 1 for rows of up to 65,536 columns else 4,
+        attention 1)."""
+        wl = self.wl
+        topk = lambda n_cols: 1 if n_cols <= 65536 else 4
+        n = 0
+        for kind, _ in self.plan:
+            n += 1 + 1   # append, attention
+            if kind == "full":
+                n += 2 + topk(self.cap)
+            elif kind == "reindex":
+                n += 2 + topk(wl.P * 8)
+        return n
+
     def algorithmic_bytes(self) -> dict:
         """Bytes each entry point must move per step (cold caches)."""
         wl, B, D = self.wl, self.wl.B, self.wl.D
