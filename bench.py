@@ -67,20 +67,27 @@ def peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+INDEX_SOURCES = ("index.cu", "common.cuh", "kernels.h")   # what builds the index kernels
+
+
+def source_sha(names=INDEX_SOURCES) -> str:
+    """Hash of the sources a kernel is built from (first 16 hex digits)."""
+    import hashlib
+    src = os.path.join(ROOT, "fp4_kv_cache_append_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(names):
+        with open(os.path.join(src, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
 def ncu_traffic(kernel_tag: str):
     """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
     summary was taken on the current kernel source (else None)."""
-    import hashlib
     summ = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
     if not os.path.exists(summ):
         return None
-    src = os.path.join(ROOT, "fp4_kv_cache_append_b200", "csrc")
-    h = hashlib.sha256()
-    for name in sorted(os.listdir(src)):
-        if name.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(src, name), "rb") as f:
-                h.update(f.read())
-    want = h.hexdigest()[:16]
+    want = source_sha()
     sha = traffic = None
     with open(summ) as f:
         for line in f:
