@@ -152,6 +152,10 @@ def csa2_index_workspace_size(rows: int, d_I: int) -> int:
     return int(lib().csa2_index_workspace_size(rows, d_I))
 
 
+def _nbytes(t) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def _ws_or_alloc(ws, nbytes, device):
     """A caller workspace, or a fresh one of the needed size (binding convenience)."""
     if ws is None:
@@ -165,8 +169,8 @@ def csa2_index_full(main: MainCache, q_idx, w, q_pos, scores, n_valid=None, ws=N
     ws = _ws_or_alloc(ws, csa2_index_workspace_size(main.B * T_q, main.d_I), scores.device)
     _check(lib().csa2_index_full(ctypes.byref(main.desc()), _ptr(q_idx, torch.bfloat16), _ptr(w, torch.float32),
                                  _ptr(q_pos, torch.int32), T_q, H_I, _ptr(scores, torch.float32),
-                                 scores.shape[-1], _ptr(n_valid, torch.int32), _ptr(ws),
-                                 ws.numel() * ws.element_size(), _stream(stream)))
+                                 scores.shape[-1], _ptr(n_valid, torch.int32), _ptr(ws), _nbytes(ws),
+                                 _stream(stream)))
 
 
 def csa2_index_reindex(main: MainCache, q_idx, w, q_pos, pool_blocks, pool_scores, ws=None, stream=None):
@@ -176,7 +180,7 @@ def csa2_index_reindex(main: MainCache, q_idx, w, q_pos, pool_blocks, pool_score
     _check(lib().csa2_index_reindex(ctypes.byref(main.desc()), _ptr(q_idx, torch.bfloat16), _ptr(w, torch.float32),
                                     _ptr(q_pos, torch.int32), T_q, H_I, _ptr(pool_blocks, torch.int32),
                                     pool_blocks.shape[-1], _ptr(pool_scores, torch.float32), _ptr(ws),
-                                    ws.numel() * ws.element_size(), _stream(stream)))
+                                    _nbytes(ws), _stream(stream)))
 
 
 def csa2_topk_workspace_size(rows: int, n_cols: int, K: int, P_out: int = 0) -> int:

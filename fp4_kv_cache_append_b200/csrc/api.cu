@@ -211,6 +211,15 @@ csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, c
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "append launch");
 }
 
+// Blocks per row of a scan: about three resident blocks per SM in one wave,
+// the row's tiles split evenly over them.
+static int index_ctas_per_row(int tiles_per_row, int rows, int sms) {
+  int64_t c = (int64_t)sms * 3 / rows;
+  if (c < 1) c = 1;
+  if (c > tiles_per_row) c = tiles_per_row;
+  return (int)c;
+}
+
 static csa2_status index_common(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                                 const int32_t *q_pos, int T_q, int H_I, float *scores, void *ws, size_t ws_bytes,
                                 IndexArgs *a, CUtensorMap *map, int box_rows) {
@@ -255,13 +264,7 @@ csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, 
   if ((st = device_state(&d)) != CSA2_OK) return st;
   a.ld = ld; a.n_valid = n_valid; a.status = d->status;
   a.tiles_per_row = main->cap / 128;
-  // about three resident blocks per SM in one wave
-  const int64_t total = (int64_t)a.tiles_per_row * main->B * T_q;
-  int64_t target = (int64_t)d->sms * 3;
-  int64_t tpc = (total + target - 1) / target;
-  if (tpc < 1) tpc = 1;
-  if (tpc > a.tiles_per_row) tpc = a.tiles_per_row;
-  a.tiles_per_cta = (int)tpc;
+  a.ctas_per_row = index_ctas_per_row(a.tiles_per_row, main->B * T_q, d->sms);
   cudaError_t e = launch_index(map, a, false, d->sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
 }
@@ -280,12 +283,7 @@ csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_id
   if ((st = device_state(&d)) != CSA2_OK) return st;
   a.ld = (int64_t)P * 8; a.pool = pool_blocks; a.P = P; a.status = d->status;
   a.tiles_per_row = P / 16;
-  const int64_t total = (int64_t)a.tiles_per_row * main->B * T_q;
-  int64_t target = (int64_t)d->sms * 3;
-  int64_t tpc = (total + target - 1) / target;
-  if (tpc < 1) tpc = 1;
-  if (tpc > a.tiles_per_row) tpc = a.tiles_per_row;
-  a.tiles_per_cta = (int)tpc;
+  a.ctas_per_row = index_ctas_per_row(a.tiles_per_row, main->B * T_q, d->sms);
   cudaError_t e = launch_index(map, a, true, d->sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_reindex launch");
 }

@@ -10,8 +10,12 @@
 // and one block per window row.  The quantised bytes are
 // decided in binary32 with IEEE division, no contraction (explicit _rn
 // intrinsics), so they are reproducible bit for bit.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
+
+namespace cg = cooperative_groups;
 
 namespace csa2 {
 
@@ -233,7 +237,132 @@ __global__ void append_kernel(const AppendArgs a) {
   }
 }
 
+// Decode (one new token per sequence, m = 1): a cluster of 8 blocks per
+// sequence.  Every block quantises the new entry (the same binary32 steps as
+// append_entries, so all blocks hold the same x^); block c projects indexer
+// outputs [c*dI/8, (c+1)*dI/8) from its slice of W_ik and writes 1/8 of the
+// window row; the FP8 key scale needs the maximum over all outputs, which the
+// blocks push into each other's shared memory before one cluster barrier.
+// Block 0 writes the FP4 codes, the scales, the key scale and n_entries.
+constexpr int kDecCl = 8;
+
+__global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_decode_kernel(const AppendArgs a) {
+  __shared__ float xh[512];
+  __shared__ alignas(16) uint16_t wsl[512 * 16];   // W_ik[:, c*OPB .. c*OPB+OPB), row-major [D][OPB]
+  __shared__ float part[16 * 16];                  // [G][OPB] chain partials
+  __shared__ float kmx[kDecCl];                    // the blocks' local key maxima
+  cg::cluster_group cl = cg::this_cluster();
+  const int c = (int)cl.block_rank();
+  const int b = blockIdx.y, t = threadIdx.x;
+  const int D = a.D, dI = a.dI, G = D / 32, OPB = dI / kDecCl;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int p0 = a.pos0[b];
+  if (p0 < 0) {   // the same in every block of the cluster: none of them waits
+    if (t == 0 && c == 0) flag(a.status, CSA2_DEV_BAD_POSITION);
+    return;
+  }
+  const int e = p0;   // m = 1: token p0 completes entry p0
+  // ---- loads: this block's W_ik slice (16-byte pieces), the entry's kv pair, its window pair
+  {
+    const int ppr = OPB * 2 / 16;   // 16-byte pieces per W row of the slice
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.w_ik);
+    uint4 *dst = reinterpret_cast<uint4 *>(wsl);
+    for (int i = t; i < D * ppr; i += blockDim.x) {
+      const int r = i / ppr, j = i % ppr;
+      dst[i] = src[((size_t)r * dI + c * OPB) * 2 / 16 + j];
+    }
+  }
+  uint32_t kvp = 0u, swp = 0u;
+  if (t < D / 2) kvp = reinterpret_cast<const uint32_t *>(a.kv + (size_t)b * D)[t];
+  const int wch = D / (2 * kDecCl);   // window channel pairs per block
+  if (a.swa_rows && t < wch) swp = reinterpret_cast<const uint32_t *>(a.kv_swa + (size_t)b * D)[c * wch + t];
+
+  // ---- FP4: thread t < D/2 owns channels 2t, 2t+1 (8 threads per 16-channel group)
+  if (t < D / 2) {
+    const float x0 = bf16_to_f32((uint16_t)(kvp & 0xFFFFu)), x1 = bf16_to_f32((uint16_t)(kvp >> 16));
+    float amax = fmaxf(fabsf(x0), fabsf(x1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    uint32_t sb = amax == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+    const float sc = e4m3_to_f32(sb);
+    uint32_t c0 = 0, c1 = 0;
+    if (sc != 0.0f) {
+      c0 = f32_to_e2m1(__fdiv_rn(x0, sc));
+      c1 = f32_to_e2m1(__fdiv_rn(x1, sc));
+    } else {
+      sb = 0;
+    }
+    if (c == 0) {
+      if (e < a.cap) {
+        const size_t row = (size_t)b * a.cap + e;
+        a.codes[row * (D / 2) + t] = (uint8_t)(c0 | (c1 << 4));
+        if ((t & 7) == 0) a.scales[row * (D / 16) + (t >> 3)] = (uint8_t)sb;
+      } else if (t == 0) {
+        flag(a.status, CSA2_DEV_APPEND_RANGE);
+      }
+    }
+    xh[2 * t] = __fmul_rn(e2m1_to_f32(c0), sc);
+    xh[2 * t + 1] = __fmul_rn(e2m1_to_f32(c1), sc);
+  }
+  // ---- window: channels [2*wch*c, 2*wch*(c+1)) of the ring slot p0 mod W_cap
+  if (a.swa_rows && t < wch) {
+    const uint32_t lo = f32_to_e4m3(__fdiv_rn(bf16_to_f32((uint16_t)(swp & 0xFFFFu)), a.s_swa));
+    const uint32_t hi = f32_to_e4m3(__fdiv_rn(bf16_to_f32((uint16_t)(swp >> 16)), a.s_swa));
+    uint8_t *dst = a.swa_rows + ((size_t)b * a.W_cap + (p0 % a.W_cap)) * D;
+    reinterpret_cast<uint16_t *>(dst)[c * wch + t] = (uint16_t)(lo | (hi << 8));
+  }
+  __syncthreads();
+  // ---- indexer key: thread (o, g) forms the 32-channel fmaf chain of group g
+  // for output c*OPB + o (ascending channels from +0), as append_entries does
+  if (t < OPB * G) {
+    const int o = t % OPB, g = t / OPB;
+    const float *xg = xh + 32 * g;
+    const uint16_t *wcol = wsl + (32 * g) * OPB + o;
+    float acc = 0.0f;
+#pragma unroll
+    for (int cc = 0; cc < 32; ++cc) acc = __fmaf_rn(xg[cc], bf16_to_f32(wcol[cc * OPB]), acc);
+    part[g * OPB + o] = acc;
+  }
+  __syncthreads();
+  float k = 0.0f;
+  if (t < 32) {
+    if (t < OPB) {   // group sums added pairwise, level by level
+      int n = G;
+      float v[16];
+#pragma unroll
+      for (int g = 0; g < 16; ++g) v[g] = g < G ? part[g * OPB + t] : 0.0f;
+      while (n > 1) {
+        const int h = n >> 1;
+        for (int q = 0; q < h; ++q) v[q] = __fadd_rn(v[2 * q], v[2 * q + 1]);
+        if (n & 1) { v[h] = v[n - 1]; n = h + 1; } else n = h;
+      }
+      k = v[0];
+    }
+    float m = t < OPB ? fabsf(k) : 0.0f;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (t < kDecCl) *cl.map_shared_rank(&kmx[c], t) = m;   // push into every block
+  }
+  cl.sync();
+  if (t < OPB) {
+    float kmax = kmx[0];
+#pragma unroll
+    for (int r = 1; r < kDecCl; ++r) kmax = fmaxf(kmax, kmx[r]);
+    const float sk = __fdiv_rn(kmax, 448.0f);
+    if (e < a.cap) {
+      const size_t row = (size_t)b * a.cap + e;
+      a.ik[row * dI + c * OPB + t] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(k, sk)));
+      if (c == 0 && t == 0) a.ik_scale[row] = sk;
+    }
+  }
+  if (c == 0 && t == 0) a.n_entries[b] = p0 + 1;
+}
+
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
+  if (a.codes && a.m == 1 && a.T == 1 && a.D <= 512 && a.dI % (8 * kDecCl) == 0 && a.dI / kDecCl <= 16 &&
+      (!a.swa_rows || a.W_cap >= 1))
+    return launch_pdl(append_decode_kernel, dim3(kDecCl, a.B), dim3(256), 0, s, dim3(1, 1, 1), a);
   const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq);
   if (blocks == 0) return cudaSuccess;
   const int threads = 512;   // quantisation uses the first D/2, the projection all of them

@@ -79,6 +79,14 @@ __device__ __forceinline__ void reduce_scatter32(float *t, int lane) {
   }
 }
 
+// 2^x by the hardware's approximate exponential (relative error ~2^-22,
+// far below the fp16 rounding of P it feeds).
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ int ordered(float f) {
   const int b = __float_as_int(f);
   return b >= 0 ? b : (b ^ 0x7FFFFFFF);
@@ -339,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const int j = 4 * j4 + k;
-          sv[j] = (sv[j] == -INFINITY || mm[k] == -INFINITY) ? 0.f : exp2f(sv[j] - mm[k]);
+          sv[j] = (sv[j] == -INFINITY || mm[k] == -INFINITY) ? 0.f : ex2_approx(sv[j] - mm[k]);
         }
         const __half2 h0 = __floats2half2_rn(sv[4 * j4] * psc, sv[4 * j4 + 1] * psc);
         const __half2 h1 = __floats2half2_rn(sv[4 * j4 + 2] * psc, sv[4 * j4 + 3] * psc);

@@ -18,7 +18,8 @@
 //              its 64 head accumulators with tcgen05.ld and reduces
 //              s_k * sum_h (w_h s_q,h) * max(acc_h, 0) -> one fp32 score
 // The head reduction never leaves registers; scores are written once,
-// coalesced.  The FP8 query of each row is prepared once by
+// coalesced.  The visible tiles of a row are split evenly over the row's
+// blocks (about three blocks per SM in one wave).  The FP8 query of each row is prepared once by
 // index_prep_kernel (into the caller's workspace, already in the MMA's
 // swizzled layout) and bulk-copied into every block of that row.  All waits are bounded: a wait that gives up sets the device
 // status bit and an abort flag that stops every role; in-flight copies and
@@ -114,24 +115,8 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int row = blockIdx.y;   // b * T_q + query
   const int b = row / a.T_q;
-  pdl_wait();
-  const int t = a.q_pos[row];
-  int n_vis = (t + 1) / a.m;
-  const int ne = a.n_entries[b];
-  if (n_vis > ne) n_vis = ne;
-  if (n_vis > a.cap) n_vis = a.cap;
-  if (n_vis < 0 || t < 0) n_vis = 0;
 
-  const int tile0 = blockIdx.x * a.tiles_per_cta;
-  const int tiles_row = REINDEX ? a.tiles_per_row : (n_vis + kTileRows - 1) / kTileRows;
-  int tile1 = tile0 + a.tiles_per_cta;
-  if (tile1 > tiles_row) tile1 = tiles_row;
-  if (!REINDEX && blockIdx.x == 0 && tid == 0 && a.n_valid) a.n_valid[row] = n_vis;
-  const int ntiles = tile1 - tile0;
-  if (ntiles <= 0) return;
-  const int32_t *pool = REINDEX ? a.pool + (size_t)row * a.P : nullptr;
-
-  // ---- set-up: barriers (warp 0), TMEM (warp 1)
+  // ---- set-up that touches no global memory: barriers (warp 0), TMEM (warp 1)
   if (tid == 0) {
     for (int s = 0; s < kStages; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
     for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 4); }
@@ -141,12 +126,27 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
     S.n_issued = 0;
     S.n_mma = 0;
     fence_barrier_init();
+    prefetch_tmap(&ik_map);
   }
   if (warp == 1) {
     tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
   }
-  __syncthreads();
+  pdl_wait();
+
+  // ---- this block's tiles: the row's visible tiles split evenly over gridDim.x
+  const int t = a.q_pos[row];
+  int n_vis = (t + 1) / a.m;
+  const int ne = a.n_entries[b];
+  if (n_vis > ne) n_vis = ne;
+  if (n_vis > a.cap) n_vis = a.cap;
+  if (n_vis < 0 || t < 0) n_vis = 0;
+  const int tiles_row = REINDEX ? a.tiles_per_row : (n_vis + kTileRows - 1) / kTileRows;
+  const int tile0 = (int)(((int64_t)blockIdx.x * tiles_row) / gridDim.x);
+  const int tile1 = (int)(((int64_t)(blockIdx.x + 1) * tiles_row) / gridDim.x);
+  if (!REINDEX && blockIdx.x == 0 && tid == 0 && a.n_valid) a.n_valid[row] = n_vis;
+  const int ntiles = tile1 - tile0;
+  const int32_t *pool = REINDEX ? a.pool + (size_t)row * a.P : nullptr;
 
   auto issue = [&](int i) {   // tile tile0+i into stage i % kStages
     const int s = i % kStages;
@@ -163,9 +163,12 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
       tma_load_2d(&S.tile[s][0], &ik_map, 0, b * a.cap + tile * kTileRows, &S.full[s]);
     }
   };
-  if (tid == 0) {
-    prefetch_tmap(&ik_map);
-    // the prepared query (B operand) and head weights of this row
+  tc_fence_before();
+  __syncthreads();   // barriers initialised, TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  if (ntiles > 0 && tid == 0) {
+    // the prepared query (B operand) and head weights of this row, then the first tiles
     mbar_arrive_expect_tx(&S.qbar, kHeads * DI + kHeads * 4);
     bulk_load(S.q8, a.q8 + (size_t)row * kHeads * DI, kHeads * DI, &S.qbar);
     bulk_load(S.wq, a.wq + (size_t)row * kHeads, kHeads * 4, &S.qbar);
@@ -173,12 +176,10 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
     for (int i = 0; i < first; ++i) issue(i);
     S.n_issued = first;
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
 
-  if (warp == 0) {
+  if (ntiles <= 0) {
+    // nothing to score
+  } else   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
       for (int i = kStages; i < ntiles; ++i) {
@@ -270,7 +271,7 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
   if (S.abort) {
     if (tid == 0) {
       flag(a.status, CSA2_DEV_TIMEOUT);
-      mbar_wait_bounded(&S.qbar, 0, kWaitLimit);
+      if (ntiles > 0) mbar_wait_bounded(&S.qbar, 0, kWaitLimit);
       for (int j = S.n_mma; j < S.n_issued; ++j)
         mbar_wait_bounded(&S.full[j % kStages], (j / kStages) & 1, kWaitLimit);
     }
@@ -299,7 +300,7 @@ static cudaError_t launch_t(const CUtensorMap &map, const IndexArgs &a, cudaStre
   auto k = index_kernel<DI, REINDEX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid((a.tiles_per_row + a.tiles_per_cta - 1) / a.tiles_per_cta, a.B * a.T_q);
+  dim3 grid(a.ctas_per_row, a.B * a.T_q);
   return launch_pdl(k, grid, dim3(kThreads), smem, s, dim3(1, 1, 1), map, a);
 }
 

@@ -44,7 +44,8 @@ struct IndexArgs {
   int32_t *n_valid;       // full mode, optional
   const int32_t *pool;    // reindex mode: [B*T_q][P]
   int P;
-  int tiles_per_row, tiles_per_cta;
+  int tiles_per_row;      // reindex: P/16; full: cap/128 (the visible count is found in the kernel)
+  int ctas_per_row;       // blocks sharing one row's tiles
   uint8_t *q8;            // workspace: [B*T_q][64*dI] prepared FP8 query (MMA layout)
   float *wq;              // workspace: [B*T_q][64] w_h * s_q,h
   unsigned int *status;

@@ -71,3 +71,29 @@ def test_workspace_sizes_are_pure_host_functions():
     assert C.csa2_topk_workspace_size(8, 100000, 512, 2048) > 0
     assert C.csa2_topk_workspace_size(8, 65536, 512, 2048) == 0   # single-launch cluster path
     assert C.csa2_topk_workspace_size(0, 65536, 512, 2048) == 0
+
+
+def test_binding_marshals_every_entry_point_without_a_gpu():
+    """Each Python wrapper reaches the library (which then reports that it
+    cannot run here) instead of failing in its own argument handling."""
+    import torch
+    B, cap, D, dI = 1, 128, 128, 64
+    m = C.MainCache(B, cap, D, dI, 1, device="cpu")
+    sw = C.SwaCache(B, 128, D, device="cpu")
+    bf = lambda *s: torch.zeros(*s, dtype=torch.bfloat16)
+    i32 = lambda *s: torch.zeros(*s, dtype=torch.int32)
+    f32 = lambda *s: torch.zeros(*s, dtype=torch.float32)
+    calls = [
+        lambda: C.csa2_append_quant(m, bf(B, 1, D), None, bf(D, dI), sw, bf(B, 1, D), i32(B), 1, stream=0),
+        lambda: C.csa2_index_full(m, bf(B, 1, 4, dI), f32(B, 1, 4), i32(B, 1), f32(B, cap), i32(B), stream=0),
+        lambda: C.csa2_index_reindex(m, bf(B, 1, 4, dI), f32(B, 1, 4), i32(B, 1), i32(B, 16), f32(B, 128),
+                                     stream=0),
+        lambda: C.csa2_topk(f32(B, cap), cap, 8, i32(B, 8), n_valid=i32(B), P_out=16, out_pool=i32(B, 16),
+                            stream=0),
+        lambda: C.csa2_topk_noalloc(f32(B, cap), cap, 8, i32(B, 8), stream=0),
+        lambda: C.csa2_sparse_attn_decode(m, sw, bf(B, 1, 8, D), i32(B, 1), i32(B, 8), 0.1, bf(B, 1, 8, D),
+                                          stream=0),
+    ]
+    for call in calls:
+        with pytest.raises(C.Csa2Error):
+            call()

@@ -85,18 +85,26 @@ def test_append_m1_bit_exact(D, dI):
     assert C.csa2_device_status() == 0
 
 
-def test_append_decode_single_token_and_ring_wrap():
-    B, D, dI, cap = 2, 512, 128, 1024
-    gm, gs, om, osw, W = build_pair(B=B, cap=cap, D=D, dI=dI, m=1, T=700, pos0=[0, 5], seed=3)
+@pytest.mark.parametrize("D,dI,with_window", [(512, 128, True), (256, 64, True), (128, 64, False), (512, 64, True)])
+def test_append_decode_single_token_and_ring_wrap(D, dI, with_window):
+    # one token per sequence per call: the decode path (an 8-block cluster per entry)
+    B, cap = 3, 1024
+    gm, gs, om, osw, W = build_pair(B=B, cap=cap, D=D, dI=dI, m=1, T=700, pos0=[0, 5, 9], seed=3 + D + dI)
     g = gen(4)
     for step in range(3):
         kv = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+        kv[1, 0, : D // 2] = 0   # all-zero groups: scale byte 0, codes 0
         kvs = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
-        pos = np.array([700 + step, 705 + step], np.int32)
-        C.csa2_append_quant(gm, kv.cuda(), None, W.cuda(), gs, kvs.cuda(), torch.from_numpy(pos).cuda(), 1)
-        oracle.append(om, bits(kv), None, bits(W), osw, bits(kvs), pos, 1)
+        pos = np.array([700 + step, 705 + step, 709 + step], np.int32)
+        C.csa2_append_quant(gm, kv.cuda(), None, W.cuda(), gs if with_window else None,
+                            kvs.cuda() if with_window else None, torch.from_numpy(pos).cuda(), 1)
+        oracle.append(om, bits(kv), None, bits(W), osw if with_window else None, bits(kvs) if with_window else None,
+                      pos, 1)
     torch.cuda.synchronize()
-    assert_cache_equal(gm, om, gs, osw)
+    if with_window:
+        assert_cache_equal(gm, om, gs, osw)
+    else:
+        assert_cache_equal(gm, om)
 
 
 def test_append_m2_pending_across_calls():
