@@ -44,7 +44,9 @@ _PM, _PS = ctypes.POINTER(MainCacheDesc), ctypes.POINTER(SwaCacheDesc)
 
 SIGNATURES = {
     "csa2_append_quant": (_I, [_PM, _P, _P, _P, _PS, _P, _P, _I, _P]),
+    "csa2_append_quant_ex": (_I, [_PM, _P, _P, _P, _PS, _P, _P, _I, _P, _P, _I, _I, _P, _SZ, _P]),
     "csa2_index_full": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _P, _SZ, _P]),
+    "csa2_index_full_prepared": (_I, [_PM, _P, _I, _P, _I64, _P, _P, _SZ, _P]),
     "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "csa2_index_workspace_size": (_SZ, [_I, _I]),
     "csa2_topk": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P, _SZ, _P]),
@@ -146,6 +148,26 @@ def csa2_append_quant(main: MainCache | None, kv, gate, w_ik, swa: SwaCache | No
     _check(lib().csa2_append_quant(md, _ptr(kv, torch.bfloat16), _ptr(gate, torch.bfloat16),
                                    _ptr(w_ik, torch.bfloat16), sd, _ptr(kv_swa, torch.bfloat16),
                                    _ptr(pos0, torch.int32), int(T), _stream(stream)))
+
+
+def csa2_append_quant_ex(main: MainCache, kv, gate, w_ik, swa: SwaCache | None, kv_swa, pos0, T: int,
+                         q_idx, w, ws, stream=None):
+    """csa2_append_quant plus the preparation of the following scan's query
+    (q_idx [B][T_q][H_I][d_I], w [B][T_q][H_I]) into ws."""
+    sd = ctypes.byref(swa.desc()) if swa is not None else None
+    T_q, H_I = q_idx.shape[-3], q_idx.shape[-2]
+    _check(lib().csa2_append_quant_ex(ctypes.byref(main.desc()), _ptr(kv, torch.bfloat16), _ptr(gate, torch.bfloat16),
+                                      _ptr(w_ik, torch.bfloat16), sd, _ptr(kv_swa, torch.bfloat16),
+                                      _ptr(pos0, torch.int32), int(T), _ptr(q_idx, torch.bfloat16),
+                                      _ptr(w, torch.float32), T_q, H_I, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def csa2_index_full_prepared(main: MainCache, q_pos, scores, n_valid=None, ws=None, stream=None):
+    """csa2_index_full with the query prepared in ws by csa2_append_quant_ex."""
+    T_q = q_pos.shape[-1]
+    _check(lib().csa2_index_full_prepared(ctypes.byref(main.desc()), _ptr(q_pos, torch.int32), T_q,
+                                          _ptr(scores, torch.float32), scores.shape[-1], _ptr(n_valid, torch.int32),
+                                          _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def csa2_index_workspace_size(rows: int, d_I: int) -> int:

@@ -159,10 +159,9 @@ csa2_status csa2_device_status(csa2_stream_t stream, uint32_t *flags, int clear)
   return v ? CSA2_ERR_DEVICE_CHECK : CSA2_OK;
 }
 
-csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, const uint16_t *gate,
-                              const uint16_t *w_ik, const csa2_swa_cache *swa, const uint16_t *kv_swa,
-                              const int32_t *pos0, int T, csa2_stream_t stream) {
-  t_err.clear();
+static csa2_status append_impl(const csa2_main_cache *main, const uint16_t *kv, const uint16_t *gate,
+                               const uint16_t *w_ik, const csa2_swa_cache *swa, const uint16_t *kv_swa,
+                               const int32_t *pos0, int T, const QueryPrep *prep, csa2_stream_t stream) {
   if (!main && !swa) return fail(CSA2_ERR_INVALID_ARG, "append needs a main or a window cache");
   if (T < 0) return fail(CSA2_ERR_INVALID_ARG, "T=%d", T);
   if (!pos0 || !aligned16(pos0)) return fail(CSA2_ERR_INVALID_ARG, "pos0 must be a 16-byte aligned device pointer");
@@ -170,9 +169,9 @@ csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, c
   int B = 0, D = 0;
   if (main) {
     if ((st = check_main(main, true)) != CSA2_OK) return st;
-    if (!kv || !w_ik || !aligned16(kv) || !aligned16(w_ik))
+    if (T > 0 && (!kv || !w_ik || !aligned16(kv) || !aligned16(w_ik)))
       return fail(CSA2_ERR_INVALID_ARG, "kv and w_ik must be 16-byte aligned device pointers");
-    if (main->m == 2 && (!gate || !aligned16(gate))) return fail(CSA2_ERR_INVALID_ARG, "m=2 needs gate");
+    if (T > 0 && main->m == 2 && (!gate || !aligned16(gate))) return fail(CSA2_ERR_INVALID_ARG, "m=2 needs gate");
     if (main->m == 2 && (!aligned16(main->pending_kv) || !aligned16(main->pending_gate)))
       return fail(CSA2_ERR_INVALID_ARG, "pending buffers must be 16-byte aligned");
     B = main->B;
@@ -180,21 +179,23 @@ csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, c
   }
   if (swa) {
     if ((st = check_swa(swa)) != CSA2_OK) return st;
-    if (!kv_swa || !aligned16(kv_swa)) return fail(CSA2_ERR_INVALID_ARG, "kv_swa must be a 16-byte aligned device pointer");
+    if (T > 0 && (!kv_swa || !aligned16(kv_swa)))
+      return fail(CSA2_ERR_INVALID_ARG, "kv_swa must be a 16-byte aligned device pointer");
     if (main && (swa->B != B || swa->D != D)) return fail(CSA2_ERR_INVALID_ARG, "window and main cache disagree on B or D");
     B = swa->B;
     D = swa->D;
   }
-  if (T == 0) return CSA2_OK;
+  if (T == 0 && !prep) return CSA2_OK;
   DeviceState *d;
   if ((st = device_state(&d)) != CSA2_OK) return st;
   AppendArgs a{};
+  if (prep) a.prep = *prep;
   if (main) {
     a.codes = main->codes; a.scales = main->scales; a.ik = main->ik; a.ik_scale = main->ik_scale;
     a.n_entries = main->n_entries; a.pending_kv = main->pending_kv; a.pending_gate = main->pending_gate;
     a.cap = main->cap; a.dI = main->d_I; a.m = main->m;
     a.kv = kv; a.gate = gate; a.w_ik = w_ik;
-    const int max_new = main->m == 1 ? T : T / 2 + 1;   // upper bound of complete entries
+    const int max_new = T == 0 ? 0 : (main->m == 1 ? T : T / 2 + 1);   // upper bound of complete entries
     a.entries_per_block = max_new >= 64 ? 8 : 1;
     a.main_blocks_per_seq = (max_new + a.entries_per_block - 1) / a.entries_per_block;
   }
@@ -211,6 +212,35 @@ csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, c
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "append launch");
 }
 
+csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, const uint16_t *gate,
+                              const uint16_t *w_ik, const csa2_swa_cache *swa, const uint16_t *kv_swa,
+                              const int32_t *pos0, int T, csa2_stream_t stream) {
+  t_err.clear();
+  return append_impl(main, kv, gate, w_ik, swa, kv_swa, pos0, T, nullptr, stream);
+}
+
+csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uint16_t *kv, const uint16_t *gate,
+                                 const uint16_t *w_ik, const csa2_swa_cache *swa, const uint16_t *kv_swa,
+                                 const int32_t *pos0, int T, const uint16_t *q_idx, const float *w, int T_q,
+                                 int H_I, void *ws, size_t ws_bytes, csa2_stream_t stream) {
+  t_err.clear();
+  if (!main) return fail(CSA2_ERR_INVALID_ARG, "preparing a scan's query needs the main cache (its d_I)");
+  if (!q_idx || !w || !aligned16(q_idx) || !aligned16(w))
+    return fail(CSA2_ERR_INVALID_ARG, "q_idx and w must be 16-byte aligned device pointers");
+  if (T_q <= 0 || (int64_t)main->B * T_q > 65535) return fail(CSA2_ERR_INVALID_ARG, "T_q=%d", T_q);
+  if (H_I < 1 || H_I > 64) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "H_I=%d not in [1,64]", H_I);
+  if (main->d_I != 64 && main->d_I != 128) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "d_I=%d", main->d_I);
+  const int rows = main->B * T_q;
+  const size_t need = index_workspace_bytes(rows, main->d_I);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(CSA2_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  QueryPrep p{};
+  p.q_idx = q_idx; p.w = w; p.rows = rows; p.H_I = H_I; p.dI = main->d_I;
+  p.q8 = static_cast<uint8_t *>(ws);
+  p.wq = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (((size_t)rows * 64 * main->d_I + 15) & ~size_t(15)));
+  return append_impl(main, kv, gate, w_ik, swa, kv_swa, pos0, T, &p, stream);
+}
+
 // Blocks per row of a scan: about three resident blocks per SM in one wave,
 // the row's tiles split evenly over them.
 static int index_ctas_per_row(int tiles_per_row, int rows, int sms) {
@@ -222,14 +252,15 @@ static int index_ctas_per_row(int tiles_per_row, int rows, int sms) {
 
 static csa2_status index_common(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                                 const int32_t *q_pos, int T_q, int H_I, float *scores, void *ws, size_t ws_bytes,
-                                IndexArgs *a, CUtensorMap *map, int box_rows) {
+                                IndexArgs *a, CUtensorMap *map, int box_rows, bool prepared = false) {
   csa2_status st;
   if ((st = check_main(main, false)) != CSA2_OK) return st;
-  if (!q_idx || !w || !q_pos || !scores) return fail(CSA2_ERR_INVALID_ARG, "NULL argument");
-  if (!aligned16(q_idx) || !aligned16(w) || !aligned16(q_pos) || !aligned16(scores))
+  if (!prepared && (!q_idx || !w)) return fail(CSA2_ERR_INVALID_ARG, "NULL argument");
+  if (!q_pos || !scores) return fail(CSA2_ERR_INVALID_ARG, "NULL argument");
+  if ((!prepared && (!aligned16(q_idx) || !aligned16(w))) || !aligned16(q_pos) || !aligned16(scores))
     return fail(CSA2_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (T_q <= 0) return fail(CSA2_ERR_INVALID_ARG, "T_q=%d", T_q);
-  if (H_I < 1 || H_I > 64) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "H_I=%d not in [1,64]", H_I);
+  if (!prepared && (H_I < 1 || H_I > 64)) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "H_I=%d not in [1,64]", H_I);
   if ((int64_t)main->B * T_q > 65535) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "B*T_q must be <= 65535");
   const size_t need = index_workspace_bytes(main->B * T_q, main->d_I);
   if (!ws || ws_bytes < need || !aligned16(ws))
@@ -242,6 +273,7 @@ static csa2_status index_common(const csa2_main_cache *main, const uint16_t *q_i
   a->ik_scale = main->ik_scale; a->n_entries = main->n_entries;
   a->B = main->B; a->cap = main->cap; a->m = main->m; a->dI = main->d_I;
   a->q_idx = q_idx; a->w = w; a->q_pos = q_pos; a->T_q = T_q; a->H_I = H_I; a->scores = scores;
+  a->prepared = prepared;
   return CSA2_OK;
 }
 
@@ -250,13 +282,12 @@ size_t csa2_index_workspace_size(int rows, int d_I) {
   return index_workspace_bytes(rows, d_I);
 }
 
-csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
-                            const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
-                            int32_t *n_valid, void *ws, size_t ws_bytes, csa2_stream_t stream) {
-  t_err.clear();
+static csa2_status index_full_impl(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
+                                   const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
+                                   int32_t *n_valid, void *ws, size_t ws_bytes, bool prepared, csa2_stream_t stream) {
   IndexArgs a;
   CUtensorMap map;
-  csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, scores, ws, ws_bytes, &a, &map, 128);
+  csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, scores, ws, ws_bytes, &a, &map, 128, prepared);
   if (st != CSA2_OK) return st;
   if (ld < main->cap) return fail(CSA2_ERR_INVALID_ARG, "ld=%lld < cap=%d", (long long)ld, main->cap);
   if (n_valid && !aligned16(n_valid)) return fail(CSA2_ERR_INVALID_ARG, "n_valid must be 16-byte aligned");
@@ -267,6 +298,21 @@ csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, 
   a.ctas_per_row = index_ctas_per_row(a.tiles_per_row, main->B * T_q, d->sms);
   cudaError_t e = launch_index(map, a, false, d->sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
+}
+
+csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
+                            const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
+                            int32_t *n_valid, void *ws, size_t ws_bytes, csa2_stream_t stream) {
+  t_err.clear();
+  return index_full_impl(main, q_idx, w, q_pos, T_q, H_I, scores, ld, n_valid, ws, ws_bytes, false, stream);
+}
+
+csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const int32_t *q_pos, int T_q, float *scores,
+                                     int64_t ld, int32_t *n_valid, const void *ws, size_t ws_bytes,
+                                     csa2_stream_t stream) {
+  t_err.clear();
+  return index_full_impl(main, nullptr, nullptr, q_pos, T_q, 64, scores, ld, n_valid, const_cast<void *>(ws),
+                         ws_bytes, true, stream);
 }
 
 csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,

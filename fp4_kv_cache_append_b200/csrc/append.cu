@@ -223,11 +223,25 @@ __device__ void append_window_row(const AppendArgs &a, int b, int r) {
   reinterpret_cast<uint16_t *>(dst)[t] = (uint16_t)(lo | (hi << 8));
 }
 
+// Blocks beyond the cache work prepare the following scan's indexer query:
+// 8 blocks per query row, warp w of block j handles head 8j + w.
+__device__ __forceinline__ void prep_block(const AppendArgs &a, int i) {
+  const int row = i / 8, h = (i % 8) * 8 + (int)(threadIdx.x >> 5);
+  if (row >= a.prep.rows || threadIdx.x >= 256) return;
+  if (a.prep.dI == 128) prep_query_head<128>(a.prep, row, h, threadIdx.x & 31);
+  else prep_query_head<64>(a.prep, row, h, threadIdx.x & 31);
+}
+
 __global__ void append_kernel(const AppendArgs a) {
   extern __shared__ float sm[];
   pdl_launch_dependents();
   pdl_wait();
   const int nm = a.B * a.main_blocks_per_seq;
+  const int nw = a.B * a.swa_blocks_per_seq;
+  if ((int)blockIdx.x >= nm + nw) {
+    prep_block(a, (int)blockIdx.x - nm - nw);
+    return;
+  }
   if ((int)blockIdx.x < nm) {
     append_entries(a, blockIdx.x / a.main_blocks_per_seq,
                    (blockIdx.x % a.main_blocks_per_seq) * a.entries_per_block, sm);
@@ -257,6 +271,10 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
   const int D = a.D, dI = a.dI, G = D / 32, OPB = dI / kDecCl;
   pdl_launch_dependents();
   pdl_wait();
+  if (b >= a.B) {   // a cluster of query-preparation blocks (no cluster barrier)
+    prep_block(a, (b - a.B) * kDecCl + c);
+    return;
+  }
   const int p0 = a.pos0[b];
   if (p0 < 0) {   // the same in every block of the cluster: none of them waits
     if (t == 0 && c == 0) flag(a.status, CSA2_DEV_BAD_POSITION);
@@ -362,8 +380,8 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
   if (a.codes && a.m == 1 && a.T == 1 && a.D <= 512 && a.dI % (8 * kDecCl) == 0 && a.dI / kDecCl <= 16 &&
       (!a.swa_rows || a.W_cap >= 1))
-    return launch_pdl(append_decode_kernel, dim3(kDecCl, a.B), dim3(256), 0, s, dim3(1, 1, 1), a);
-  const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq);
+    return launch_pdl(append_decode_kernel, dim3(kDecCl, a.B + a.prep.rows), dim3(256), 0, s, dim3(1, 1, 1), a);
+  const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq) + 8 * a.prep.rows;
   if (blocks == 0) return cudaSuccess;
   const int threads = 512;   // quantisation uses the first D/2, the projection all of them
   // [E][D] + [E][G][dI] floats, 32 floats, then W_ik [D][dI] bf16

@@ -19,9 +19,11 @@
 //              s_k * sum_h (w_h s_q,h) * max(acc_h, 0) -> one fp32 score
 // The head reduction never leaves registers; scores are written once,
 // coalesced.  The visible tiles of a row are split evenly over the row's
-// blocks (about three blocks per SM in one wave).  The FP8 query of each row is prepared once by
-// index_prep_kernel (into the caller's workspace, already in the MMA's
-// swizzled layout) and bulk-copied into every block of that row.  All waits are bounded: a wait that gives up sets the device
+// blocks (about three blocks per SM in one wave).  The FP8 query of each row
+// is prepared once (index_prep_kernel, or by the append launch that precedes
+// the scan: csa2_append_quant_ex) into the caller's workspace, already in the
+// MMA's swizzled layout, and bulk-copied into every block of that row.  All
+// waits are bounded: a wait that gives up sets the device
 // status bit and an abort flag that stops every role; in-flight copies and
 // MMAs are then drained (bounded) and TMEM is freed before the block exits.
 #include "common.cuh"
@@ -32,7 +34,7 @@ namespace csa2 {
 namespace {
 
 constexpr int kThreads = 192;
-constexpr int kStages = 4;
+constexpr int kStages = 2;   // measured: deeper rings lower the scan's DRAM throughput
 constexpr int kTileRows = 128;
 constexpr int kHeads = 64;          // N of the MMA (indexer heads, zero padded)
 constexpr uint32_t kTmemCols = 128; // two 64-column fp32 accumulators
@@ -65,40 +67,13 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
 
 }  // namespace
 
-// Indexer query of one row: per head, E4M3 codes with scale amax/448 (the
-// rule of the keys), laid out as the MMA's B operand (64 rows x DI bytes,
-// K-major, swizzled), and the head weights w_h * s_q,h.
-// One warp per head: grid (rows, 8) x 256 threads.
+// Indexer query of each row (prep_query_head): grid (rows, 8) x 256 threads,
+// one warp per head.
 template <int DI>
 __global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
-  constexpr int MASK = DI == 128 ? 7 : 3;
-  const int row = blockIdx.x, lane = threadIdx.x & 31;
   pdl_launch_dependents();
   pdl_wait();
-  const uint16_t *qrow = a.q_idx + (size_t)row * a.H_I * DI;
-  const float *wrow = a.w + (size_t)row * a.H_I;
-  uint8_t *q8 = a.q8 + (size_t)row * kHeads * DI;
-  {
-    const int h = blockIdx.y * 8 + (threadIdx.x >> 5);
-    float v[DI / 32];
-    float amax = 0.f;
-    if (h < a.H_I) {
-#pragma unroll
-      for (int i = 0; i < DI / 32; ++i) {
-        v[i] = bf16_to_f32(qrow[h * DI + lane + 32 * i]);
-        amax = fmaxf(amax, fabsf(v[i]));
-      }
-      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    }
-    const float sq = __fdiv_rn(amax, 448.0f);
-#pragma unroll
-    for (int i = 0; i < DI / 32; ++i) {
-      const int c = lane + 32 * i;
-      const uint32_t code = (h < a.H_I && sq != 0.f) ? f32_to_e4m3(__fdiv_rn(v[i], sq)) : 0u;
-      q8[swz<MASK>(h * DI + c)] = (uint8_t)code;
-    }
-    if (lane == 0) a.wq[(size_t)row * kHeads + h] = h < a.H_I ? wrow[h] * sq : 0.f;
-  }
+  prep_query_head<DI>(a, blockIdx.x, blockIdx.y * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
 }
 
 template <int DI, bool REINDEX>
@@ -246,17 +221,24 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      uint32_t acc[kHeads];
+      // heads in two halves of 32 columns (fewer live registers); chain j
+      // takes heads j, j+4, ... in ascending order
       const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * kHeads;
-      tmem_ld_x32(taddr, acc);
-      tmem_ld_x32(taddr + 32, acc + 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.tempty[ab]);
       float s4[4] = {0.f, 0.f, 0.f, 0.f};   // independent chains
 #pragma unroll
-      for (int h = 0; h < kHeads; ++h) s4[h & 3] = fmaf(S.wq[h], fmaxf(__uint_as_float(acc[h]), 0.f), s4[h & 3]);
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t acc[32];
+        tmem_ld_x32(taddr + 32 * hh, acc);
+        tmem_wait_ld();
+        if (hh == 1) {   // the accumulator is free once both halves are in registers
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&S.tempty[ab]);
+        }
+#pragma unroll
+        for (int h = 0; h < 32; ++h)
+          s4[h & 3] = fmaf(S.wq[32 * hh + h], fmaxf(__uint_as_float(acc[h]), 0.f), s4[h & 3]);
+      }
       const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       float *out = a.scores + (size_t)row * a.ld;
       if (REINDEX) out[tile * kTileRows + r] = valid ? sum * sk : -INFINITY;
@@ -294,8 +276,10 @@ size_t index_workspace_bytes(int rows, int dI) {
 
 template <int DI, bool REINDEX>
 static cudaError_t launch_t(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
-  cudaError_t pe = launch_pdl(index_prep_kernel<DI>, dim3(a.B * a.T_q, kHeads / 8), dim3(256), 0, s, dim3(1, 1, 1), a);
-  if (pe != cudaSuccess) return pe;
+  if (!a.prepared) {
+    cudaError_t pe = launch_pdl(index_prep_kernel<DI>, dim3(a.B * a.T_q, kHeads / 8), dim3(256), 0, s, dim3(1, 1, 1), a);
+    if (pe != cudaSuccess) return pe;
+  }
   const size_t smem = sizeof(IndexSmem<DI>) + 1024;
   auto k = index_kernel<DI, REINDEX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

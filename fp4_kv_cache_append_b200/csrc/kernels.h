@@ -10,6 +10,18 @@
 
 namespace csa2 {
 
+// Preparation of a scan's indexer query (one warp per head): per head E4M3
+// codes with scale amax/448 in the scan's B-operand layout (64 rows x dI
+// bytes, K-major, swizzled) and the head weights w_h * s_q,h.
+constexpr int kIndexHeads = 64;   // N of the scan's MMA (indexer heads, zero padded)
+struct QueryPrep {
+  const uint16_t *q_idx;  // [rows][H_I][dI] bf16
+  const float *w;         // [rows][H_I]
+  int rows, H_I, dI;      // rows == 0: nothing to prepare
+  uint8_t *q8;            // [rows][64*dI]
+  float *wq;              // [rows][64]
+};
+
 struct AppendArgs {
   // main cache (codes == nullptr: no main part)
   uint8_t *codes, *scales, *ik;
@@ -28,6 +40,7 @@ struct AppendArgs {
   int main_blocks_per_seq, swa_blocks_per_seq;
   int entries_per_block;   // 1 .. 8
   unsigned int *status;
+  QueryPrep prep;          // optional: the following scan's query, 8 blocks per row
 };
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s);
 
@@ -48,6 +61,7 @@ struct IndexArgs {
   int ctas_per_row;       // blocks sharing one row's tiles
   uint8_t *q8;            // workspace: [B*T_q][64*dI] prepared FP8 query (MMA layout)
   float *wq;              // workspace: [B*T_q][64] w_h * s_q,h
+  bool prepared;          // q8/wq already hold the query (no preparation kernel)
   unsigned int *status;
 };
 size_t index_workspace_bytes(int rows, int dI);

@@ -169,10 +169,12 @@ class Step:
 
         for kind, l in self.plan:
             if kind == "full":
-                timed("append", lambda: C.csa2_append_quant(main, self.kv_new, self.gate_new, self.w_ik, swa[l],
-                                                            self.kv_swa_new[l], self.pos0, wl.T))
-                timed("index_full", lambda: C.csa2_index_full(main, self.q_idx[l], self.w[l], self.q_pos,
-                                                              self.scores, self.n_valid, ws=self.ws_index))
+                # the append launch also prepares the scan's indexer query
+                timed("append", lambda: C.csa2_append_quant_ex(main, self.kv_new, self.gate_new, self.w_ik, swa[l],
+                                                               self.kv_swa_new[l], self.pos0, wl.T, self.q_idx[l],
+                                                               self.w[l], self.ws_index))
+                timed("index_full", lambda: C.csa2_index_full_prepared(main, self.q_pos, self.scores, self.n_valid,
+                                                                       ws=self.ws_index))
                 timed("topk", lambda: C.csa2_topk(self.scores, self.cap, wl.K, self.idx, n_valid=self.n_valid,
                                                   P_out=wl.P, out_pool=self.pool if wl.P else None,
                                                   ws=self.ws_topk))
@@ -193,16 +195,16 @@ class Step:
     # ------------------------------------------------------------------ accounting
 
     def launches_per_step(self) -> int:
-        """libcsa2 kernel launches one step enqueues (append 1, index 2 =
-        query prep + scan, Top-K 1 for rows of up to 65,536 columns else 4,
-        attention 1)."""
+        """libcsa2 kernel launches one step enqueues (append 1, which also
+        prepares a Full scan's query; Full scan 1; Reindex 2 = query prep +
+        scan; Top-K 1 for rows of up to 65,536 columns else 4; attention 1)."""
         wl = self.wl
         topk = lambda n_cols: 1 if n_cols <= 65536 else 4
         n = 0
         for kind, _ in self.plan:
             n += 1 + 1   # append, attention
             if kind == "full":
-                n += 2 + topk(self.cap)
+                n += 1 + topk(self.cap)
             elif kind == "reindex":
                 n += 2 + topk(wl.P * 8)
         return n

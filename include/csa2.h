@@ -124,6 +124,23 @@ CSA2_API csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16
                               const int32_t *pos0, int T, csa2_stream_t stream);
 
 /*
+ * 1b. Append, and prepare the indexer query of the scan that follows, in one
+ *     launch: csa2_append_quant plus, for each of the B*T_q query rows, the
+ *     query preparation csa2_index_full performs (per head E4M3 codes with
+ *     scale amax/448 and the weights w_h * s_q,h) written into ws, for
+ *     csa2_index_full_prepared.  Saves the scan a launch in a decode step.
+ *  main  required (its d_I sets the layout); T may be 0 (preparation only)
+ *  q_idx [B][T_q][H_I][d_I] bf16, w [B][T_q][H_I] f32 (as for csa2_index_full)
+ *  ws, ws_bytes: csa2_index_workspace_size(B*T_q, d_I) bytes, kept by the
+ *         caller until the prepared scan has run
+ */
+CSA2_API csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uint16_t *kv,
+                              const uint16_t *gate, const uint16_t *w_ik,
+                              const csa2_swa_cache *swa, const uint16_t *kv_swa,
+                              const int32_t *pos0, int T, const uint16_t *q_idx, const float *w,
+                              int T_q, int H_I, void *ws, size_t ws_bytes, csa2_stream_t stream);
+
+/*
  * 2. Full indexer scoring  [jaehun "2) CSA2": a Full layer scores all entries
  *    with its own indexer; score_j = sum_h w_h ReLU(q_h . k_j) as an FP8
  *    contraction].
@@ -144,6 +161,15 @@ CSA2_API csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t
                             float *scores, int64_t ld, int32_t *n_valid,
                             void *ws, size_t ws_bytes, csa2_stream_t stream);
 CSA2_API size_t csa2_index_workspace_size(int rows, int d_I);
+
+/*
+ * 2b. Full indexer scoring with the query already prepared in ws by
+ *     csa2_append_quant_ex (same rows, same T_q); otherwise as
+ *     csa2_index_full.
+ */
+CSA2_API csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const int32_t *q_pos, int T_q,
+                              float *scores, int64_t ld, int32_t *n_valid,
+                              const void *ws, size_t ws_bytes, csa2_stream_t stream);
 
 /*
  * 3. Reindex scoring  [jaehun "2) CSA2": later Reindex layers rescore only the

@@ -86,6 +86,11 @@ def test_binding_marshals_every_entry_point_without_a_gpu():
     calls = [
         lambda: C.csa2_append_quant(m, bf(B, 1, D), None, bf(D, dI), sw, bf(B, 1, D), i32(B), 1, stream=0),
         lambda: C.csa2_index_full(m, bf(B, 1, 4, dI), f32(B, 1, 4), i32(B, 1), f32(B, cap), i32(B), stream=0),
+        lambda: C.csa2_append_quant_ex(m, bf(B, 1, D), None, bf(D, dI), sw, bf(B, 1, D), i32(B), 1,
+                                       bf(B, 1, 4, dI), f32(B, 1, 4), torch.zeros(1 << 16, dtype=torch.uint8),
+                                       stream=0),
+        lambda: C.csa2_index_full_prepared(m, i32(B, 1), f32(B, cap), i32(B),
+                                           ws=torch.zeros(1 << 16, dtype=torch.uint8), stream=0),
         lambda: C.csa2_index_reindex(m, bf(B, 1, 4, dI), f32(B, 1, 4), i32(B, 1), i32(B, 16), f32(B, 128),
                                      stream=0),
         lambda: C.csa2_topk(f32(B, cap), cap, 8, i32(B, 8), n_valid=i32(B), P_out=16, out_pool=i32(B, 16),

@@ -180,6 +180,42 @@ def test_index_full_vs_oracle(D, dI, H_I, n, T_q, m):
     assert C.csa2_device_status() == 0
 
 
+@pytest.mark.parametrize("D,dI,H_I,T_q", [(512, 128, 64, 1), (256, 64, 17, 3)])
+def test_index_full_prepared_by_the_append(D, dI, H_I, T_q):
+    """Append + query preparation in one launch, then the prepared scan: the
+    cache bytes of the appended token, and scores bit-identical to the plain
+    scan (which itself is checked against the oracle above)."""
+    B, n = 2, 3000
+    cap = (n + 1 + 127) // 128 * 128
+    gm, gs, om, osw, W = build_pair(B=B, cap=cap, D=D, dI=dI, m=1, T=n, pos0=[0, 0], seed=31 + D)
+    q, w = _rows_queries(B, T_q, H_I, dI, seed=32)
+    g = gen(33)
+    kv = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+    kvs = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+    pos = np.array([n, n], np.int32)
+    qpos = np.array([[n - T_q + 1 + j for j in range(T_q)] for _ in range(B)], np.int32)
+    qpos[:, -1] = n
+    ws = C.workspace(C.csa2_index_workspace_size(B * T_q, dI))
+    C.csa2_append_quant_ex(gm, kv.cuda(), None, W.cuda(), gs, kvs.cuda(), torch.from_numpy(pos).cuda(), 1,
+                           q.cuda(), w.cuda(), ws)
+    oracle.append(om, bits(kv), None, bits(W), osw, bits(kvs), pos, 1)
+    got = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nv = torch.empty(B * T_q, dtype=torch.int32, device="cuda")
+    C.csa2_index_full_prepared(gm, torch.from_numpy(qpos).cuda(), got, nv, ws=ws)
+    plain = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    C.csa2_index_full(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), plain, nv)
+    torch.cuda.synchronize()
+    assert_cache_equal(gm, om, gs, osw)
+    a, b_ = got.cpu().numpy(), plain.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b_.view(np.uint32))
+    # preparation only (T = 0): the same workspace contents
+    ws2 = C.workspace(C.csa2_index_workspace_size(B * T_q, dI))
+    C.csa2_append_quant_ex(gm, None, None, None, None, None, torch.from_numpy(pos).cuda(), 0, q.cuda(), w.cuda(), ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(ws.cpu(), ws2.cpu())
+    assert C.csa2_device_status() == 0
+
+
 # ------------------------------------------------------------------ A4 Top-K
 
 
