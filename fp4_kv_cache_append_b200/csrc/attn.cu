@@ -23,10 +23,10 @@
 // than 2^8 (then O^T and the running sum are rescaled in place), so P stays
 // within fp16 range and rescaling is rare.  Window rows keep their raw E4M3
 // values; the layer's window scale multiplies their logits and their P.
-// The splits of one row form a thread-block cluster: each writes its
-// unnormalised O^T and (max, sum) per head to the workspace, and after one
-// cluster barrier each split merges a slice of the channels from all splits
-// and writes the bf16 output.  Straight-line code is kept short (rolled
+// The splits of one row form a thread-block cluster: each writes O / l per
+// head (fp16, [head][channel]) and its (max, sum) per head to the workspace, and
+// after one cluster barrier each split merges a slice of the channels from all
+// splits (weights 2^(m_s - M) l_s / L) and writes the bf16 output.  Straight-line code is kept short (rolled
 // loops): each block runs it about once, so fetching it costs as much as
 // executing it.
 #include "common.cuh"
@@ -92,6 +92,11 @@ __device__ __forceinline__ int ordered(float f) {
   return b >= 0 ? b : (b ^ 0x7FFFFFFF);
 }
 __device__ __forceinline__ float unordered(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7FFFFFFF)); }
+
+// f32 (max, sum) per (row, split, head), after the fp16 partials.
+__device__ __forceinline__ float *partial_stats(const AttnArgs &a, size_t nrows) {
+  return reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.ws) + nrows * a.nsplit * (size_t)a.D * kHeads * 2);
+}
 
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -414,6 +419,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   } else {
     tc_fence_after();
     const size_t nrows = (size_t)a.B * a.T_q;
+    // split partials: O / l per head in fp16, head-major [64 heads][D]
+    float linv[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const float l = S.l_run[32 * half + j];
+      linv[j] = l > 0.f ? 1.f / l : 0.f;
+    }
 #pragma unroll 1
     for (int mt = 0; mt < MT; ++mt) {
       const int ch = mt * 128 + 32 * quarter + lane;
@@ -437,13 +449,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
           }
         }
       } else {
-        float *po = a.ws + ((size_t)row * a.nsplit + split) * kHeads * D;
+        __half *po = reinterpret_cast<__half *>(a.ws) + ((size_t)row * a.nsplit + split) * kHeads * D + ch;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) po[(size_t)(32 * half + j) * D + ch] = __uint_as_float(o[j]);
+        for (int j = 0; j < 32; ++j) po[(size_t)(32 * half + j) * D] = __float2half_rn(__uint_as_float(o[j]) * linv[j]);
       }
     }
     if (a.nsplit > 1 && tid < kHeads) {
-      float *pm = a.ws + nrows * a.nsplit * kHeads * D + ((size_t)row * a.nsplit + split) * kHeads;
+      float *pm = partial_stats(a, nrows) + ((size_t)row * a.nsplit + split) * kHeads;
       float *pl = pm + nrows * a.nsplit * kHeads;
       pm[tid] = S.m_ref[tid];
       pl[tid] = S.l_run[tid];
@@ -460,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   if (a.nsplit > 1) {
     cluster_sync_all();   // every split's partials are written
     const size_t nrows = (size_t)a.B * a.T_q;
-    const float *pm = a.ws + nrows * a.nsplit * kHeads * D + (size_t)row * a.nsplit * kHeads;
+    const float *pm = partial_stats(a, nrows) + (size_t)row * a.nsplit * kHeads;
     const float *pl = pm + nrows * a.nsplit * kHeads;
     if (tid < kHeads) {   // all 2 x nsplit loads in flight together
       float ms[8], ls[8];
@@ -475,52 +487,61 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       float L = 0.f;
 #pragma unroll
       for (int s = 0; s < 8; ++s) {
-        ms[s] = ms[s] == -INFINITY ? 0.f : exp2f(ms[s] - M);
-        L += ms[s] * ls[s];
+        ms[s] = ms[s] == -INFINITY ? 0.f : exp2f(ms[s] - M) * ls[s];   // the partials are O_s / l_s
+        L += ms[s];
       }
       const float inv = L > 0.f ? 1.f / L : 0.f;
 #pragma unroll
       for (int s = 0; s < 8; ++s) S.wgt[s][tid] = ms[s] * inv;
     }
     __syncthreads();
-    // this split's channel slice, in 4-channel groups
+    // this split's channel slice; item = (head, 8 channels): 16 bytes per split in, 16 bytes out
     const int cs = ((D / a.nsplit) + 7) / 8 * 8;
     const int c_lo = split * cs;
     const int c_hi = c_lo + cs < D ? c_lo + cs : D;
-    const int ng = c_hi > c_lo ? (c_hi - c_lo) / 4 : 0;
-    const float *base = a.ws + (size_t)row * a.nsplit * kHeads * D;
+    const int ng = c_hi > c_lo ? (c_hi - c_lo) / 8 : 0;
     const int n_items = a.H * ng;
+    const __half *base = reinterpret_cast<const __half *>(a.ws) + (size_t)row * a.nsplit * kHeads * D;
 #pragma unroll 1
     for (int it0 = tid; it0 < n_items; it0 += 4 * kThreads) {   // 4 items' loads in flight
-      float4 acc[4];
+      uint4 x[4][8];
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
-        acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
         const int it = it0 + v * kThreads;
-        if (it < n_items) {
-          const int h = it / ng, ch = c_lo + 4 * (it % ng);
+        const int h = it / ng, ch = c_lo + 8 * (it % ng);
 #pragma unroll
-          for (int s = 0; s < 8; ++s) {
-            if (s < a.nsplit) {
-              const float w = S.wgt[s][h];
-              const float4 x = __ldcg(reinterpret_cast<const float4 *>(base + ((size_t)s * kHeads + h) * D + ch));
-              acc[v].x += w * x.x; acc[v].y += w * x.y; acc[v].z += w * x.z; acc[v].w += w * x.w;
-            }
-          }
-        }
+        for (int s = 0; s < 8; ++s)
+          x[v][s] = (it < n_items && s < a.nsplit)
+                        ? __ldcg(reinterpret_cast<const uint4 *>(base + ((size_t)s * kHeads + h) * D + ch))
+                        : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int v = 0; v < 4; ++v) {
         const int it = it0 + v * kThreads;
-        if (it < n_items) {
-          const int h = it / ng, ch = c_lo + 4 * (it % ng);
-          const __nv_bfloat162 v0 = __floats2bfloat162_rn(acc[v].x, acc[v].y);
-          const __nv_bfloat162 v1 = __floats2bfloat162_rn(acc[v].z, acc[v].w);
-          uint2 pk;
-          pk.x = *reinterpret_cast<const uint32_t *>(&v0);
-          pk.y = *reinterpret_cast<const uint32_t *>(&v1);
-          *reinterpret_cast<uint2 *>(a.out + ((size_t)row * a.H + h) * D + ch) = pk;
+        if (it >= n_items) continue;
+        const int h = it / ng, ch = c_lo + 8 * (it % ng);
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+#pragma unroll
+        for (int s = 0; s < 8; ++s) {
+          if (s >= a.nsplit) break;
+          const float w = S.wgt[s][h];
+          const uint32_t w4[4] = {x[v][s].x, x[v][s].y, x[v][s].z, x[v][s].w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w4[i]));
+            acc[2 * i] += w * f.x;
+            acc[2 * i + 1] += w * f.y;
+          }
         }
+        uint32_t pk[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const __nv_bfloat162 bv = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+          pk[i] = *reinterpret_cast<const uint32_t *>(&bv);
+        }
+        *reinterpret_cast<uint4 *>(a.out + ((size_t)row * a.H + h) * D + ch) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
     }
   }
@@ -541,7 +562,8 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   nsplit = (nc + cps - 1) / cps;
   p.nsplit = nsplit;
   p.chunks_per_split = cps;
-  p.bytes = nsplit > 1 ? (size_t)rows * nsplit * kHeads * ((size_t)D + 2) * sizeof(float) : 0;
+  // fp16 partials [rows][nsplit][64][D] then f32 max and sum [rows][nsplit][64] each
+  p.bytes = nsplit > 1 ? (size_t)rows * nsplit * kHeads * ((size_t)D * 2 + 2 * sizeof(float)) : 0;
   return p;
 }
 

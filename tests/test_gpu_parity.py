@@ -337,6 +337,8 @@ def _check_attn(got_bf16, ref_bits):
     ref = oracle.bf16_to_f32(ref_bits).astype(np.float64)
     got = got_bf16.float().cpu().numpy().astype(np.float64)
     err = np.abs(got - ref)
+    print(f"attention error: max {err.max() / np.abs(ref).max():.2e} of max|ref|, "
+          f"mean rel {err.sum() / np.abs(ref).sum():.2e}")
     assert err.max() <= 1e-2 * np.abs(ref).max(), f"max err {err.max()} vs {np.abs(ref).max()}"
     assert err.sum() <= 1e-3 * np.abs(ref).sum(), f"mean rel err {err.sum() / np.abs(ref).sum()}"
 
