@@ -295,7 +295,16 @@ static csa2_status index_full_impl(const csa2_main_cache *main, const uint16_t *
   if ((st = device_state(&d)) != CSA2_OK) return st;
   a.ld = ld; a.n_valid = n_valid; a.status = d->status;
   a.tiles_per_row = main->cap / 128;
-  a.ctas_per_row = index_ctas_per_row(a.tiles_per_row, main->B * T_q, d->sms);
+  const int R = index_rows_per_block(T_q, false);
+  if (R == 1) {
+    a.ctas_per_row = index_ctas_per_row(a.tiles_per_row, main->B * T_q, d->sms);
+  } else {   // R rows per block, 4/R blocks per SM
+    const int64_t groups = (int64_t)main->B * T_q / R;
+    int64_t c = (int64_t)d->sms * (4 / R) / groups;
+    if (c < 1) c = 1;
+    if (c > a.tiles_per_row) c = a.tiles_per_row;
+    a.ctas_per_row = (int)c;
+  }
   cudaError_t e = launch_index(map, a, false, d->sms, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "index_full launch");
 }

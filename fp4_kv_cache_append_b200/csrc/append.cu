@@ -281,20 +281,28 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
     return;
   }
   const int e = p0;   // m = 1: token p0 completes entry p0
-  // ---- loads: this block's W_ik slice (16-byte pieces), the entry's kv pair, its window pair
-  {
-    const int ppr = OPB * 2 / 16;   // 16-byte pieces per W row of the slice
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.w_ik);
-    uint4 *dst = reinterpret_cast<uint4 *>(wsl);
-    for (int i = t; i < D * ppr; i += blockDim.x) {
-      const int r = i / ppr, j = i % ppr;
-      dst[i] = src[((size_t)r * dI + c * OPB) * 2 / 16 + j];
-    }
-  }
+  // ---- loads, all issued before any is used: the entry's kv pair, its window
+  // pair, and this block's W_ik slice (16-byte pieces, at most 4 per thread)
   uint32_t kvp = 0u, swp = 0u;
   if (t < D / 2) kvp = reinterpret_cast<const uint32_t *>(a.kv + (size_t)b * D)[t];
   const int wch = D / (2 * kDecCl);   // window channel pairs per block
   if (a.swa_rows && t < wch) swp = reinterpret_cast<const uint32_t *>(a.kv_swa + (size_t)b * D)[c * wch + t];
+  {
+    const int ppr = OPB * 2 / 16;   // 16-byte pieces per W row of the slice
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.w_ik);
+    uint4 *dst = reinterpret_cast<uint4 *>(wsl);
+    uint4 wv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = t + u * 256;
+      if (i < D * ppr) wv[u] = __ldg(src + ((size_t)(i / ppr) * dI + c * OPB) * 2 / 16 + i % ppr);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = t + u * 256;
+      if (i < D * ppr) dst[i] = wv[u];
+    }
+  }
 
   // ---- FP4: thread t < D/2 owns channels 2t, 2t+1 (8 threads per 16-channel group)
   if (t < D / 2) {

@@ -44,7 +44,7 @@ template <int DI>
 struct IndexSmem {
   alignas(1024) uint8_t tile[kStages][kTileRows * DI];   // A operand ring (K-major, swizzled)
   alignas(1024) uint8_t q8[kHeads * DI];                 // B operand (K-major, swizzled)
-  float wq[kHeads];                                      // w_h * s_q,h
+  alignas(16) float wq[kHeads];                          // w_h * s_q,h
   uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain, qbar;
   uint32_t tmem_base;
   int abort;
@@ -63,6 +63,31 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, vo
   }
   *abort = 1;
   return false;
+}
+
+// acc[0..1] += w[0..1] * x[0..1] as one packed f32x2 fused multiply-add (each
+// lane rounds exactly as a scalar fmaf).
+__device__ __forceinline__ void fma2(float &a0, float &a1, float w0, float w1, float x0, float x1) {
+  unsigned long long acc, w, x;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(acc) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(w) : "f"(w0), "f"(w1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "f"(x0), "f"(x1));
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(w), "l"(x));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a0), "=f"(a1) : "l"(acc));
+}
+
+// s4[j] += w_h * max(acc_h, 0) for heads h = j, j+4, ... of one 32-head half
+// (wq: the half's 32 weights, 16-byte aligned).
+__device__ __forceinline__ void head_reduce32(float *s4, const float *wq, const uint32_t *acc) {
+  const float4 *wp = reinterpret_cast<const float4 *>(wq);
+#pragma unroll
+  for (int h4 = 0; h4 < 8; ++h4) {
+    const float4 w = wp[h4];
+    const float r0 = fmaxf(__uint_as_float(acc[4 * h4]), 0.f), r1 = fmaxf(__uint_as_float(acc[4 * h4 + 1]), 0.f);
+    const float r2 = fmaxf(__uint_as_float(acc[4 * h4 + 2]), 0.f), r3 = fmaxf(__uint_as_float(acc[4 * h4 + 3]), 0.f);
+    fma2(s4[0], s4[1], w.x, w.y, r0, r1);
+    fma2(s4[2], s4[3], w.z, w.w, r2, r3);
+  }
 }
 
 }  // namespace
@@ -235,9 +260,7 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
           __syncwarp();
           if (lane == 0) mbar_arrive(&S.tempty[ab]);
         }
-#pragma unroll
-        for (int h = 0; h < 32; ++h)
-          s4[h & 3] = fmaf(S.wq[32 * hh + h], fmaxf(__uint_as_float(acc[h]), 0.f), s4[h & 3]);
+        head_reduce32(s4, &S.wq[32 * hh], acc);
       }
       const float sum = (s4[0] + s4[1]) + (s4[2] + s4[3]);
       float *out = a.scores + (size_t)row * a.ld;
@@ -269,9 +292,225 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
   }
 }
 
+// ---------------------------------------------------------------------------
+// Full scan of R consecutive query rows of one sequence per block (T_q >= 2:
+// multi-token decode and prefill).  The rows share the sequence's keys, so
+// each 128-entry key tile feeds one MMA with N = 64 R (the R rows' prepared
+// queries are consecutive 64-row blocks of one K-major operand), and the
+// accumulator of a tile is 64 R TMEM columns (two buffers: 128 R columns).
+//   warp 0     TMA producer (4-stage ring of key tiles)
+//   warp 1     TMEM allocation, tcgen05.mma kind::f8f6f4 M128 N(64R) K32
+//   warps 2-9  epilogue: warp w reads TMEM lane quarter w%4 and R/2 of the
+//              rows; per (entry, row) the same head reduction as the
+//              one-row kernel (chain j: heads j, j+4, ... ascending)
+// Entries beyond a row's causal limit are not written.
+constexpr int kMultiStages = 4;
+constexpr int kMultiThreads = 64 + 8 * 32;
+
+template <int DI, int R>
+struct MultiSmem {
+  alignas(1024) uint8_t tile[kMultiStages][kTileRows * DI];
+  alignas(1024) uint8_t q8[R * kHeads * DI];
+  alignas(16) float wq[R][kHeads];
+  uint64_t full[kMultiStages], empty[kMultiStages], tfull[2], tempty[2], drain, qbar;
+  uint32_t tmem_base;
+  int abort;
+  int n_issued, n_mma;
+};
+
+template <int DI, int R>
+__global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __grid_constant__ CUtensorMap ik_map,
+                                                                      const IndexArgs a) {
+  constexpr int KS = DI / 32;
+  constexpr uint32_t kCols = 2 * R * kHeads;   // 256 (R = 2) or 512 (R = 4)
+  constexpr uint32_t kIdesc = mma_idesc(128, R * kHeads, 0u /*E4M3*/, 0u /*E4M3*/);
+  constexpr int RPW = R / 2;                   // rows per epilogue warp
+  extern __shared__ uint8_t smem_raw[];
+  MultiSmem<DI, R> &S = *reinterpret_cast<MultiSmem<DI, R> *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  volatile int *abort = &S.abort;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int groups = a.T_q / R;                // row groups per sequence
+  const int b = blockIdx.y / groups;
+  const int row0 = b * a.T_q + (blockIdx.y % groups) * R;
+
+  if (tid == 0) {
+    for (int s = 0; s < kMultiStages; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
+    for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 8); }
+    mbar_init(&S.drain, 1);
+    mbar_init(&S.qbar, 1);
+    S.abort = 0;
+    S.n_issued = 0;
+    S.n_mma = 0;
+    fence_barrier_init();
+    prefetch_tmap(&ik_map);
+  }
+  if (warp == 1) {
+    tmem_alloc(&S.tmem_base, kCols);
+    tmem_relinquish();
+  }
+  pdl_wait();
+
+  // ---- the group's rows and this block's tiles (the widest row sets the range)
+  const int ne = a.n_entries[b];
+  int n_vis_max = 0;
+  int nv_mine[RPW];
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    const int t = a.q_pos[row0 + i];
+    int n = (t + 1) / a.m;
+    if (n > ne) n = ne;
+    if (n > a.cap) n = a.cap;
+    if (n < 0 || t < 0) n = 0;
+    n_vis_max = n > n_vis_max ? n : n_vis_max;
+    if (blockIdx.x == 0 && tid == 0 && a.n_valid) a.n_valid[row0 + i] = n;
+    const int half = warp >= 2 ? (warp - 2) / 4 : 0;
+    if (i / RPW == half) nv_mine[i % RPW] = n;
+  }
+  const int tiles_row = (n_vis_max + kTileRows - 1) / kTileRows;
+  const int tile0 = (int)(((int64_t)blockIdx.x * tiles_row) / gridDim.x);
+  const int tile1 = (int)(((int64_t)(blockIdx.x + 1) * tiles_row) / gridDim.x);
+  const int ntiles = tile1 - tile0;
+
+  auto issue = [&](int i) {
+    const int s = i % kMultiStages;
+    mbar_arrive_expect_tx(&S.full[s], kTileRows * DI);
+    tma_load_2d(&S.tile[s][0], &ik_map, 0, b * a.cap + (tile0 + i) * kTileRows, &S.full[s]);
+  };
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  if (ntiles > 0 && tid == 0) {
+    // the R prepared query rows are consecutive in the workspace
+    mbar_arrive_expect_tx(&S.qbar, R * kHeads * DI + R * kHeads * 4);
+    bulk_load(S.q8, a.q8 + (size_t)row0 * kHeads * DI, R * kHeads * DI, &S.qbar);
+    bulk_load(&S.wq[0][0], a.wq + (size_t)row0 * kHeads, R * kHeads * 4, &S.qbar);
+    const int first = ntiles < kMultiStages ? ntiles : kMultiStages;
+    for (int i = 0; i < first; ++i) issue(i);
+    S.n_issued = first;
+  }
+
+  if (ntiles <= 0) {
+    // nothing to score
+  } else if (warp == 0) {
+    if (lane == 0) {
+      for (int i = kMultiStages; i < ntiles; ++i) {
+        const int s = i % kMultiStages;
+        if (!wait_or_abort(&S.empty[s], ((i / kMultiStages) - 1) & 1, abort)) break;
+        issue(i);
+        S.n_issued = i + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t q_addr = smem_u32(S.q8);
+      const bool qok = wait_or_abort(&S.qbar, 0, abort);
+      for (int i = 0; i < ntiles && qok; ++i) {
+        const int s = i % kMultiStages, ab = i & 1;
+        if (!wait_or_abort(&S.full[s], (i / kMultiStages) & 1, abort)) break;
+        if (i >= 2 && !wait_or_abort(&S.tempty[ab], ((i / 2) - 1) & 1, abort)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(S.tile[s]);
+#pragma unroll
+        for (int kk = 0; kk < KS; ++kk)
+          tc_mma_f8(tmem + ab * R * kHeads, smem_desc_kmajor(a_addr + kk * 32, DI),
+                    smem_desc_kmajor(q_addr + kk * 32, DI), kIdesc, kk > 0 ? 1u : 0u);
+        tc_commit(&S.empty[s]);
+        tc_commit(&S.tfull[ab]);
+        S.n_mma = i + 1;
+      }
+    }
+  } else {
+    const int q = warp & 3;                  // TMEM lane quarter (warp w accesses lanes 32 (w % 4) ..)
+    const int half = (warp - 2) / 4;         // rows half*RPW .. half*RPW + RPW - 1
+    const int r = 32 * q + lane;
+    int qok = 1;
+    if (lane == 0) qok = wait_or_abort(&S.qbar, 0, abort);   // head weights in smem
+    qok = __shfl_sync(0xffffffffu, qok, 0);
+    for (int i = 0; i < ntiles && qok; ++i) {
+      const int ab = i & 1;
+      const int e = (tile0 + i) * kTileRows + r;
+      const float sk = e < n_vis_max ? a.ik_scale[(size_t)b * a.cap + e] : 0.f;
+      int ok = 1;
+      if (lane == 0) ok = wait_or_abort(&S.tfull[ab], (i / 2) & 1, abort);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      float sum[RPW];
+#pragma unroll
+      for (int k = 0; k < RPW; ++k) {
+        const int row = half * RPW + k;
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * R * kHeads + row * kHeads;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t acc[32];
+          tmem_ld_x32(taddr + 32 * hh, acc);
+          tmem_wait_ld();
+          if (k == RPW - 1 && hh == 1) {   // the accumulator is free once read
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&S.tempty[ab]);
+          }
+          head_reduce32(s4, &S.wq[row][32 * hh], acc);
+        }
+        sum[k] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+      }
+#pragma unroll
+      for (int k = 0; k < RPW; ++k)
+        if (e < nv_mine[k]) a.scores[(size_t)(row0 + half * RPW + k) * a.ld + e] = sum[k] * sk;
+    }
+  }
+
+  pdl_launch_dependents();
+  __syncthreads();
+  if (S.abort) {
+    if (tid == 0) {
+      flag(a.status, CSA2_DEV_TIMEOUT);
+      if (ntiles > 0) mbar_wait_bounded(&S.qbar, 0, kWaitLimit);
+      for (int j = S.n_mma; j < S.n_issued; ++j)
+        mbar_wait_bounded(&S.full[j % kMultiStages], (j / kMultiStages) & 1, kWaitLimit);
+    }
+    if (tid == 32) {
+      tc_commit(&S.drain);
+      mbar_wait_bounded(&S.drain, 0, kWaitLimit);
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
+int index_rows_per_block(int T_q, bool reindex) {
+  if (reindex) return 1;
+  if (T_q % 4 == 0) return 4;
+  if (T_q % 2 == 0) return 2;
+  return 1;
+}
+
 size_t index_workspace_bytes(int rows, int dI) {
   const size_t q = ((size_t)rows * kHeads * dI + 15) & ~size_t(15);
   return q + (size_t)rows * kHeads * 4;
+}
+
+template <int DI, int R>
+static cudaError_t launch_multi(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
+  if (!a.prepared) {
+    cudaError_t pe = launch_pdl(index_prep_kernel<DI>, dim3(a.B * a.T_q, kHeads / 8), dim3(256), 0, s, dim3(1, 1, 1), a);
+    if (pe != cudaSuccess) return pe;
+  }
+  // R = 4 takes all 512 TMEM columns: ask for enough shared memory that no
+  // second block of the kernel shares the SM (it would wait in tcgen05.alloc)
+  size_t smem = sizeof(MultiSmem<DI, R>) + 1024;
+  if (R == 4 && smem < 120 * 1024) smem = 120 * 1024;
+  auto k = index_multi_kernel<DI, R>;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(a.ctas_per_row, a.B * (a.T_q / R));
+  return launch_pdl(k, grid, dim3(kMultiThreads), smem, s, dim3(1, 1, 1), map, a);
 }
 
 template <int DI, bool REINDEX>
@@ -290,6 +529,9 @@ static cudaError_t launch_t(const CUtensorMap &map, const IndexArgs &a, cudaStre
 
 cudaError_t launch_index(const CUtensorMap &map, const IndexArgs &a, bool reindex, int sms, cudaStream_t s) {
   (void)sms;
+  const int R = index_rows_per_block(a.T_q, reindex);
+  if (R == 4) return a.dI == 128 ? launch_multi<128, 4>(map, a, s) : launch_multi<64, 4>(map, a, s);
+  if (R == 2) return a.dI == 128 ? launch_multi<128, 2>(map, a, s) : launch_multi<64, 2>(map, a, s);
   if (a.dI == 128) return reindex ? launch_t<128, true>(map, a, s) : launch_t<128, false>(map, a, s);
   return reindex ? launch_t<64, true>(map, a, s) : launch_t<64, false>(map, a, s);
 }

@@ -65,6 +65,7 @@ struct IndexArgs {
   unsigned int *status;
 };
 size_t index_workspace_bytes(int rows, int dI);
+int index_rows_per_block(int T_q, bool reindex);   // query rows sharing one scan block (1, 2 or 4)
 cudaError_t launch_index(const CUtensorMap &ik_map, const IndexArgs &a, bool reindex, int sms,
                          cudaStream_t s);
 
