@@ -90,6 +90,19 @@ __device__ __forceinline__ void head_reduce32(float *s4, const float *wq, const 
   }
 }
 
+// The same reduction for NH consecutive heads (NH a multiple of 4) with the
+// weights held in registers.
+template <int NH>
+__device__ __forceinline__ void head_reduce_reg(float *s4, const float *w, const uint32_t *acc) {
+#pragma unroll
+  for (int h4 = 0; h4 < NH / 4; ++h4) {
+    const float r0 = fmaxf(__uint_as_float(acc[4 * h4]), 0.f), r1 = fmaxf(__uint_as_float(acc[4 * h4 + 1]), 0.f);
+    const float r2 = fmaxf(__uint_as_float(acc[4 * h4 + 2]), 0.f), r3 = fmaxf(__uint_as_float(acc[4 * h4 + 3]), 0.f);
+    fma2(s4[0], s4[1], w[4 * h4], w[4 * h4 + 1], r0, r1);
+    fma2(s4[2], s4[3], w[4 * h4 + 2], w[4 * h4 + 3], r2, r3);
+  }
+}
+
 }  // namespace
 
 // Indexer query of each row (prep_query_head): grid (rows, 8) x 256 threads,
@@ -104,7 +117,6 @@ __global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
 template <int DI, bool REINDEX>
 __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constant__ CUtensorMap ik_map,
                                                             const IndexArgs a) {
-  constexpr int MASK = DI == 128 ? 7 : 3;
   constexpr int KS = DI / 32;   // MMA k-steps (32 bytes of E4M3 each)
   constexpr uint32_t kIdesc = mma_idesc(128, kHeads, 0u /*E4M3*/, 0u /*E4M3*/);
   extern __shared__ uint8_t smem_raw[];
@@ -300,12 +312,23 @@ __global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constan
 // accumulator of a tile is 64 R TMEM columns (two buffers: 128 R columns).
 //   warp 0     TMA producer (4-stage ring of key tiles)
 //   warp 1     TMEM allocation, tcgen05.mma kind::f8f6f4 M128 N(64R) K32
-//   warps 2-9  epilogue: warp w reads TMEM lane quarter w%4 and R/2 of the
-//              rows; per (entry, row) the same head reduction as the
-//              one-row kernel (chain j: heads j, j+4, ... ascending)
+//   warps 2..  epilogue, 2R warps: warp w reads TMEM lane quarter w%4 of two
+//              rows; per (entry, row) the same head reduction as the one-row
+//              kernel (chains j: heads j, j+4, ... ascending), so scores do
+//              not depend on the grouping
+// Each epilogue thread holds its two rows' 64 head weights in registers: read
+// from shared memory for every tile instead, the weights alone kept the L1
+// data pipe 80% busy (each 16-byte broadcast load takes several wavefronts).
+// The MMA issuer keeps a warp of its own: issuing the MMAs from one lane of
+// an epilogue warp (which would free registers) made the scan twice as slow.
+// With 10 warps the register budget is 168 per thread, hence 16-column TMEM
+// reads.
 // Entries beyond a row's causal limit are not written.
 constexpr int kMultiStages = 4;
-constexpr int kMultiThreads = 64 + 8 * 32;
+constexpr int kMultiChunk = 16;   // TMEM columns per tcgen05.ld + wait in the epilogue (register budget)
+constexpr int kMultiRpw = 2;      // query rows per epilogue warp
+template <int R>
+constexpr int multi_threads() { return 64 + 4 * (R / kMultiRpw) * 32; }
 
 template <int DI, int R>
 struct MultiSmem {
@@ -319,12 +342,11 @@ struct MultiSmem {
 };
 
 template <int DI, int R>
-__global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __grid_constant__ CUtensorMap ik_map,
-                                                                      const IndexArgs a) {
+__global__ void __launch_bounds__(multi_threads<R>(), 1) index_multi_kernel(const __grid_constant__ CUtensorMap ik_map,
+                                                                           const IndexArgs a) {
   constexpr int KS = DI / 32;
   constexpr uint32_t kCols = 2 * R * kHeads;   // 256 (R = 2) or 512 (R = 4)
   constexpr uint32_t kIdesc = mma_idesc(128, R * kHeads, 0u /*E4M3*/, 0u /*E4M3*/);
-  constexpr int RPW = R / 2;                   // rows per epilogue warp
   extern __shared__ uint8_t smem_raw[];
   MultiSmem<DI, R> &S = *reinterpret_cast<MultiSmem<DI, R> *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -336,7 +358,7 @@ __global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __g
 
   if (tid == 0) {
     for (int s = 0; s < kMultiStages; ++s) { mbar_init(&S.full[s], 1); mbar_init(&S.empty[s], 1); }
-    for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 8); }
+    for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 4 * R / kMultiRpw); }
     mbar_init(&S.drain, 1);
     mbar_init(&S.qbar, 1);
     S.abort = 0;
@@ -353,8 +375,8 @@ __global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __g
 
   // ---- the group's rows and this block's tiles (the widest row sets the range)
   const int ne = a.n_entries[b];
-  int n_vis_max = 0;
-  int nv_mine[RPW];
+  const int my_row = warp >= 2 ? (warp - 2) / 4 * kMultiRpw : 0;   // epilogue warps: first row they reduce
+  int n_vis_max = 0, nv_mine[kMultiRpw];
 #pragma unroll
   for (int i = 0; i < R; ++i) {
     const int t = a.q_pos[row0 + i];
@@ -364,8 +386,9 @@ __global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __g
     if (n < 0 || t < 0) n = 0;
     n_vis_max = n > n_vis_max ? n : n_vis_max;
     if (blockIdx.x == 0 && tid == 0 && a.n_valid) a.n_valid[row0 + i] = n;
-    const int half = warp >= 2 ? (warp - 2) / 4 : 0;
-    if (i / RPW == half) nv_mine[i % RPW] = n;
+#pragma unroll
+    for (int k = 0; k < kMultiRpw; ++k)
+      if (i == my_row + k) nv_mine[k] = n;
   }
   const int tiles_row = (n_vis_max + kTileRows - 1) / kTileRows;
   const int tile0 = (int)(((int64_t)blockIdx.x * tiles_row) / gridDim.x);
@@ -423,11 +446,25 @@ __global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __g
     }
   } else {
     const int q = warp & 3;                  // TMEM lane quarter (warp w accesses lanes 32 (w % 4) ..)
-    const int half = (warp - 2) / 4;         // rows half*RPW .. half*RPW + RPW - 1
     const int r = 32 * q + lane;
     int qok = 1;
     if (lane == 0) qok = wait_or_abort(&S.qbar, 0, abort);   // head weights in smem
     qok = __shfl_sync(0xffffffffu, qok, 0);
+    // the rows' head weights stay in registers: re-reading them from shared
+    // memory for every tile (64 x 128 B per warp and row) would saturate the
+    // L1 pipe
+    float wr[kMultiRpw][kHeads];
+    if (qok) {
+#pragma unroll
+      for (int k = 0; k < kMultiRpw; ++k) {
+        const float4 *wp = reinterpret_cast<const float4 *>(&S.wq[my_row + k][0]);
+#pragma unroll
+        for (int h4 = 0; h4 < kHeads / 4; ++h4) {
+          const float4 w = wp[h4];
+          wr[k][4 * h4] = w.x; wr[k][4 * h4 + 1] = w.y; wr[k][4 * h4 + 2] = w.z; wr[k][4 * h4 + 3] = w.w;
+        }
+      }
+    }
     for (int i = 0; i < ntiles && qok; ++i) {
       const int ab = i & 1;
       const int e = (tile0 + i) * kTileRows + r;
@@ -437,29 +474,25 @@ __global__ void __launch_bounds__(kMultiThreads, 1) index_multi_kernel(const __g
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      float sum[RPW];
 #pragma unroll
-      for (int k = 0; k < RPW; ++k) {
-        const int row = half * RPW + k;
-        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * R * kHeads + row * kHeads;
+      for (int k = 0; k < kMultiRpw; ++k) {
+        const uint32_t taddr = tmem + ((uint32_t)(32 * q) << 16) + ab * R * kHeads + (my_row + k) * kHeads;
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t acc[32];
-          tmem_ld_x32(taddr + 32 * hh, acc);
+        for (int c = 0; c < kHeads / kMultiChunk; ++c) {
+          uint32_t acc[kMultiChunk];
+          tmem_ld_x16(taddr + c * kMultiChunk, acc);
           tmem_wait_ld();
-          if (k == RPW - 1 && hh == 1) {   // the accumulator is free once read
+          if (k == kMultiRpw - 1 && c == kHeads / kMultiChunk - 1) {   // the accumulator is free once read
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&S.tempty[ab]);
           }
-          head_reduce32(s4, &S.wq[row][32 * hh], acc);
+          head_reduce_reg<kMultiChunk>(s4, &wr[k][c * kMultiChunk], acc);
         }
-        sum[k] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+        if (e < nv_mine[k])
+          a.scores[(size_t)(row0 + my_row + k) * a.ld + e] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * sk;
       }
-#pragma unroll
-      for (int k = 0; k < RPW; ++k)
-        if (e < nv_mine[k]) a.scores[(size_t)(row0 + half * RPW + k) * a.ld + e] = sum[k] * sk;
     }
   }
 
@@ -510,7 +543,7 @@ static cudaError_t launch_multi(const CUtensorMap &map, const IndexArgs &a, cuda
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.ctas_per_row, a.B * (a.T_q / R));
-  return launch_pdl(k, grid, dim3(kMultiThreads), smem, s, dim3(1, 1, 1), map, a);
+  return launch_pdl(k, grid, dim3(multi_threads<R>()), smem, s, dim3(1, 1, 1), map, a);
 }
 
 template <int DI, bool REINDEX>

@@ -216,6 +216,40 @@ def test_index_full_prepared_by_the_append(D, dI, H_I, T_q):
     assert C.csa2_device_status() == 0
 
 
+@pytest.mark.parametrize("T_q,m", [(8, 1), (6, 1), (4, 2)])
+def test_index_full_row_groups_match_single_rows(T_q, m):
+    """T_q a multiple of 4 (or 2) takes the multi-row scan, which puts 4 (or 2)
+    query rows on one MMA; every row's scores must equal, bit for bit, those
+    of the one-row scan of that row alone (same per-entry head reduction)."""
+    B, D, dI, H_I, n = 2, 512, 128, 64, 5000
+    cap = (n // m + 127) // 128 * 128 + 128
+    gm, _, om, _, _ = build_pair(B=B, cap=cap, D=D, dI=dI, m=m, T=n, pos0=[0, 0], seed=41 + T_q, swa=False)
+    q, w = _rows_queries(B, T_q, H_I, dI, seed=42)
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[1, 1] = 777   # rows of one group with different causal limits
+    grouped = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nval = torch.zeros(B * T_q, dtype=torch.int32, device="cuda")
+    C.csa2_index_full(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), grouped, nval)
+    single = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nv1 = torch.zeros(B, dtype=torch.int32, device="cuda")
+    for j in range(T_q):
+        out = torch.full((B, cap), float("nan"), device="cuda")
+        C.csa2_index_full(gm, q[:, j:j + 1].contiguous().cuda(), w[:, j:j + 1].contiguous().cuda(),
+                          torch.from_numpy(qpos[:, j:j + 1].copy()).cuda(), out, nv1)
+        single[j::T_q] = out
+    torch.cuda.synchronize()
+    a, b_ = grouped.cpu().numpy(), single.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b_.view(np.uint32))
+    nv = nval.cpu().numpy()
+    for b in range(B):
+        for j in (0, T_q - 1):
+            r = b * T_q + j
+            n_vis = oracle.n_visible(int(om.n_entries[b]), int(qpos[b, j]), m)
+            assert nv[r] == n_vis
+            _check_scores(a[r, :n_vis], oracle.index_scores(om, b, bits(q[b, j]), w[b, j].numpy(), n_vis))
+    assert C.csa2_device_status() == 0
+
+
 # ------------------------------------------------------------------ A4 Top-K
 
 
