@@ -39,6 +39,7 @@ WORKLOAD = "dec_full"
 WORKLOAD_DESC = ("decoder decode step, Full layer: batch 8, context 65,536, m=1, 64 heads sharing one KV of "
                  "dim 512 (FP4 E2M1 + E4M3/16ch), indexer 64x128 FP8, Top-512 + 2048x8 pool, window 128 FP8")
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -52,6 +53,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
+    ap.add_argument("--attn-sweep", action="store_true",
+                    help="print only the gather + attention batch sweep (rank 0, one GPU) and exit")
     return ap.parse_args()
 
 
@@ -65,6 +68,15 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def bf16_peak() -> float:
+    """Dense bf16 tensor TFLOP/s (burst) of MEASURED_PEAKS.json, else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return float(json.load(f)["bf16_tflops"])
+    return FALLBACK_BF16_TFLOPS
 
 
 INDEX_SOURCES = ("index.cu", "common.cuh", "kernels.h")   # what builds the index kernels
@@ -342,6 +354,71 @@ def run_ours(args, rank, world, dist):
     }
 
 
+SWEEP_ROWS = (8, 16, 32, 64, 128)
+
+
+def attn_batch_sweep(hbm, bf16_peak):
+    """Gather + attention alone (csa2_sparse_attn_decode, dec_full shapes:
+    64 heads, D 512, Top-512 + a 128-row window) at 8 ... 128 query rows.
+    Each launch is timed on its own with CUDA events, after a 256 MB write
+    that evicts the previous launch's lines from L2 (cold gathers).  Caches
+    hold 16,384 random entries per sequence (the kernel reads only the 512
+    selected rows and the window, so the context length does not enter);
+    codes are random bytes, scales E4M3 in [2^-6, 2^1], window rows positive
+    E4M3, q ~ N(0, 1).  Algorithmic bytes per row: 512 x 288 B gathered +
+    128 x 512 B window + 64 KB q + 64 KB out = 344,064 B; FLOPs per row:
+    640 keys x 64 heads x 512 x 4 = 83.9 M (S and P.V)."""
+    import math
+
+    import torch
+
+    from fp4_kv_cache_append_b200 import csa2 as C
+    from fp4_kv_cache_append_b200 import inputs as I
+    wl = I.WORKLOADS[WORKLOAD]
+    n = 16384
+    per_row_bytes = wl.K * (wl.D // 2 + wl.D // 16) + wl.window * wl.D + 2 * wl.H * wl.D * 2
+    per_row_flops = (wl.K + wl.window) * wl.H * wl.D * 4
+    g = torch.Generator(device="cuda")
+    g.manual_seed(20261202)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    res = []
+    for rows in SWEEP_ROWS:
+        main = C.MainCache(rows, n, wl.D, wl.dI, 1)
+        main.codes.random_(0, 256, generator=g)
+        main.scales.random_(0x28, 0x49, generator=g)
+        main.n_entries.fill_(n)
+        swa = C.SwaCache(rows, wl.window, wl.D)
+        swa.rows.random_(0, 0x7F, generator=g)
+        q = torch.randn(rows, 1, wl.H, wl.D, generator=g, device="cuda").to(torch.bfloat16)
+        q_pos = torch.full((rows, 1), n - 1, dtype=torch.int32, device="cuda")
+        idx = torch.rand(rows, n, generator=g, device="cuda").argsort(dim=1)[:, :wl.K]
+        idx = idx.to(torch.int32).reshape(rows, 1, wl.K).contiguous()
+        out = torch.empty(rows, 1, wl.H, wl.D, dtype=torch.bfloat16, device="cuda")
+        ws = C.workspace(C.csa2_attn_workspace_size(rows, 1, wl.H, wl.D, wl.K, wl.window))
+        call = lambda: C.csa2_sparse_attn_decode(main, swa, q, q_pos, idx, 1.0 / math.sqrt(wl.D), out, ws=ws)
+        call()
+        torch.cuda.synchronize()
+        times = []
+        for it in range(24):
+            flush.fill_(it & 255)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            call()
+            e1.record()
+            times.append((e0, e1))
+        torch.cuda.synchronize()
+        us = sorted(a.elapsed_time(b) * 1e3 for a, b in times[4:])
+        us = us[len(us) // 2]
+        gbs = rows * per_row_bytes / us / 1e3
+        tflops = rows * per_row_flops / us / 1e6
+        res.append({"rows": rows, "us": round(us, 2), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                    "tflops": round(tflops, 1), "frac_bf16": round(tflops / bf16_peak, 4)})
+        assert C.csa2_device_status() == 0
+        del main, swa, q, idx, out, ws
+    return {"per_row_bytes": per_row_bytes, "per_row_flops": per_row_flops, "timing": "median of 20 cold launches",
+            "points": res}
+
+
 def run_e2e(st, n_steps):
     """The same step through the public API with pinned host inputs: every
     step copies its inputs host->device and reads the attention output back."""
@@ -485,9 +562,15 @@ def main():
         tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                  device_id=torch.device("cuda", local))
         dist = tdist
+    if args.attn_sweep:
+        if rank == 0:
+            hbm, _ = peaks()
+            print(json.dumps({"attn_batch_sweep": attn_batch_sweep(hbm, bf16_peak())}), flush=True)
+        return
     try:
         res = run_ours(args, rank, world, dist)
         if rank == 0:
+            res["attn_batch_sweep"] = attn_batch_sweep(peaks()[0], bf16_peak())
             if world == 1 and not args.no_cpu_baseline:
                 res["cpu_baseline"] = oracle_sample(seconds=args.cpu_seconds)
             print(json.dumps(res), flush=True)

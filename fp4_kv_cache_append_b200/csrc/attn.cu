@@ -102,10 +102,17 @@ __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Key ids of tile c (threads 0..127): entry ids of the selected entries, or
-// ring slots of the window rows; -1 = masked.
-__device__ __forceinline__ void load_key_ids(const AttnArgs &a, int row, int c, int n_fp4_tiles, int wlo, int nwin,
-                                             int *dst, int tid) {
+// ring slots of the window rows; -1 = masked.  With `warm`, each thread also
+// asks L2 for its key's bytes (codes and scales, or the window row), so the
+// tile's gather, issued a few thousand cycles later, finds them there.
+template <int D>
+__device__ __forceinline__ void load_key_ids(const AttnArgs &a, int row, int b, int c, int n_fp4_tiles, int wlo,
+                                             int nwin, int *dst, int tid, bool warm) {
   if (tid >= kTile) return;
   int id = -1;
   if (c < n_fp4_tiles) {
@@ -115,9 +122,19 @@ __device__ __forceinline__ void load_key_ids(const AttnArgs &a, int row, int c, 
       if (e >= a.cap) flag(a.status, CSA2_DEV_INDEX_RANGE);
       id = (e >= 0 && e < a.cap) ? e : -1;
     }
+    if (warm && id >= 0) {
+      const size_t er = (size_t)b * a.cap + id;
+#pragma unroll
+      for (int o = 0; o < D / 2; o += 128) prefetch_l2(a.codes + er * (D / 2) + o);
+      prefetch_l2(a.scales + er * (D / 16));
+    }
   } else {
     const int j = (c - n_fp4_tiles) * kTile + tid;
     id = j < nwin ? (wlo + j) % a.W_cap : -1;
+    if (warm && id >= 0) {
+#pragma unroll
+      for (int o = 0; o < D; o += 128) prefetch_l2(a.swa_rows + ((size_t)b * a.W_cap + id) * D + o);
+    }
   }
   dst[tid] = id;
 }
@@ -178,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
     }
   }
-  if (c_begin < c_end) load_key_ids(a, row, c_begin, n_fp4_tiles, wlo, nwin, S.key_ent[c_begin & 1], tid);
+  if (c_begin < c_end) load_key_ids<D>(a, row, b, c_begin, n_fp4_tiles, wlo, nwin, S.key_ent[c_begin & 1], tid, false);
   if (tid < kHeads) { S.m_ref[tid] = -INFINITY; S.l_run[tid] = 0.f; S.alpha[tid] = 1.f; }
   tc_fence_before();
   __syncthreads();
@@ -296,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       tc_commit(&S.sbar);
     }
     // the next tile's key ids (the other buffer) while the MMAs run
-    if (c + 1 < c_end) load_key_ids(a, row, c + 1, n_fp4_tiles, wlo, nwin, S.key_ent[(c + 1) & 1], tid);
+    if (c + 1 < c_end) load_key_ids<D>(a, row, b, c + 1, n_fp4_tiles, wlo, nwin, S.key_ent[(c + 1) & 1], tid, true);
     ok = mbar_wait_bounded(&S.sbar, (c - c_begin) & 1, kWaitLimit);
     if (__syncthreads_or(!ok)) { aborted = true; break; }
     tc_fence_after();
@@ -313,17 +330,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       tmem_ld_x32(tmem + ((uint32_t)(32 * quarter) << 16) + 32 * half, rv);
       tmem_wait_ld();
       const bool valid = ids[r] >= 0;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) sv[j] = valid ? __uint_as_float(rv[j]) * lsc : -INFINITY;
+    }
+    // After the first tile the reference max usually holds: the per-head
+    // maxima are needed only when some logit exceeds it by more than 2^8.
+    bool need_max = first;
+    if (!first) {
+      const float4 *mp = reinterpret_cast<const float4 *>(&S.m_ref[32 * half]);
+      bool over = false;
+#pragma unroll
+      for (int j4 = 0; j4 < 8; ++j4) {
+        const float4 m4 = mp[j4];
+        over |= (sv[4 * j4] > m4.x + kLazy) | (sv[4 * j4 + 1] > m4.y + kLazy) | (sv[4 * j4 + 2] > m4.z + kLazy) |
+                (sv[4 * j4 + 3] > m4.w + kLazy);
+      }
+      need_max = __syncthreads_or(over);
+    }
+    if (need_max) {
       int mine = 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
-        sv[j] = valid ? __uint_as_float(rv[j]) * lsc : -INFINITY;
         const int m = __reduce_max_sync(0xffffffffu, ordered(sv[j]));
         mine = lane == j ? m : mine;
       }
       S.red[quarter][32 * half + lane] = unordered(mine);
+      __syncthreads();
     }
-    __syncthreads();
-    if (tid < kHeads) {   // new reference max of head tid
+    if (need_max && tid < kHeads) {   // new reference max of head tid
       const float m_old = S.m_ref[tid];
       const float mt = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]), fmaxf(S.red[2][tid], S.red[3][tid]));
       float al = 1.f;
@@ -340,7 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       S.alpha[tid] = al;
       S.l_run[tid] *= al;
     }
-    __syncthreads();
+    if (need_max) __syncthreads();
     // P = 2^(s - m_ref): row r of the P operand (fp16, window rows scaled)
     {
       const float4 *mp = reinterpret_cast<const float4 *>(&S.m_ref[32 * half]);
@@ -419,13 +453,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   } else {
     tc_fence_after();
     const size_t nrows = (size_t)a.B * a.T_q;
-    // split partials: O / l per head in fp16, head-major [64 heads][D]
+    // O / l per head.  One split: bf16, staged head-major [64 heads][D] in
+    // the K^ tile (free once the last O^T MMA completed), then written out in
+    // 16-byte pieces.  Several splits: fp16 partials straight from registers
+    // (a channel per lane; staging measured slower on this latency-bound path).
     float linv[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
       const float l = S.l_run[32 * half + j];
       linv[j] = l > 0.f ? 1.f / l : 0.f;
     }
+    uint16_t *ob = reinterpret_cast<uint16_t *>(S.kh);
 #pragma unroll 1
     for (int mt = 0; mt < MT; ++mt) {
       const int ch = mt * 128 + 32 * quarter + lane;
@@ -438,21 +476,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
         for (int j = 0; j < 32; ++j) o[j] = 0u;
       }
       if (a.nsplit == 1) {
-        uint16_t *orow = a.out + (size_t)row * a.H * D;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const int h = 32 * half + j;
-          if (h < a.H) {
-            const float l = S.l_run[h];
-            const __nv_bfloat16 bv = __float2bfloat16_rn(l > 0.f ? __uint_as_float(o[j]) / l : 0.f);
-            orow[(size_t)h * D + ch] = *reinterpret_cast<const uint16_t *>(&bv);
-          }
+          const __nv_bfloat16 bv = __float2bfloat16_rn(__uint_as_float(o[j]) * linv[j]);
+          ob[(32 * half + j) * D + ch] = *reinterpret_cast<const uint16_t *>(&bv);
         }
       } else {
         __half *po = reinterpret_cast<__half *>(a.ws) + ((size_t)row * a.nsplit + split) * kHeads * D + ch;
 #pragma unroll
         for (int j = 0; j < 32; ++j) po[(size_t)(32 * half + j) * D] = __float2half_rn(__uint_as_float(o[j]) * linv[j]);
       }
+    }
+    if (a.nsplit == 1) {
+      __syncthreads();
+      const uint4 *src = reinterpret_cast<const uint4 *>(ob);
+      uint4 *dst = reinterpret_cast<uint4 *>(a.out + (size_t)row * a.H * D);
+      const int n16 = a.H * (D / 8);
+#pragma unroll 4
+      for (int i = tid; i < n16; i += kThreads) dst[i] = src[i];
     }
     if (a.nsplit > 1 && tid < kHeads) {
       float *pm = partial_stats(a, nrows) + ((size_t)row * a.nsplit + split) * kHeads;
@@ -552,14 +593,20 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   AttnPlan p;
   const int rows = B * T_q;
   const int nc = (K + kTile - 1) / kTile + (window + kTile - 1) / kTile;
-  int nsplit = 1;
-  if (rows < sms) {
-    nsplit = (2 * sms + rows - 1) / rows;
-    if (nsplit > nc) nsplit = nc;
-    if (nsplit > 8) nsplit = 8;   // one cluster per row
+  // One block per SM at a time (shared memory), so a launch takes
+  // ceil(blocks / SMs) waves; a block costs one unit per key tile, plus
+  // about 0.8 for writing and merging split partials, plus 0.2 of set-up
+  // (measured per-phase cycle counts).  Take the split count of least cost
+  // (at most 8: the splits of a row form one cluster).
+  int nsplit = 1, cps = nc;
+  double best = 1e30;
+  for (int ns = 1; ns <= 8 && ns <= nc; ++ns) {
+    const int c = (nc + ns - 1) / ns;
+    const int ne = (nc + c - 1) / c;
+    const long long waves = ((long long)rows * ne + sms - 1) / sms;
+    const double cost = (double)waves * (c + (ne > 1 ? 0.8 : 0.0) + 0.2);
+    if (cost < best - 1e-9) { best = cost; nsplit = ne; cps = c; }
   }
-  const int cps = (nc + nsplit - 1) / nsplit;
-  nsplit = (nc + cps - 1) / cps;
   p.nsplit = nsplit;
   p.chunks_per_split = cps;
   // fp16 partials [rows][nsplit][64][D] then f32 max and sum [rows][nsplit][64] each
