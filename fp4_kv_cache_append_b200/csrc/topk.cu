@@ -501,11 +501,190 @@ __global__ void __launch_bounds__(kTS) topk_select_kernel(const TopkArgs a, cons
 
 size_t align16(size_t x) { return (x + 15) & ~size_t(15); }
 
+// ---------------------------------------------------------------------------
+// Many long rows (prefill chunks): one block of kRT threads per row and no
+// workspace.  The row is read once from HBM and then from L2 (the blocks
+// resident at a time hold about 2 x 148 rows, well inside L2).  A radix
+// select over the 32-bit keys in digit levels of 11, 11 and 10 bits: a
+// level's histogram counts only the keys whose higher digits equal the ones
+// fixed so far, and the selection stops as soon as the bin of the K-th key
+// is taken whole (after one or two levels for all but heavily tied rows).
+// One marking pass then sets a bitmap of the chosen columns (exact ties at
+// the last level go to the smaller columns), and a prefix popcount writes
+// them in ascending order.
+constexpr int kRT = 512;               // threads of the row kernel
+constexpr int kRowsMin = 128;          // rows from which the row kernel is used
+constexpr int kRowColsMax = 131072;    // a row's bitmaps fit in shared memory
+
+struct RowSel {
+  uint32_t prefix, mask;   // key bits fixed so far (mask: the top bits)
+  int need;                // keys still to take among those matching prefix
+  int done;                // all keys matching prefix are taken
+};
+
+// One atomic per distinct bin of the warp's active lanes.
+__device__ __forceinline__ void hist_add_match(uint32_t *h, bool act, uint32_t bin, int lane) {
+  const unsigned am = __ballot_sync(0xffffffffu, act);
+  if (!am) return;
+  const unsigned peers = __match_any_sync(0xffffffffu, act ? bin : 0xFFFFFFFFu);
+  if (act && (__ffs(peers) - 1) == lane) atomicAdd(&h[bin], (uint32_t)__popc(peers));
+}
+
+// Calls f(column, key) for every column of the row, four columns per thread
+// and step where the row is 16-byte aligned.  Every thread of the block makes
+// the same number of calls (f may use warp collectives): columns past the
+// row's end come with key 0 (absent).
+template <class F>
+__device__ __forceinline__ void for_row(const float *srow, int n, bool vec, F f) {
+  const int tid = threadIdx.x;
+  if (vec) {
+    const int n4 = n >> 2;
+    const float4 *r4 = reinterpret_cast<const float4 *>(srow);
+    for (int base = 0; base < n4; base += kRT) {
+      const int i = base + tid;
+      const float4 v = i < n4 ? r4[i] : make_float4(NAN, NAN, NAN, NAN);
+      f(4 * i, score_key(v.x));
+      f(4 * i + 1, score_key(v.y));
+      f(4 * i + 2, score_key(v.z));
+      f(4 * i + 3, score_key(v.w));
+    }
+    const int c = 4 * n4 + tid;   // the last n % 4 columns
+    f(c, c < n ? score_key(srow[c]) : 0u);
+  } else {
+    for (int base = 0; base < n; base += kRT) {
+      const int c = base + tid;
+      f(c, c < n ? score_key(srow[c]) : 0u);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kRT, 2) topk_rows_kernel(const TopkArgs a) {
+  extern __shared__ uint32_t smr[];
+  const int nwords = (a.n_cols + 31) >> 5;
+  uint32_t *hist = smr;                       // [kBins]
+  uint32_t *bitmap = smr + kBins;             // [nwords] chosen columns
+  uint32_t *tiemap = bitmap + nwords;         // [nwords] exact ties at the last level
+  __shared__ RowSel st;
+  __shared__ int red[40];
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float *srow = a.scores + (size_t)row * a.ld;
+  const int n = row_cols(a, row);
+  const bool vec = (a.ld & 3) == 0;
+  for (int i = tid; i < nwords; i += kRT) { bitmap[i] = 0u; tiemap[i] = 0u; }
+  if (tid == 0) { st.prefix = 0u; st.mask = 0u; st.need = a.K; st.done = 0; }
+  __syncthreads();
+#pragma unroll 1
+  for (int lv = 0; lv < 3; ++lv) {
+    const int sh = lv == 0 ? 21 : (lv == 1 ? 10 : 0);
+    const uint32_t dm = lv == 2 ? 0x3FFu : 0x7FFu;
+    for (int i = tid; i < kBins; i += kRT) hist[i] = 0u;
+    __syncthreads();
+    const uint32_t prefix = st.prefix, mask = st.mask;
+    for_row(srow, n, vec, [&](int, uint32_t key) {
+      const bool act = key != 0u && (key & mask) == prefix;
+      hist_add_match(hist, act, (key >> sh) & dm, lane);
+    });
+    __syncthreads();
+    int T, above;
+    find_threshold<kRT>(hist, st.need, T, above, red);
+    if (tid == 0) {
+      if (T < 0) {
+        st.done = 1;   // the matching keys are fewer than need: all taken
+      } else {
+        st.need -= above;
+        st.prefix |= (uint32_t)T << sh;
+        st.mask |= dm << sh;
+        if (hist[T] == (uint32_t)st.need) st.done = 1;
+      }
+    }
+    __syncthreads();
+    if (st.done) break;
+  }
+  // marking pass: keys above the fixed digits, and the matching ones (all of
+  // them when done, else exact ties: the need smallest columns)
+  {
+    const uint32_t prefix = st.prefix, mask = st.mask;
+    const bool done = st.done != 0;
+    for_row(srow, n, vec, [&](int c, uint32_t key) {
+      if (key == 0u) return;
+      const uint32_t top = key & mask;
+      if (top > prefix || (done && top == prefix)) atomicOr(&bitmap[c >> 5], 1u << (c & 31));
+      else if (top == prefix) atomicOr(&tiemap[c >> 5], 1u << (c & 31));
+    });
+  }
+  __syncthreads();
+  const int per = (nwords + kRT - 1) / kRT;
+  const int w0 = tid * per, w1 = min(w0 + per, nwords);
+  if (!st.done) {   // the first need tie columns join the chosen ones
+    int mine = 0;
+    for (int wi = w0; wi < w1; ++wi) mine += __popc(tiemap[wi]);
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) red[warp] = incl;
+    __syncthreads();
+    int before = incl - mine;
+#pragma unroll
+    for (int w = 0; w < kRT / 32; ++w)
+      if (w < warp) before += red[w];
+    const int need = st.need;
+    for (int wi = w0; wi < w1 && before < need; ++wi) {
+      uint32_t bits = tiemap[wi], take = 0u;
+      while (bits && before < need) {
+        const uint32_t b = bits & (0u - bits);
+        take |= b;
+        bits ^= b;
+        ++before;
+      }
+      bitmap[wi] |= take;
+    }
+    __syncthreads();
+  }
+  // ascending output by prefix popcount over the chosen columns
+  int mine = 0;
+  for (int wi = w0; wi < w1; ++wi) mine += __popc(bitmap[wi]);
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) red[warp] = incl;
+  __syncthreads();
+  int before = incl - mine, total = 0;
+#pragma unroll
+  for (int w = 0; w < kRT / 32; ++w) {
+    const int v = red[w];
+    if (w < warp) before += v;
+    total += v;
+  }
+  int32_t *out = a.out_idx + (size_t)row * a.K;
+  const int32_t *pb = a.pool_blocks ? a.pool_blocks + (size_t)row * (a.n_cols / 8) : nullptr;
+  for (int wi = w0; wi < w1; ++wi) {
+    uint32_t bits = bitmap[wi];
+    while (bits) {
+      const int bpos = __ffs(bits) - 1;
+      bits &= bits - 1;
+      const int c = wi * 32 + bpos;
+      if (before < a.K) out[before] = pb ? pb[c >> 3] * 8 + (c & 7) : c;
+      ++before;
+    }
+  }
+  for (int i = total + tid; i < a.K; i += kRT) out[i] = -1;
+}
+
+bool topk_rows_path(int rows, int n_cols, int P_out) {
+  return rows >= kRowsMin && !topk_cluster_fits(n_cols) && n_cols <= kRowColsMax && P_out == 0;
+}
+
 }  // namespace
 
 TopkPlan plan_topk(int rows, int n_cols, int K, int P_out) {
   TopkPlan p{};
-  if (topk_cluster_fits(n_cols)) return p;   // the cluster kernel needs no workspace
+  if (topk_cluster_fits(n_cols) || topk_rows_path(rows, n_cols, P_out)) return p;   // no workspace
   p.nchunks = n_cols > 0 ? (n_cols + kColsPerBlock - 1) / kColsPerBlock : 1;
   p.nb = (n_cols + 7) / 8;
   const size_t R = (size_t)(rows > 0 ? rows : 0);
@@ -534,6 +713,13 @@ TopkPlan plan_topk(int rows, int n_cols, int K, int P_out) {
 
 cudaError_t launch_topk(const TopkArgs &a, const TopkPlan &p, cudaStream_t s) {
   if (topk_cluster_fits(a.n_cols)) return launch_topk_cluster(a, s);
+  if (topk_rows_path(a.rows, a.n_cols, a.P_out)) {
+    const size_t sm = sizeof(uint32_t) * (kBins + 2 * (((size_t)a.n_cols + 31) / 32));
+    cudaError_t e = cudaFuncSetAttribute(topk_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+    if (e != cudaSuccess) return e;
+    topk_rows_kernel<<<a.rows, kRT, sm, s>>>(a);
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaMemsetAsync(a.ws, 0, p.zero_bytes, s);
   if (e != cudaSuccess) return e;
   if (a.n_cols > 0) {

@@ -107,6 +107,30 @@ def test_append_decode_single_token_and_ring_wrap(D, dI, with_window):
         assert_cache_equal(gm, om)
 
 
+@pytest.mark.parametrize("D,s_swa", [(512, 1.0), (256, 0.5)])
+def test_swa_replay_rebuild_matches_incremental_ring(D, s_swa):
+    """SWA bounded replay: re-encoding the last 128 tokens' window rows with
+    one window-only append (no main cache) into an empty ring gives the same
+    ring bytes as the ring built token by token, and as the oracle's."""
+    B, W_cap, n = 2, 128, 300
+    g = gen(61 + D)
+    kvs = torch.randn(B, n, D, generator=g).to(torch.bfloat16)
+    inc = C.SwaCache(B, W_cap, D, scale=s_swa)
+    osw = oracle.SwaCache(B, W_cap, D, s_swa, 128)
+    for t in range(n):   # decode-style: one token per call
+        pos = torch.full((B,), t, dtype=torch.int32)
+        C.csa2_append_quant(None, None, None, None, inc, kvs[:, t:t + 1].contiguous().cuda(), pos.cuda(), 1)
+    oracle.append(None, None, None, None, osw, bits(kvs), np.zeros(B, np.int32), n)
+    reb = C.SwaCache(B, W_cap, D, scale=s_swa)
+    first = n - W_cap
+    C.csa2_append_quant(None, None, None, None, reb, kvs[:, first:].contiguous().cuda(),
+                        torch.full((B,), first, dtype=torch.int32).cuda(), W_cap)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(reb.rows.cpu().numpy(), inc.rows.cpu().numpy())
+    np.testing.assert_array_equal(reb.rows.cpu().numpy(), osw.rows)
+    assert C.csa2_device_status() == 0
+
+
 def test_append_m2_pending_across_calls():
     B, D, dI, cap = 2, 256, 64, 256
     g = gen(5)
@@ -321,6 +345,43 @@ def test_topk_exact_on_hard_distributions(kind, n):
     np.testing.assert_array_equal(out.cpu().numpy(), _ref_topk_rows(s, n_valid, K))
     refp = np.stack([oracle.block_pool(s[r, :n_valid[r]].astype(np.float64), P) for r in range(rows)])
     np.testing.assert_array_equal(pool.cpu().numpy(), refp)
+
+
+@pytest.mark.parametrize("kind", ["normal", "outlier", "constant", "huge_range", "two_clusters", "tiny", "few_values"])
+@pytest.mark.parametrize("pad", [3, 0])
+def test_topk_many_long_rows(kind, pad):
+    """128 or more rows of more than 65,536 columns (prefill chunks) take the
+    one-block-per-row kernel, which needs no workspace: exact against the
+    oracle with ragged n_valid, absent scores, rows shorter than K or empty,
+    and a row pitch that is (pad 3: 70,004) or is not (pad 0: 70,001) a
+    multiple of 4."""
+    rows, n, K = 136, 70001, 512
+    ld = n + pad
+    rng = np.random.default_rng(zlib.crc32(f"rows/{kind}/{pad}".encode()))
+    s = rng.standard_normal((rows, n)).astype(np.float32) if kind == "normal" else _hard_scores(kind, rows, n, rng)
+    s[1, rng.choice(n, n // 10, replace=False)] = -np.inf
+    n_valid = rng.integers(n // 2, n + 1, rows).astype(np.int32)
+    n_valid[2], n_valid[3], n_valid[4] = 300, 0, n
+    buf = np.full((rows, ld), np.nan, np.float32)
+    buf[:, :n] = s
+    assert C.csa2_topk_workspace_size(rows, n, K, 0) == 0
+    out = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    C.csa2_topk(torch.from_numpy(buf).cuda(), n, K, out, n_valid=torch.from_numpy(n_valid).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy(), _ref_topk_rows(s, n_valid, K))
+    assert C.csa2_device_status() == 0
+
+
+@pytest.mark.parametrize("rows,n,K", [(128, 131072, 2048), (200, 65537, 1), (128, 100000, 2000)])
+def test_topk_many_long_rows_extremes(rows, n, K):
+    rng = np.random.default_rng(zlib.crc32(f"rowsx/{rows}/{n}/{K}".encode()))
+    s = rng.standard_normal((rows, n)).astype(np.float32)
+    s[:, : n // 7] = np.round(s[:, : n // 7] * 4) / 4   # a tied stretch
+    n_valid = np.full(rows, n, np.int32)
+    out = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    C.csa2_topk(torch.from_numpy(s).cuda(), n, K, out, n_valid=torch.from_numpy(n_valid).cuda())
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy(), _ref_topk_rows(s, n_valid, K))
 
 
 def test_topk_pool_mapping_for_reindex_rows():
