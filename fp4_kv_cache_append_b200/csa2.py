@@ -115,10 +115,17 @@ class MainCache:
         self.pending_kv = torch.zeros(B, D, dtype=torch.bfloat16, device=device)
         self.pending_gate = torch.zeros(B, D, dtype=torch.bfloat16, device=device)
 
+    def __setattr__(self, name, value):   # any change rebuilds the descriptor
+        object.__setattr__(self, name, value)
+        object.__setattr__(self, "_desc", None)
+
     def desc(self) -> MainCacheDesc:
-        return MainCacheDesc(self.codes.data_ptr(), self.scales.data_ptr(), self.ik.data_ptr(),
-                             self.ik_scale.data_ptr(), self.n_entries.data_ptr(), self.pending_kv.data_ptr(),
-                             self.pending_gate.data_ptr(), self.B, self.cap, self.D, self.d_I, self.m)
+        if self._desc is None:
+            object.__setattr__(self, "_desc", MainCacheDesc(
+                self.codes.data_ptr(), self.scales.data_ptr(), self.ik.data_ptr(), self.ik_scale.data_ptr(),
+                self.n_entries.data_ptr(), self.pending_kv.data_ptr(), self.pending_gate.data_ptr(), self.B,
+                self.cap, self.D, self.d_I, self.m))
+        return self._desc
 
     @property
     def nbytes(self) -> int:
@@ -134,8 +141,15 @@ class SwaCache:
         self.B, self.W_cap, self.D, self.scale, self.window = B, W_cap, D, float(scale), window
         self.rows = torch.zeros(B, W_cap, D, dtype=torch.uint8, device=device)
 
+    def __setattr__(self, name, value):   # any change rebuilds the descriptor
+        object.__setattr__(self, name, value)
+        object.__setattr__(self, "_desc", None)
+
     def desc(self) -> SwaCacheDesc:
-        return SwaCacheDesc(self.rows.data_ptr(), self.scale, self.B, self.W_cap, self.D, self.window)
+        if self._desc is None:
+            object.__setattr__(self, "_desc", SwaCacheDesc(self.rows.data_ptr(), self.scale, self.B, self.W_cap,
+                                                           self.D, self.window))
+        return self._desc
 
 
 # --------------------------------------------------------------------------- entry points

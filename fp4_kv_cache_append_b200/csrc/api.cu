@@ -399,6 +399,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   if (p.nsplit > 1 && (!ws || ws_bytes < p.bytes || !aligned16(ws))) {   // no workspace: one block per row
     p.nsplit = 1;
     p.chunks_per_split = 1 << 20;
+    p.csplit = 1;
   }
   AttnArgs a{};
   a.codes = main->codes; a.scales = main->scales; a.cap = main->cap; a.D = main->D;
@@ -406,7 +407,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   a.q = q; a.q_pos = q_pos; a.B = main->B; a.T_q = T_q; a.H = H; a.idx = idx; a.K = K;
   a.scale = softmax_scale; a.out = out;
   a.ws = p.nsplit > 1 ? static_cast<float *>(ws) : nullptr;
-  a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.status = d->status;
+  a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.csplit = p.csplit; a.status = d->status;
   cudaError_t e = launch_attn(a, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "attention launch");
 }

@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   const int row = blockIdx.x;   // b * T_q + query
   const int split = blockIdx.y;
   const int b = row / a.T_q;
+  const int mt_lo = (int)blockIdx.z * (MT / a.csplit), mt_hi = mt_lo + MT / a.csplit;   // O^T blocks of this block
   pdl_launch_dependents();
 
   // ---- set-up that touches no global memory overlaps the previous kernel
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     // rare: a head's reference max moved -> rescale its O^T column
     if (S.rescale) {
 #pragma unroll 1
-      for (int mt = 0; mt < MT; ++mt) {
+      for (int mt = mt_lo; mt < mt_hi; ++mt) {
         const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + kHeads + mt * kHeads + 32 * half;
         uint32_t o[32];
         tmem_ld_x32(taddr, o);
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       const uint64_t db = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
+        if (mt < mt_lo || mt >= mt_hi) continue;
 #pragma unroll
         for (int ks = 0; ks < kTile / 16; ++ks)
           tc_mma_f16(tmem + kHeads + mt * kHeads, da + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
@@ -465,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     }
     uint16_t *ob = reinterpret_cast<uint16_t *>(S.kh);
 #pragma unroll 1
-    for (int mt = 0; mt < MT; ++mt) {
+    for (int mt = mt_lo; mt < mt_hi; ++mt) {
       const int ch = mt * 128 + 32 * quarter + lane;
       uint32_t o[32];
       if (n_done > 0) {
@@ -537,9 +539,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     }
     __syncthreads();
     // this split's channel slice; item = (head, 8 channels): 16 bytes per split in, 16 bytes out
-    const int cs = ((D / a.nsplit) + 7) / 8 * 8;
-    const int c_lo = split * cs;
-    const int c_hi = c_lo + cs < D ? c_lo + cs : D;
+    const int Dz = D / a.csplit, z_lo = (int)blockIdx.z * Dz;   // this block's channel half (or all)
+    const int cs = ((Dz / a.nsplit) + 7) / 8 * 8;
+    const int c_lo = z_lo + split * cs;
+    const int c_hi = c_lo + cs < z_lo + Dz ? c_lo + cs : z_lo + Dz;
     const int ng = c_hi > c_lo ? (c_hi - c_lo) / 8 : 0;
     const int n_items = a.H * ng;
     const __half *base = reinterpret_cast<const __half *>(a.ws) + (size_t)row * a.nsplit * kHeads * D;
@@ -609,6 +612,9 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   }
   p.nsplit = nsplit;
   p.chunks_per_split = cps;
+  // small batches: two blocks per split, each issuing the O^T MMAs of, and
+  // writing and merging, half of the channels (both compute S and P)
+  p.csplit = (nsplit > 1 && D % 256 == 0 && (long long)rows * nsplit * 2 <= sms) ? 2 : 1;
   // fp16 partials [rows][nsplit][64][D] then f32 max and sum [rows][nsplit][64] each
   p.bytes = nsplit > 1 ? (size_t)rows * nsplit * kHeads * ((size_t)D * 2 + 2 * sizeof(float)) : 0;
   return p;
@@ -619,7 +625,8 @@ static cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s) {
   const size_t smem = sizeof(AttnSmem<D>) + 1024;
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_kernel<D>, dim3(a.B * a.T_q, a.nsplit), dim3(kThreads), smem, s, dim3(1, (unsigned)a.nsplit, 1),
+  return launch_pdl(attn_kernel<D>, dim3(a.B * a.T_q, a.nsplit, a.csplit), dim3(kThreads), smem, s,
+                    dim3(1, (unsigned)a.nsplit, 1),
                     a);
 }
 

@@ -136,10 +136,11 @@ struct AttnArgs {
   uint16_t *out;          // [B][T_q][H][D]
   float *ws;              // split partials (nullptr when unsplit)
   int nsplit, chunks_per_split;
+  int csplit;             // 2: a pair of blocks per split, each with half of the O channels
   unsigned int *status;
 };
 struct AttnPlan {
-  int nsplit, chunks_per_split;
+  int nsplit, chunks_per_split, csplit;
   size_t bytes;
 };
 AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms);
