@@ -241,10 +241,10 @@ csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uint16_t *kv
   return append_impl(main, kv, gate, w_ik, swa, kv_swa, pos0, T, &p, stream);
 }
 
-// Blocks per row of a scan: about three resident blocks per SM in one wave,
+// Blocks per row of a scan: about four resident blocks per SM in one wave,
 // the row's tiles split evenly over them.
 static int index_ctas_per_row(int tiles_per_row, int rows, int sms) {
-  int64_t c = (int64_t)sms * 3 / rows;
+  int64_t c = (int64_t)sms * 4 / rows;
   if (c < 1) c = 1;
   if (c > tiles_per_row) c = tiles_per_row;
   return (int)c;

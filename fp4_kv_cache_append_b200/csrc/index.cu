@@ -19,7 +19,7 @@
 //              s_k * sum_h (w_h s_q,h) * max(acc_h, 0) -> one fp32 score
 // The head reduction never leaves registers; scores are written once,
 // coalesced.  The visible tiles of a row are split evenly over the row's
-// blocks (about three blocks per SM in one wave).  The FP8 query of each row
+// blocks (about four blocks per SM in one wave).  The FP8 query of each row
 // is prepared once (index_prep_kernel, or by the append launch that precedes
 // the scan: csa2_append_quant_ex) into the caller's workspace, already in the
 // MMA's swizzled layout, and bulk-copied into every block of that row.  All
@@ -115,7 +115,7 @@ __global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
 }
 
 template <int DI, bool REINDEX>
-__global__ void __launch_bounds__(kThreads, 3) index_kernel(const __grid_constant__ CUtensorMap ik_map,
+__global__ void __launch_bounds__(kThreads, 4) index_kernel(const __grid_constant__ CUtensorMap ik_map,
                                                             const IndexArgs a) {
   constexpr int KS = DI / 32;   // MMA k-steps (32 bytes of E4M3 each)
   constexpr uint32_t kIdesc = mma_idesc(128, kHeads, 0u /*E4M3*/, 0u /*E4M3*/);

@@ -466,6 +466,29 @@ def test_attention_vs_oracle(D, H, K, T_q, window, W_cap, use_ws):
     assert C.csa2_device_status() == 0
 
 
+@pytest.mark.parametrize("B,T_q", [(8, 4), (16, 4), (40, 4)])
+def test_attention_multi_tile_splits(B, T_q):
+    """Row counts where the launch plan gives splits of several key tiles
+    each (32 rows: 3 splits of 2 tiles; 64 rows: 2 splits of 3; 160 rows:
+    one block per row over all 5 tiles): sampled rows against the oracle."""
+    D, H, K, n, cap = 512, 64, 512, 2000, 2048
+    gm, gs, om, osw, _ = build_pair(B=B, cap=cap, D=D, dI=64, m=1, T=n, pos0=[0] * B, seed=77 + B, s_swa=0.5)
+    g = gen(78)
+    q = torch.randn(B, T_q, H, D, generator=g).to(torch.bfloat16)
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    idx = torch.stack([torch.stack([I.random_indices(int(qpos[b, j]) + 1, K, g, n_missing=(b + j) % 3)
+                                    for j in range(T_q)]) for b in range(B)])
+    out = torch.empty(B, T_q, H, D, dtype=torch.bfloat16, device="cuda")
+    ws = C.workspace(C.csa2_attn_workspace_size(B, T_q, H, D, K, 128))
+    scale = 1 / math.sqrt(D)
+    C.csa2_sparse_attn_decode(gm, gs, q.cuda(), torch.from_numpy(qpos).cuda(), idx.cuda(), scale, out, ws=ws)
+    torch.cuda.synchronize()
+    for b, j in [(0, 0), (B // 2, 1), (B - 1, T_q - 1)]:
+        ref = oracle.attention(om, osw, b, bits(q[b, j]), idx[b, j].numpy(), int(qpos[b, j]), scale)
+        _check_attn(out[b, j], ref)
+    assert C.csa2_device_status() == 0
+
+
 def test_attention_out_of_range_index_is_masked_and_flagged():
     B, D, n, cap, K = 1, 128, 300, 384, 16
     gm, gs, om, osw, _ = build_pair(B=B, cap=cap, D=D, dI=64, m=1, T=n, pos0=[0], seed=41)
