@@ -42,6 +42,11 @@ constexpr int kHeads = 64;         // heads padded to 64 (N)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.0f;      // log2 headroom before the reference max moves
 constexpr uint32_t kWaitLimit = 1u << 22;
+// Merge items (head, 8 channels) per thread whose loads are in flight
+// together.  Each block runs the merge once, from a cold instruction cache,
+// so its unrolled size matters: 2 items keep one round of L2 reads for a
+// dec_full split (448 items) at 10 KB less code than 4.
+constexpr int kMergeItems = 2;
 
 template <int D>
 struct AttnSmem {
@@ -547,10 +552,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     const int n_items = a.H * ng;
     const __half *base = reinterpret_cast<const __half *>(a.ws) + (size_t)row * a.nsplit * kHeads * D;
 #pragma unroll 1
-    for (int it0 = tid; it0 < n_items; it0 += 4 * kThreads) {   // 4 items' loads in flight
-      uint4 x[4][8];
+    for (int it0 = tid; it0 < n_items; it0 += kMergeItems * kThreads) {   // kMergeItems items' loads in flight
+      uint4 x[kMergeItems][8];
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
+      for (int v = 0; v < kMergeItems; ++v) {
         const int it = it0 + v * kThreads;
         const int h = it / ng, ch = c_lo + 8 * (it % ng);
 #pragma unroll
@@ -560,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
                         : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
+      for (int v = 0; v < kMergeItems; ++v) {
         const int it = it0 + v * kThreads;
         if (it >= n_items) continue;
         const int h = it / ng, ch = c_lo + 8 * (it % ng);
