@@ -84,6 +84,23 @@ __device__ __forceinline__ void reduce_scatter32(float *t, int lane) {
   }
 }
 
+// After the call, lane l holds in t[0] the maximum over the warp of column l
+// (the same transposing butterfly; t is consumed).
+__device__ __forceinline__ void reduce_scatter32_max(float *t, int lane) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < o) {
+        const float lo = t[j], hi = t[j + o];
+        const float recv = __shfl_xor_sync(0xffffffffu, up ? lo : hi, o);
+        t[j] = fmaxf(up ? hi : lo, recv);
+      }
+    }
+  }
+}
+
 // 2^x by the hardware's approximate exponential (relative error ~2^-22,
 // far below the fp16 rounding of P it feeds).
 __device__ __forceinline__ float ex2_approx(float x) {
@@ -92,11 +109,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-__device__ __forceinline__ int ordered(float f) {
-  const int b = __float_as_int(f);
-  return b >= 0 ? b : (b ^ 0x7FFFFFFF);
-}
-__device__ __forceinline__ float unordered(int k) { return __int_as_float(k >= 0 ? k : (k ^ 0x7FFFFFFF)); }
 
 // f32 (max, sum) per (row, split, head), after the fp16 partials.
 __device__ __forceinline__ float *partial_stats(const AttnArgs &a, size_t nrows) {
@@ -331,14 +343,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     const bool first = (c == c_begin);
     const int r = 32 * quarter + lane;
     float sv[32];
-    {
+    const bool valid = ids[r] >= 0;
+    auto load_logits = [&]() {
       uint32_t rv[32];
       tmem_ld_x32(tmem + ((uint32_t)(32 * quarter) << 16) + 32 * half, rv);
       tmem_wait_ld();
-      const bool valid = ids[r] >= 0;
 #pragma unroll
       for (int j = 0; j < 32; ++j) sv[j] = valid ? __uint_as_float(rv[j]) * lsc : -INFINITY;
-    }
+    };
+    load_logits();
     // After the first tile the reference max usually holds: the per-head
     // maxima are needed only when some logit exceeds it by more than 2^8.
     bool need_max = first;
@@ -354,14 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       need_max = __syncthreads_or(over);
     }
     if (need_max) {
-      int mine = 0;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const int m = __reduce_max_sync(0xffffffffu, ordered(sv[j]));
-        mine = lane == j ? m : mine;
-      }
-      S.red[quarter][32 * half + lane] = unordered(mine);
+      // per-head maxima of this warp's 32 keys (the butterfly consumes sv;
+      // the logits are read from TMEM again afterwards)
+      reduce_scatter32_max(sv, lane);
+      S.red[quarter][32 * half + lane] = sv[0];
       __syncthreads();
+      load_logits();
     }
     if (need_max && tid < kHeads) {   // new reference max of head tid
       const float m_old = S.m_ref[tid];
