@@ -199,7 +199,11 @@ CSA2_API csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint1
  *  out_pool [rows][P_out] i32 out (P_out > 0, pool_blocks NULL): the P_out
  *         blocks of 8 columns with the largest block maximum (ties -> smaller
  *         block), ascending, -1 padded
- *  ws, ws_bytes: workspace of csa2_topk_workspace_size(rows, n_cols, K, P_out)
+ *  ws, ws_bytes: workspace of csa2_topk_workspace_size(rows, n_cols, K, P_out);
+ *         none (size 0, ws may be NULL) for rows of at most 65,536 columns
+ *         (one thread-block cluster per row) and for 128 or more rows of at
+ *         most 131,072 columns without a pool (one block per row, the row
+ *         re-read from L2: prefill chunks)
  * Supported: 1 <= K <= 2048, 0 <= P_out <= 4096, n_cols <= 2^20.
  */
 CSA2_API csa2_status csa2_topk(const float *scores, int rows, int64_t ld, int n_cols,

@@ -71,6 +71,12 @@ def test_workspace_sizes_are_pure_host_functions():
     assert C.csa2_topk_workspace_size(8, 100000, 512, 2048) > 0
     assert C.csa2_topk_workspace_size(8, 65536, 512, 2048) == 0   # single-launch cluster path
     assert C.csa2_topk_workspace_size(0, 65536, 512, 2048) == 0
+    # many long rows without a pool: one block per row, no workspace
+    assert C.csa2_topk_workspace_size(8192, 69632, 512, 0) == 0
+    assert C.csa2_topk_workspace_size(128, 131072, 2048, 0) == 0
+    assert C.csa2_topk_workspace_size(127, 69632, 512, 0) > 0      # too few rows
+    assert C.csa2_topk_workspace_size(128, 69632, 512, 2048) > 0   # a pool is asked for
+    assert C.csa2_topk_workspace_size(128, 131073, 512, 0) > 0     # the row's bitmaps exceed shared memory
 
 
 def test_binding_marshals_every_entry_point_without_a_gpu():
