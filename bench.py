@@ -18,7 +18,9 @@ barrier and a device synchronisation, the maximum over ranks.  With N > 1
 data-path collective.  Prints one JSON line on rank 0.
 
 --impl reference times the CPU oracle (oracle/) on this machine's host cores
-on a bounded sample of the same workload.
+on a bounded sample of the same workload: one sequence's append, Full scores
+over a slice of its entries, Top-K and pool over that slice and attention,
+extrapolated to the whole step (oracle_sample).
 """
 from __future__ import annotations
 
