@@ -85,7 +85,7 @@ csa2_status get_encoder(EncodeTiled *fn) {
 // rows x d_I bytes (128: a whole Full tile per copy; 8: one pool block),
 // swizzled to the d_I-byte pattern of the MMA's shared-memory descriptors.
 csa2_status encode_ik_map(const csa2_main_cache *m, CUtensorMap *map, int box_rows) {
-  EncodeTiled enc;
+  EncodeTiled enc = nullptr;
   csa2_status st = get_encoder(&enc);
   if (st != CSA2_OK) return st;
   cuuint64_t dims[2] = {(cuuint64_t)m->d_I, (cuuint64_t)m->B * (cuuint64_t)m->cap};
