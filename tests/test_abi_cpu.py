@@ -79,6 +79,21 @@ def test_workspace_sizes_are_pure_host_functions():
     assert C.csa2_topk_workspace_size(128, 131073, 512, 0) > 0     # the row's bitmaps exceed shared memory
 
 
+@pytest.mark.parametrize("rows,nsplit", [(1, 5), (8, 5), (24, 5), (32, 3), (48, 3), (64, 2), (74, 2), (96, 1),
+                                         (128, 1), (8192, 1)])
+def test_attention_split_plan(rows, nsplit):
+    """The attention launch plan (no GPU here: 148 SMs assumed) minimises
+    waves x (tiles per split + merge): its workspace holds the fp16 partials
+    and the f32 (max, sum) of every split, none when a row is not split."""
+    D, H, K, window = 512, 64, 512, 128
+    per_split = 64 * (D * 2 + 8)
+    expect = rows * nsplit * per_split if nsplit > 1 else 0
+    assert C.csa2_attn_workspace_size(rows, 1, H, D, K, window) == expect
+    # the plan depends on rows = B x T_q only
+    if rows % 4 == 0:
+        assert C.csa2_attn_workspace_size(rows // 4, 4, H, D, K, window) == expect
+
+
 def test_binding_marshals_every_entry_point_without_a_gpu():
     """Each Python wrapper reaches the library (which then reports that it
     cannot run here) instead of failing in its own argument handling."""
