@@ -26,9 +26,16 @@
 // The splits of one row form a thread-block cluster: each writes O / l per
 // head (fp16, [head][channel]) and its (max, sum) per head to the workspace, and
 // after one cluster barrier each split merges a slice of the channels from all
-// splits (weights 2^(m_s - M) l_s / L) and writes the bf16 output.  Straight-line code is kept short (rolled
-// loops): each block runs it about once, so fetching it costs as much as
-// executing it.
+// splits (weights 2^(m_s - M) l_s / L) and writes the bf16 output.
+// Launch shape (plan_attn): the split count minimises waves x (tiles per split
+// + merge cost) with one block per SM; at small batch each split is a pair of
+// blocks (grid z) that both compute S and P and each issue the O^T MMAs of,
+// write and merge half of the channels.  A block that runs several tiles has
+// L2 fetch the next tile's rows during the current tile's MMAs and skips the
+// per-head max reduction while the reference max holds.
+// Each block runs its code about once, from a cold instruction cache, so the
+// unrolled size of the straight-line parts (merge, maxima) is kept down:
+// fetching code costs as much as executing it here.
 #include "common.cuh"
 #include "kernels.h"
 
