@@ -1,6 +1,8 @@
-// Top-K selection and the hierarchical candidate pool (rows of more than
-// 65,536 columns; shorter rows use the single-launch cluster kernel of
-// topk_cluster.cu).
+// Top-K selection and the hierarchical candidate pool for rows of more than
+// 65,536 columns (shorter rows use the single-launch cluster kernel of
+// topk_cluster.cu): 128 or more rows of at most 131,072 columns without a
+// pool take topk_rows_kernel (one block per row, below); the other shapes the
+// four-kernel path described here.
 //   DeepSeek-V4.1-Flash (jaehun.me review), section "2) CSA2": each Full or
 //   Reindex layer keeps the Top-512 entries; the first Full layer of the
 //   decoder also builds the pool of <= 2,048 blocks x 8 positions that the
