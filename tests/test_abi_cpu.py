@@ -67,6 +67,33 @@ def test_host_validation_rejects_bad_arguments_without_a_gpu():
     assert L.csa2_append_quant(ctypes.byref(m2), p, p, p, None, None, p, 2, None) == 1
 
 
+def test_attention_and_prepared_scan_validation_without_a_gpu():
+    """Host-side checks of csa2_sparse_attn_decode, csa2_append_quant_ex and
+    csa2_index_full_prepared return their documented status codes before
+    anything touches a device."""
+    L = C.lib()
+    d = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 2, 128, 512, 128, 1)
+    w = C.SwaCacheDesc(16, 1.0, 2, 128, 512, 128)
+    p = ctypes.c_void_p(16)
+    attn = lambda main, swa, q, T_q, H, K, out: L.csa2_sparse_attn_decode(main, swa, q, p, T_q, H, p, K, 0.1, out,
+                                                                         None, 0, None)
+    assert attn(ctypes.byref(d), None, p, 1, 64, 512, p) == 1                      # no window cache
+    assert attn(ctypes.byref(d), ctypes.byref(w), ctypes.c_void_p(24), 1, 64, 512, p) == 1   # misaligned q
+    assert attn(ctypes.byref(d), ctypes.byref(w), p, 1, 64, 512, None) == 1        # no output
+    assert attn(ctypes.byref(d), ctypes.byref(w), p, 0, 64, 512, p) == 1           # T_q = 0
+    assert attn(ctypes.byref(d), ctypes.byref(w), p, 1, 65, 512, p) == 2           # H > 64
+    assert attn(ctypes.byref(d), ctypes.byref(w), p, 1, 64, 4096, p) == 2          # K > 2048
+    other = C.SwaCacheDesc(16, 1.0, 2, 128, 256, 128)                              # D disagrees
+    assert attn(ctypes.byref(d), ctypes.byref(other), p, 1, 64, 512, p) == 1
+    # query preparation without the main cache, bad H_I, too small a workspace
+    assert L.csa2_append_quant_ex(None, p, None, p, None, p, p, 0, p, p, 1, 64, p, 1 << 20, None) == 1
+    assert L.csa2_append_quant_ex(ctypes.byref(d), p, None, p, None, p, p, 0, p, p, 1, 80, p, 1 << 20, None) == 2
+    assert L.csa2_append_quant_ex(ctypes.byref(d), p, None, p, None, p, p, 0, p, p, 1, 64, p, 16, None) == 5
+    assert "workspace" in L.csa2_last_error().decode()
+    # the prepared scan needs the workspace the preparation filled
+    assert L.csa2_index_full_prepared(ctypes.byref(d), p, 1, p, 128, None, p, 16, None) == 5
+
+
 def test_workspace_sizes_are_pure_host_functions():
     assert C.csa2_topk_workspace_size(8, 100000, 512, 2048) > 0
     assert C.csa2_topk_workspace_size(8, 65536, 512, 2048) == 0   # single-launch cluster path
