@@ -83,6 +83,19 @@ def _check(status: int):
         raise Csa2Error(status, lib().csa2_last_error().decode())
 
 
+_cuda = None
+
+
+def _device_required() -> bool:
+    """Whether tensors must live on a CUDA device: wherever CUDA is available
+    (a host pointer handed to a kernel would fault the GPU).  Without CUDA the
+    call goes on to the library, which reports that there is no device."""
+    global _cuda
+    if _cuda is None:
+        _cuda = torch.cuda.is_available()
+    return _cuda
+
+
 def _ptr(t: torch.Tensor | None, dtype=None):
     if t is None:
         return None
@@ -90,6 +103,8 @@ def _ptr(t: torch.Tensor | None, dtype=None):
         raise TypeError(f"expected {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
+    if t.device.type != "cuda" and _device_required():
+        raise ValueError(f"tensors must be CUDA device tensors (got one on {t.device})")
     return t.data_ptr()
 
 
@@ -121,6 +136,8 @@ class MainCache:
 
     def desc(self) -> MainCacheDesc:
         if self._desc is None:
+            if self.codes.device.type != "cuda" and _device_required():
+                raise ValueError(f"the cache must live on a CUDA device (it is on {self.codes.device})")
             object.__setattr__(self, "_desc", MainCacheDesc(
                 self.codes.data_ptr(), self.scales.data_ptr(), self.ik.data_ptr(), self.ik_scale.data_ptr(),
                 self.n_entries.data_ptr(), self.pending_kv.data_ptr(), self.pending_gate.data_ptr(), self.B,
@@ -147,6 +164,8 @@ class SwaCache:
 
     def desc(self) -> SwaCacheDesc:
         if self._desc is None:
+            if self.rows.device.type != "cuda" and _device_required():
+                raise ValueError(f"the window cache must live on a CUDA device (it is on {self.rows.device})")
             object.__setattr__(self, "_desc", SwaCacheDesc(self.rows.data_ptr(), self.scale, self.B, self.W_cap,
                                                            self.D, self.window))
         return self._desc
