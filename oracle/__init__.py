@@ -56,6 +56,7 @@ _SIGS = {
     "orc_pool_pair": (None, [_P, _P, _P, _P, _I, _P]),
     "orc_quant_fp8_row": (None, [_P, _I, _P, _P]),
     "orc_quant_query": (None, [_P, _I, _P, _P]),
+    "orc_project_key": (None, [_P, _P, _P, _I, _I, _P]),
     "orc_index_key": (None, [_P, _P, _P, _I, _I, _P, _P]),
     "orc_append": (None, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
                           _P, _P, _P, _P, _I, _F, _P, _P, _I]),
@@ -173,6 +174,17 @@ def quant_query(q):
     s = np.zeros(1, np.float32)
     lib().orc_quant_query(_p(q), q.shape[-1], _p(codes), _p(s))
     return codes, s[0]
+
+
+def project_key(codes, scales, W):
+    """The binary32 indexer key k = W^T x^ of one entry, before FP8."""
+    codes = _c(codes, np.uint8)
+    scales = _c(scales, np.uint8)
+    W = _c(W, np.uint16)
+    D, dI = W.shape
+    k = np.zeros(dI, np.float32)
+    lib().orc_project_key(_p(codes), _p(scales), _p(W), D, dI, _p(k))
+    return k
 
 
 def index_key(codes, scales, W):

@@ -252,34 +252,31 @@ void orc_quant_query(const uint16_t *q, int dI, uint8_t *codes, float *scale)
 /* Indexer key projected from the main KV  [jaehun "2) CSA2": the indexer K  */
 /* is obtained by projecting the main KV instead of a separate compression   */
 /* path].  Reading: project the dequantised stored FP4 entry x^ with a bf16  */
-/* matrix W[D][dI]:  k_i = sum_c x^_c * W[c][i], in binary32 with a fixed    */
-/* order -- groups of 32 channels are each accumulated by fmaf in ascending  */
-/* channel order from +0, then the group sums are added pairwise level by    */
-/* level ((g0+g1)+(g2+g3))+..., an odd last element passing up unchanged.    */
-/* Then the FP8 rule (s_k = amax/448, E4M3 codes).                           */
+/* matrix W[D][dI]:  k_i = sum_c x^_c * W[c][i], in binary32 as ONE fused    */
+/* multiply-add chain per output, channels in ascending order, starting from */
+/* +0:  acc = fmaf(x^_c, W[c][i], acc) for c = 0 .. D-1.  That is the plain  */
+/* left-to-right sum of the definition with each product fused into its      */
+/* addition; the pages give no other order.                                  */
 /* ------------------------------------------------------------------------ */
 
+void orc_project_key(const uint8_t *codes, const uint8_t *scales, const uint16_t *W,
+                     int D, int dI, float *k)
+{
+    float xh[4096];
+    for (int c = 0; c < D; ++c) xh[c] = (float)orc_fp4_value(codes, scales, c);
+    for (int i = 0; i < dI; ++i) {
+        float acc = 0.0f;
+        for (int c = 0; c < D; ++c) acc = fmaf(xh[c], orc_bf16_to_f32(W[(size_t)c * dI + i]), acc);
+        k[i] = acc;
+    }
+}
+
+/* The key's FP8 form: the rule above (s_k = amax/448, E4M3 codes of k/s_k). */
 void orc_index_key(const uint8_t *codes, const uint8_t *scales, const uint16_t *W,
                    int D, int dI, uint8_t *ik, float *ik_scale)
 {
-    float k[1024], part[64], xh[4096];
-    int G = D / 32;
-    for (int c = 0; c < D; ++c) xh[c] = (float)orc_fp4_value(codes, scales, c);
-    for (int i = 0; i < dI; ++i) {
-        for (int g = 0; g < G; ++g) {
-            float acc = 0.0f;
-            for (int c = 32 * g; c < 32 * g + 32; ++c)
-                acc = fmaf(xh[c], orc_bf16_to_f32(W[(size_t)c * dI + i]), acc);
-            part[g] = acc;
-        }
-        int n = G;
-        while (n > 1) {
-            int h = n / 2;
-            for (int j = 0; j < h; ++j) part[j] = part[2 * j] + part[2 * j + 1];
-            if (n & 1) { part[h] = part[n - 1]; n = h + 1; } else n = h;
-        }
-        k[i] = part[0];
-    }
+    float k[1024];
+    orc_project_key(codes, scales, W, D, dI, k);
     orc_quant_fp8_row(k, dI, ik, ik_scale);
 }
 

@@ -260,13 +260,120 @@ def test_index_key_within_error_bound_of_exact_sum():
     exact = [sum(Fraction(float(xh[c])) * Fraction(float(Wf[c, i])) for c in range(D)) for i in range(dI)]
     absum = [sum(abs(float(xh[c]) * float(Wf[c, i])) for c in range(D)) for i in range(dI)]
     amax = max(abs(float(e)) for e in exact)
-    # s = fl(amax_f32 / 448) where amax_f32 is within the summation error bound of amax
-    gamma = (32 + 4) * 2.0 ** -24
+    # one chain of D fused multiply-adds: |error| <= gamma_D * sum |x_c W_ci|
+    gamma = (D + 4) * 2.0 ** -24
     bound_amax = gamma * max(absum)
     assert abs(float(s) * 448 - amax) <= bound_amax + amax * 2 ** -23
     dec = np.array([oracle.e4m3_value(int(c)) for c in ik]) * float(s)
     for i in range(dI):
         assert abs(dec[i] - float(exact[i])) <= abs(float(exact[i])) * 2 ** -4 + float(s) * 2 ** -9 + gamma * absum[i] * 2
+
+
+# ---------------------------------------------------------------- the projection's order
+# The indexer key is one fused multiply-add chain per output, channels in
+# ascending order from +0 (the plain left-to-right sum of k_i = sum_c x^_c W_ci).
+# Every quantised key byte depends on that order, so it is pinned exactly.
+
+
+def _round_f32(v: Fraction) -> float:
+    """Exact rational -> nearest binary32, ties to even (IEEE 754 roundTiesToEven)."""
+    if v == 0:
+        return 0.0
+    sign = -1.0 if v < 0 else 1.0
+    a = abs(v)
+    e = a.numerator.bit_length() - a.denominator.bit_length()   # 2^e <= a < 2^(e+2)
+    if Fraction(2) ** e > a:
+        e -= 1
+    elif Fraction(2) ** (e + 1) <= a:
+        e += 1
+    e = max(e, -126)                           # subnormal quantum 2^-149
+    q = Fraction(2) ** (e - 23)                # spacing of binary32 in [2^e, 2^(e+1))
+    m = a / q
+    fl = m.numerator // m.denominator
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    r = sign * float(fl * q)
+    assert np.float32(r) == r
+    return r
+
+
+def _fmaf_exact(a: float, b: float, c: float) -> float:
+    return _round_f32(Fraction(a) * Fraction(b) + Fraction(c))
+
+
+def _ascending_chain(xh, Wf, i):
+    acc = 0.0
+    for c in range(len(xh)):
+        acc = _fmaf_exact(float(xh[c]), float(Wf[c, i]), acc)
+    return acc
+
+
+def _blocked_pairwise(xh, Wf, i):
+    """32-channel chains added pairwise: a plausible other order, used only to
+    show that the fixtures below tell the orders apart."""
+    parts = []
+    for g in range(len(xh) // 32):
+        acc = 0.0
+        for c in range(32 * g, 32 * g + 32):
+            acc = _fmaf_exact(float(xh[c]), float(Wf[c, i]), acc)
+        parts.append(acc)
+    while len(parts) > 1:
+        nxt = [_round_f32(Fraction(parts[j]) + Fraction(parts[j + 1])) for j in range(0, len(parts) - 1, 2)]
+        if len(parts) % 2:
+            nxt.append(parts[-1])
+        parts = nxt
+    return parts[0]
+
+
+def test_index_key_chain_order_hand_case():
+    """Worked by hand.  Column 0: product 2^24 at channel 0, then 31 products
+    of 1 at channels 32..62.  In one ascending chain every +1 meets an
+    accumulator of 2^24, where binary32 has spacing 2: 2^24 + 1 is a tie and
+    goes to the even 2^24, so k_0 = 2^24 exactly.  (Summing channels 32..63
+    on their own first would give 31 and k_0 = 2^24 + 32.)  Column 1 starts
+    from -2^24: -2^24 + j is exact for j < 2^24, so k_1 = -2^24 + 31."""
+    D, dI = 64, 2
+    codes = np.zeros(D // 2, np.uint8)
+    scales = np.zeros(D // 16, np.uint8)
+    scales[0] = 0x78            # E4M3 2^8
+    codes[0] = 0x6              # channel 0: E2M1 code 6 = 4.0 -> x^ = 1024
+    scales[2] = scales[3] = 0x38    # E4M3 1.0
+    for c in range(32, 63):     # channels 32..62: E2M1 code 2 = 1.0
+        codes[c // 2] |= 0x2 << (4 * (c & 1))
+    xh = oracle.fp4_dequant_row(codes, scales, D)
+    assert xh[0] == 1024 and xh[32:63].tolist() == [1.0] * 31 and xh[63] == 0
+    Wf = np.zeros((D, dI), np.float32)
+    Wf[0, 0], Wf[0, 1] = 2.0 ** 14, -(2.0 ** 14)
+    Wf[32:63, :] = 1.0
+    W = oracle_bits(torch.tensor(Wf).to(torch.bfloat16))
+    k = oracle.project_key(codes, scales, W)
+    assert k[0] == np.float32(2 ** 24)
+    assert k[1] == np.float32(-(2 ** 24) + 31)
+    assert _blocked_pairwise(xh, Wf.astype(np.float64), 0) == 2 ** 24 + 32   # the other order differs
+    ik, s = oracle.index_key(codes, scales, W)
+    assert s == np.float32(2 ** 24) / np.float32(448)
+
+
+@pytest.mark.parametrize("seed,D,dI", [(11, 512, 16), (12, 256, 32), (13, 128, 32)])
+def test_index_key_matches_exact_rounding_of_each_fma(seed, D, dI):
+    """Random entries: every output equals the ascending chain evaluated with
+    exact rationals, each step rounded once to binary32; on the same data the
+    blocked pairwise order gives other bits for some outputs."""
+    rng = np.random.default_rng(seed)
+    x = torch.tensor(rng.standard_normal(D), dtype=torch.float32).to(torch.bfloat16).float().numpy()
+    codes, scales = _entry(x)
+    xh = oracle.fp4_dequant_row(codes, scales, D)
+    Wt = torch.tensor(rng.standard_normal((D, dI)) / math.sqrt(D), dtype=torch.float32).to(torch.bfloat16)
+    Wf = Wt.double().numpy()
+    k = oracle.project_key(codes, scales, oracle_bits(Wt))
+    ref = [_ascending_chain(xh, Wf, i) for i in range(dI)]
+    assert [float(v) for v in k] == ref
+    other = [_blocked_pairwise(xh, Wf, i) for i in range(dI)]
+    assert other != ref
+    ik, s = oracle.index_key(codes, scales, oracle_bits(Wt))
+    codes_ref, s_ref = oracle.quant_fp8_row(np.array(ref, np.float32))
+    assert s == s_ref and np.array_equal(ik, codes_ref)
 
 
 def test_quant_query_follows_fp8_rule():
