@@ -96,6 +96,19 @@ def _device_required() -> bool:
     return _cuda
 
 
+def _check_device(device, what: str):
+    """Where CUDA is available, `device` must be the current CUDA device: the
+    kernels run there, and a pointer into another GPU's memory would be read
+    across the link (or fault without peer access)."""
+    if not _device_required():
+        return
+    if device.type != "cuda":
+        raise ValueError(f"{what} must be CUDA device tensors (got one on {device})")
+    cur = torch.cuda.current_device()
+    if device.index is not None and device.index != cur:
+        raise ValueError(f"{what} must be on the current device cuda:{cur} (got one on {device})")
+
+
 def _ptr(t: torch.Tensor | None, dtype=None):
     if t is None:
         return None
@@ -103,8 +116,7 @@ def _ptr(t: torch.Tensor | None, dtype=None):
         raise TypeError(f"expected {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
-    if t.device.type != "cuda" and _device_required():
-        raise ValueError(f"tensors must be CUDA device tensors (got one on {t.device})")
+    _check_device(t.device, "tensors")
     return t.data_ptr()
 
 
@@ -135,9 +147,8 @@ class MainCache:
         object.__setattr__(self, "_desc", None)
 
     def desc(self) -> MainCacheDesc:
+        _check_device(self.codes.device, "the cache's planes")
         if self._desc is None:
-            if self.codes.device.type != "cuda" and _device_required():
-                raise ValueError(f"the cache must live on a CUDA device (it is on {self.codes.device})")
             object.__setattr__(self, "_desc", MainCacheDesc(
                 self.codes.data_ptr(), self.scales.data_ptr(), self.ik.data_ptr(), self.ik_scale.data_ptr(),
                 self.n_entries.data_ptr(), self.pending_kv.data_ptr(), self.pending_gate.data_ptr(), self.B,
@@ -163,9 +174,8 @@ class SwaCache:
         object.__setattr__(self, "_desc", None)
 
     def desc(self) -> SwaCacheDesc:
+        _check_device(self.rows.device, "the window cache's rows")
         if self._desc is None:
-            if self.rows.device.type != "cuda" and _device_required():
-                raise ValueError(f"the window cache must live on a CUDA device (it is on {self.rows.device})")
             object.__setattr__(self, "_desc", SwaCacheDesc(self.rows.data_ptr(), self.scale, self.B, self.W_cap,
                                                            self.D, self.window))
         return self._desc
@@ -267,9 +277,12 @@ def csa2_attn_workspace_size(B: int, T_q: int, H: int, D: int, K: int, window: i
 
 def csa2_sparse_attn_decode(main: MainCache, swa: SwaCache, q, q_pos, idx, softmax_scale: float, out, ws=None,
                             stream=None):
+    """idx None (or with a last dimension of 0): window-only attention (K = 0)."""
     T_q = q_pos.shape[-1]
     H = q.shape[-2]
-    K = idx.shape[-1]
+    K = 0 if idx is None else idx.shape[-1]
+    if K == 0:
+        idx = None
     _check(lib().csa2_sparse_attn_decode(ctypes.byref(main.desc()), ctypes.byref(swa.desc()),
                                          _ptr(q, torch.bfloat16), _ptr(q_pos, torch.int32), T_q, H,
                                          _ptr(idx, torch.int32), K, float(softmax_scale),

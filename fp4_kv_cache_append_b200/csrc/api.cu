@@ -388,11 +388,13 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   if (!swa) return fail(CSA2_ERR_INVALID_ARG, "window cache is NULL");
   if ((st = check_swa(swa)) != CSA2_OK) return st;
   if (swa->B != main->B || swa->D != main->D) return fail(CSA2_ERR_INVALID_ARG, "window and main cache disagree");
-  if (!q || !q_pos || !idx || !out || !aligned16(q) || !aligned16(q_pos) || !aligned16(idx) || !aligned16(out))
-    return fail(CSA2_ERR_INVALID_ARG, "q/q_pos/idx/out must be 16-byte aligned device pointers");
+  if (!q || !q_pos || !out || !aligned16(q) || !aligned16(q_pos) || !aligned16(out))
+    return fail(CSA2_ERR_INVALID_ARG, "q/q_pos/out must be 16-byte aligned device pointers");
+  if (K < 0 || K > 2048) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "K=%d not in [0,2048]", K);
+  if (K > 0 && (!idx || !aligned16(idx)))
+    return fail(CSA2_ERR_INVALID_ARG, "idx must be a 16-byte aligned device pointer when K > 0");
   if (T_q <= 0 || (int64_t)main->B * T_q > 65535) return fail(CSA2_ERR_INVALID_ARG, "T_q=%d", T_q);
   if (H < 1 || H > 64) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "H=%d not in [1,64]", H);
-  if (K < 1 || K > 2048) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "K=%d not in [1,2048]", K);
   DeviceState *d;
   if ((st = device_state(&d)) != CSA2_OK) return st;
   AttnPlan p = plan_attn(main->B, T_q, H, main->D, K, swa->window, d->sms);
@@ -404,7 +406,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   AttnArgs a{};
   a.codes = main->codes; a.scales = main->scales; a.cap = main->cap; a.D = main->D;
   a.swa_rows = swa->rows; a.s_swa = swa->scale; a.W_cap = swa->W_cap; a.window = swa->window;
-  a.q = q; a.q_pos = q_pos; a.B = main->B; a.T_q = T_q; a.H = H; a.idx = idx; a.K = K;
+  a.q = q; a.q_pos = q_pos; a.B = main->B; a.T_q = T_q; a.H = H; a.idx = K > 0 ? idx : nullptr; a.K = K;
   a.scale = softmax_scale; a.out = out;
   a.ws = p.nsplit > 1 ? static_cast<float *>(ws) : nullptr;
   a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.csplit = p.csplit; a.status = d->status;

@@ -6,7 +6,8 @@
 //   projected from the main KV.  Section "3) FP4 main KV + SWA Bounded
 //   Replay": FP4 main KV, FP8 window KV.
 // One 512-thread block per group of up to 8 new entries (thread t < D/2 owns
-// channels 2t, 2t+1 and writes code byte t; all threads share the projection)
+// channels 2t, 2t+1 and writes code byte t; all threads share the projection:
+// one fused multiply-add chain per (entry, key output), channels ascending)
 // and one block per window row.  The quantised bytes are
 // decided in binary32 with IEEE division, no contraction (explicit _rn
 // intrinsics), so they are reproducible bit for bit.
@@ -53,22 +54,11 @@ __device__ __forceinline__ float pool_pair(float ka, float kb, float za, float z
   return __fadd_rn(__fmul_rn(wa, ka), __fmul_rn(wb, kb));
 }
 
-__device__ __forceinline__ float block_max(float v, float *red) {
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  v = lane < nw ? red[lane] : 0.0f;
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
-
 // Entries j0 .. j0+count-1 (count <= kEntriesPerBlock) of sequence b.  The
 // projection reads each W_ik element once for all of the block's entries.
 __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   const int t = threadIdx.x;
-  const int D = a.D, dI = a.dI, m = a.m, G = D / 32;
+  const int D = a.D, dI = a.dI, m = a.m;
   const int p0 = a.pos0[b];
   if (p0 < 0) {
     if (t == 0 && j0 == 0) flag(a.status, CSA2_DEV_BAD_POSITION);
@@ -80,9 +70,8 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   if (count > a.entries_per_block) count = a.entries_per_block;
 
   float *xh = sm;                                   // [E][D]
-  float *part = xh + a.entries_per_block * D;       // [E][G][dI]
-  float *red = part + a.entries_per_block * G * dI; // [32]
-  uint16_t *ws = reinterpret_cast<uint16_t *>(red + 32);  // W_ik [D][dI] bf16, 16-byte aligned
+  float *kbuf = xh + a.entries_per_block * D;       // [E][dI] binary32 keys
+  uint16_t *ws = reinterpret_cast<uint16_t *>(kbuf + a.entries_per_block * dI + 32);  // W_ik [D][dI] bf16, 16-byte aligned
   // stage W_ik in shared memory with 16-byte loads (issued before the
   // quantisation so their latency overlaps it)
   if (count > 0) {
@@ -147,60 +136,51 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   }
   if (count <= 0) return;
 
-  // ---- indexer key: k_i = sum_c x^_c W[c][i] in a fixed order (32-channel
-  // groups by fmaf in ascending channel order from +0, then pairwise sums)
-  if (count == 1) {   // decode: one entry, one chain per (group, output)
-    for (int p = t; p < G * dI; p += blockDim.x) {
-      const int i = p % dI, g = p / dI;
-      const uint16_t *wcol = ws + (32 * g) * dI + i;
-      const float *xg = xh + 32 * g;
-      float acc = 0.0f;
+  // ---- indexer key: k_i = sum_c x^_c W[c][i] as ONE fused multiply-add
+  // chain per output, channels in ascending order from +0.  Thread t owns
+  // output i = t % dI of entries t / dI, t / dI + slots, ... (slots = 512 /
+  // dI entries per pass); its chains share every W_ik element it reads.
+  {
+    constexpr int kChains = 2;   // 8 entries over 4 (dI = 128) or 8 (dI = 64) slots
+    const int slots = (int)blockDim.x / dI;
+    const int i = t % dI, s0 = t / dI;
+    float acc[kChains];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) acc = __fmaf_rn(xg[c], bf16_to_f32(wcol[c * dI]), acc);
-      part[g * dI + i] = acc;
-    }
-  } else {            // bulk: up to 8 entries share every W_ik read
-    constexpr int E = 8;
-    for (int p = t; p < G * dI; p += blockDim.x) {
-      const int i = p % dI, g = p / dI;
-      const uint16_t *wcol = ws + (32 * g) * dI + i;
-      float acc[E];
-#pragma unroll
-      for (int jj = 0; jj < E; ++jj) acc[jj] = 0.0f;
-#pragma unroll 4
-      for (int c = 0; c < 32; ++c) {
+    for (int k = 0; k < kChains; ++k) acc[k] = 0.0f;
+    if (s0 < count) {
+      const uint16_t *wcol = ws + i;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) {
         const float wv = bf16_to_f32(wcol[c * dI]);
 #pragma unroll
-        for (int jj = 0; jj < E; ++jj)
-          if (jj < count) acc[jj] = __fmaf_rn(xh[jj * D + 32 * g + c], wv, acc[jj]);
+        for (int k = 0; k < kChains; ++k) {
+          const int jj = s0 + k * slots;
+          if (jj < count) acc[k] = __fmaf_rn(xh[jj * D + c], wv, acc[k]);
+        }
       }
 #pragma unroll
-      for (int jj = 0; jj < E; ++jj)
-        if (jj < count) part[(jj * G + g) * dI + i] = acc[jj];
+      for (int k = 0; k < kChains; ++k) {
+        const int jj = s0 + k * slots;
+        if (jj < count) kbuf[jj * dI + i] = acc[k];
+      }
     }
   }
   __syncthreads();
-  for (int jj = 0; jj < count; ++jj) {
-    const int e = p0 / m + j0 + jj;
-    float k = 0.0f;
-    if (t < dI) {
-      int n = G;
-      float v[16];
-#pragma unroll
-      for (int g = 0; g < 16; ++g) v[g] = g < G ? part[(jj * G + g) * dI + t] : 0.0f;
-      while (n > 1) {
-        const int h = n >> 1;
-        for (int q = 0; q < h; ++q) v[q] = __fadd_rn(v[2 * q], v[2 * q + 1]);
-        if (n & 1) { v[h] = v[n - 1]; n = h + 1; } else n = h;
+  // ---- FP8 key per entry: warp jj takes entry jj (s_k = amax/448, E4M3 codes)
+  {
+    const int warp = t >> 5, lane = t & 31;
+    if (warp < count) {
+      const int jj = warp, e = p0 / m + j0 + jj;
+      float kmax = 0.0f;
+      for (int i = lane; i < dI; i += 32) kmax = fmaxf(kmax, fabsf(kbuf[jj * dI + i]));
+      for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+      const float sk = __fdiv_rn(kmax, 448.0f);
+      if (e < a.cap) {
+        const size_t row = (size_t)b * a.cap + e;
+        for (int i = lane; i < dI; i += 32)
+          a.ik[row * dI + i] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(kbuf[jj * dI + i], sk)));
+        if (lane == 0) a.ik_scale[row] = sk;
       }
-      k = v[0];
-    }
-    const float kmax = block_max(t < dI ? fabsf(k) : 0.0f, red);
-    const float sk = __fdiv_rn(kmax, 448.0f);
-    if (e < a.cap) {
-      const size_t row = (size_t)b * a.cap + e;
-      if (t < dI) a.ik[row * dI + t] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(k, sk)));
-      if (t == 0) a.ik_scale[row] = sk;
     }
   }
 }
@@ -263,12 +243,11 @@ constexpr int kDecCl = 8;
 __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_decode_kernel(const AppendArgs a) {
   __shared__ float xh[512];
   __shared__ alignas(16) uint16_t wsl[512 * 16];   // W_ik[:, c*OPB .. c*OPB+OPB), row-major [D][OPB]
-  __shared__ float part[16 * 16];                  // [G][OPB] chain partials
   __shared__ float kmx[kDecCl];                    // the blocks' local key maxima
   cg::cluster_group cl = cg::this_cluster();
   const int c = (int)cl.block_rank();
   const int b = blockIdx.y, t = threadIdx.x;
-  const int D = a.D, dI = a.dI, G = D / 32, OPB = dI / kDecCl;
+  const int D = a.D, dI = a.dI, OPB = dI / kDecCl;
   pdl_launch_dependents();
   pdl_wait();
   if (b >= a.B) {   // a cluster of query-preparation blocks (no cluster barrier)
@@ -340,31 +319,17 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
     reinterpret_cast<uint16_t *>(dst)[c * wch + t] = (uint16_t)(lo | (hi << 8));
   }
   __syncthreads();
-  // ---- indexer key: thread (o, g) forms the 32-channel fmaf chain of group g
-  // for output c*OPB + o (ascending channels from +0), as append_entries does
-  if (t < OPB * G) {
-    const int o = t % OPB, g = t / OPB;
-    const float *xg = xh + 32 * g;
-    const uint16_t *wcol = wsl + (32 * g) * OPB + o;
-    float acc = 0.0f;
-#pragma unroll
-    for (int cc = 0; cc < 32; ++cc) acc = __fmaf_rn(xg[cc], bf16_to_f32(wcol[cc * OPB]), acc);
-    part[g * OPB + o] = acc;
-  }
-  __syncthreads();
+  // ---- indexer key: thread o < OPB forms output c*OPB + o as one fused
+  // multiply-add chain over the channels in ascending order from +0, as
+  // append_entries does
   float k = 0.0f;
   if (t < 32) {
-    if (t < OPB) {   // group sums added pairwise, level by level
-      int n = G;
-      float v[16];
-#pragma unroll
-      for (int g = 0; g < 16; ++g) v[g] = g < G ? part[g * OPB + t] : 0.0f;
-      while (n > 1) {
-        const int h = n >> 1;
-        for (int q = 0; q < h; ++q) v[q] = __fadd_rn(v[2 * q], v[2 * q + 1]);
-        if (n & 1) { v[h] = v[n - 1]; n = h + 1; } else n = h;
-      }
-      k = v[0];
+    if (t < OPB) {
+      const uint16_t *wcol = wsl + t;
+      float acc = 0.0f;
+#pragma unroll 8
+      for (int cc = 0; cc < D; ++cc) acc = __fmaf_rn(xh[cc], bf16_to_f32(wcol[cc * OPB]), acc);
+      k = acc;
     }
     float m = t < OPB ? fabsf(k) : 0.0f;
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
@@ -392,8 +357,8 @@ cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {
   const int blocks = a.B * (a.main_blocks_per_seq + a.swa_blocks_per_seq) + 8 * a.prep.rows;
   if (blocks == 0) return cudaSuccess;
   const int threads = 512;   // quantisation uses the first D/2, the projection all of them
-  // [E][D] + [E][G][dI] floats, 32 floats, then W_ik [D][dI] bf16
-  const size_t smem = a.codes ? sizeof(float) * ((size_t)a.entries_per_block * (a.D + (a.D / 32) * a.dI) + 32) +
+  // [E][D] + [E][dI] floats, 32 floats, then W_ik [D][dI] bf16
+  const size_t smem = a.codes ? sizeof(float) * ((size_t)a.entries_per_block * (a.D + a.dI) + 32) +
                                     sizeof(uint16_t) * (size_t)a.D * a.dI
                               : 0;
   cudaError_t e = cudaFuncSetAttribute(append_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -22,7 +22,10 @@
 //    to start at zero: the first kernel writes every slot the second reads.
 //  - The first call on a device looks up the array's device address (host
 //    code only sees a host-side stand-in for the array's name).  Make that
-//    first call before any stream capture on that device.
+//    first call before any stream capture on that device.  The address is
+//    kept for the life of the process: after a cudaDeviceReset it would point
+//    into the destroyed context, so a process that resets a device must not
+//    call this entry point on it again.
 #include <cstdarg>
 #include <cstdio>
 #include <mutex>

@@ -24,6 +24,10 @@
  *    masked and a bit is set in the library's device status word, read with
  *    csa2_device_status().
  *  - Inputs with NaN or Inf are not supported (results unspecified, no trap).
+ *  - The library looks up, once per device, the device addresses of its own
+ *    global arrays (the status word; entry 6's scratch).  A process that
+ *    resets a device (cudaDeviceReset) must not call the library on that
+ *    device afterwards: those addresses belong to the context it destroyed.
  */
 #ifndef CSA2_H
 #define CSA2_H
@@ -218,12 +222,16 @@ CSA2_API size_t csa2_topk_workspace_size(int rows, int n_cols, int K, int P_out)
  *    window].  H query heads share one KV (K = V).
  *  q     [B][T_q][H][D] bf16
  *  q_pos [B][T_q] i32 token position t of each query
- *  idx   [B][T_q][K] i32 selected entries (-1 = none)
+ *  idx   [B][T_q][K] i32 selected entries (-1 = none); may be NULL when K = 0
+ *  K     selected entries per query; K = 0 attends to the window rows only,
+ *        the SWA-only layers of the encoder [jaehun "새로운 접근법" and its
+ *        flowchart: layers 1-2 use sliding-window attention only]
  *  out   [B][T_q][H][D] bf16: softmax over {idx != -1} U {window rows of
- *        tokens max(0,t-window+1)..t} of scale * q . x^, FP32 accumulation
+ *        tokens max(0,t-window+1)..t} of scale * q . x^, FP32 accumulation;
+ *        zeros when that set is empty
  *  ws, ws_bytes: workspace of csa2_attn_workspace_size(...); with a smaller
  *        workspace (or none) the kernel runs unsplit
- * Supported: D in {128, 256, 512}, 1 <= H <= 64, 1 <= K <= 2048, window <= 1024.
+ * Supported: D in {128, 256, 512}, 1 <= H <= 64, 0 <= K <= 2048, window <= 1024.
  */
 CSA2_API csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_cache *swa,
                                     const uint16_t *q, const int32_t *q_pos, int T_q, int H,

@@ -12,8 +12,10 @@ times (runner.Step: the same calls, grids, splits and cluster shapes).
   entries, Full and Reindex scores at sampled entries); the selections are
   checked by properties that hold at any size (the Top-K / pool of the
   scores the kernel was given, the column -> entry map, Reuse inheritance,
-  planted-key recall) and the attention by finiteness and the convex-hull
-  bound of its values.
+  planted-key recall), the Reindex selection of one sequence against the
+  oracle's scores of all pool columns, and every layer's attention of every
+  sequence against the oracle (it needs only the K selected entries and the
+  window rows, so it costs the same at any context length).
 No expected value comes from the CUDA path: the oracle's inputs are the
 seeded generators of fp4_kv_cache_append_b200.inputs.
 """
@@ -297,6 +299,58 @@ def _check_group(st, wl, seed, sample=256):
             np.testing.assert_array_equal(_np(st.swa[0][l].rows[b]), sw.rows[0])
         for l in st.layers:   # Reuse layers read the same indices; their outputs are sane
             _attn_sane(st.out[l][b, 0], gm, b)
+    _check_group_attention(st, wl, seed)
+    _check_reindex_selection(st, wl, seed, 0)
+
+
+def _oracle_window(wl, seed, l, b):
+    sw = oracle.SwaCache(1, runner.w_cap_for(wl), wl.D, window=wl.window)
+    rows = I.window_kv(wl, seed, l, b)
+    oracle.append(None, None, None, None, sw, I.bits(rows)[None], np.array([I.window_lo(wl)], np.int32),
+                  rows.shape[0])
+    return sw
+
+
+def _check_group_attention(st, wl, seed):
+    """The Reindex layer's and every Reuse layer's attention against the
+    oracle, for every sequence, with the step's own selection (the oracle
+    needs only the K selected entries and the layer's window rows)."""
+    t = wl.first_new
+    W = I.bits(I.w_ik(wl, seed))
+    idx = _np(st.idx)
+    layers = [l for k, l in st.plan if k != "full"]
+
+    def one(b):
+        sel = idx[b][idx[b] >= 0]
+        om = _entry_oracle(wl, seed, b, np.unique(sel), st._kv_ctx[b], W)
+        out = []
+        for l in layers:
+            q = I.queries(wl, seed, l, b, 1)[0]
+            out.append((l, oracle.attention(om, _oracle_window(wl, seed, l, b), 0, I.bits(q), idx[b], t, st.scale)))
+        return out
+
+    with _pool() as ex:
+        res = list(ex.map(one, range(wl.B)))
+    for b, per in enumerate(res):
+        for l, ref in per:
+            _check_attn(st.out[l][b, 0], ref)
+
+
+def _check_reindex_selection(st, wl, seed, b):
+    """The Reindex layer's Top-K of sequence b against the oracle's scores of
+    all P x 8 pool columns, equal up to the 1e-3 band around the K-th score."""
+    gm = st.main[0]
+    gpool = _np(st.group_pool) if wl.mode == "group" else _np(st.pool)
+    n_vis = oracle.n_visible(int(gm.n_entries[b]), wl.first_new, wl.m)
+    colmap = oracle.columns_to_entries(np.arange(wl.P * 8, dtype=np.int32), gpool[b])
+    ents = np.unique(colmap[(colmap >= 0) & (colmap < n_vis)]).astype(np.int32)
+    om = _entry_oracle(wl, seed, b, ents, st._kv_ctx[b], I.bits(I.w_ik(wl, seed)))
+    rl = [l for k, l in st.plan if k == "reindex"][0]
+    qi, w = I.index_queries(wl, seed, rl, b, 1)
+    col_scores = oracle.reindex_scores(om, 0, I.bits(qi[0]), w[0].numpy(), n_vis, gpool[b])
+    ref = oracle.columns_to_entries(oracle.topk(col_scores, wl.K), gpool[b])
+    by_entry = {int(e): float(v) for e, v in zip(colmap, col_scores) if e >= 0}
+    _band_equal(_np(st.idx)[b], ref, by_entry)
 
 
 def test_fullsize_dec_group():
@@ -333,4 +387,11 @@ def test_fullsize_long_context():
         _pool_property(scores[b, :n_vis], wl.P, pool2[b])
         planted = I.planted_positions(wl, 0, b).numpy()
         assert np.isin(planted, idx2[b]).mean() >= 0.9
+    # the Full layer's own attention (layer 0) over the Full selection
+    W = I.bits(I.w_ik(wl, 0))
+    for b in range(wl.B):
+        om = _entry_oracle(wl, 0, b, np.unique(idx2[b][idx2[b] >= 0]), st._kv_ctx[b], W)
+        ref = oracle.attention(om, _oracle_window(wl, 0, 0, b), 0, I.bits(I.queries(wl, 0, 0, b, 1)[0]), idx2[b],
+                               wl.first_new, st.scale)
+        _check_attn(st.out[0][b, 0], ref)
     _check_group(st, wl, 0)

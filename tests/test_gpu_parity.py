@@ -489,6 +489,34 @@ def test_attention_multi_tile_splits(B, T_q):
     assert C.csa2_device_status() == 0
 
 
+@pytest.mark.parametrize("D,H,B,T_q,window,W_cap,use_ws", [(512, 64, 2, 1, 128, 128, True),
+                                                           (512, 64, 8, 1, 128, 128, False),
+                                                           (256, 17, 3, 4, 128, 200, True),
+                                                           (128, 8, 1, 2, 64, 160, True)])
+def test_window_only_attention(D, H, B, T_q, window, W_cap, use_ws):
+    """K = 0: the SWA-only layers of the encoder (jaehun review, "새로운 접근법"
+    and its flowchart: layers 1-2 use sliding-window attention only) -- a
+    softmax over the window rows alone, no index array."""
+    n = 700
+    gm, gs, om, osw, _ = build_pair(B=B, cap=768, D=D, dI=64, m=1, T=n, pos0=[0] * B, seed=D + 7 * H, W_cap=W_cap,
+                                    s_swa=0.5, window=window)
+    g = gen(55)
+    q = torch.randn(B, T_q, H, D, generator=g).to(torch.bfloat16)
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[0, 0] = 40   # fewer rows than the window
+    out = torch.empty(B, T_q, H, D, dtype=torch.bfloat16, device="cuda")
+    ws = C.workspace(C.csa2_attn_workspace_size(B, T_q, H, D, 0, window)) if use_ws else None
+    scale = 1 / math.sqrt(D)
+    C.csa2_sparse_attn_decode(gm, gs, q.cuda(), torch.from_numpy(qpos).cuda(), None, scale, out, ws=ws)
+    torch.cuda.synchronize()
+    none = np.zeros(0, np.int32)
+    for b in range(B):
+        for j in range(T_q):
+            ref = oracle.attention(om, osw, b, bits(q[b, j]), none, int(qpos[b, j]), scale)
+            _check_attn(out[b, j], ref)
+    assert C.csa2_device_status() == 0
+
+
 def test_attention_out_of_range_index_is_masked_and_flagged():
     B, D, n, cap, K = 1, 128, 300, 384, 16
     gm, gs, om, osw, _ = build_pair(B=B, cap=cap, D=D, dI=64, m=1, T=n, pos0=[0], seed=41)
