@@ -3,24 +3,28 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (one GPU): the decoder decode step of a Full layer -- batch 8,
-context 65,536 tokens (m = 1), 64 query heads sharing one KV of dim 512
+Headline workload (one GPU): the decoder decode step of a Full layer -- batch
+8, context 65,536 tokens (m = 1), 64 query heads sharing one KV of dim 512
 (FP4 E2M1 + E4M3 per 16 channels), indexer 64 heads x 128 (FP8), Top-512 plus
 the 2048-block x 8 candidate pool, 128-token FP8 window.  A step is one token
 for all 8 sequences: append + quantise, Full indexer scan, Top-K + pool,
-sparse MQA attention (four C-ABI calls, six kernels).
+sparse MQA attention (four C-ABI calls, four kernels).
 
-Timing: W warm-up replays, then K steps as CUDA-graph replays (each graph is
-one rotation over 4 independent cache copies, 280 MB of indexer keys in all,
-more than the 126 MB L2, so no step finds its cache in L2), bracketed by a
-barrier and a device synchronisation, the maximum over ranks.  With N > 1
-(torchrun) every rank runs its own batch of 8 sequences: weak scaling, no
-data-path collective.  Prints one JSON line on rank 0.
+Timing: W warm-up replays, then repeats of exactly K steps (CUDA-graph
+replays rotating over 4 independent cache copies, 4 x 72 MB of step bytes,
+more than the 126 MB L2, so no step finds its cache in L2), each repeat
+bracketed by a barrier and a device synchronisation and timed with CUDA
+events; repeats continue until they span --min-ms (at least 5); the median
+repeat, maximum over ranks, is the headline.  With N > 1 (torchrun) every rank
+runs its own batch of 8 sequences: weak scaling, no data-path collective.
+On rank 0 of a one-GPU run the other configurations (dec_group, long,
+enc_prefill) are timed the same way and reported under "configs".  Prints
+one JSON line on rank 0.
 
 --impl reference times the CPU oracle (oracle/) on this machine's host cores
 on a bounded sample of the same workload: one sequence's append, Full scores
 over a slice of its entries, Top-K and pool over that slice and attention,
-extrapolated to the whole step (oracle_sample).
+extrapolated to the whole step (OracleSample).
 """
 from __future__ import annotations
 
@@ -47,17 +51,22 @@ FALLBACK_BF16_TFLOPS = 1590.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=24000)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--copies", type=int, default=4)
-    ap.add_argument("--graph-rotations", type=int, default=8, help="cache rotations captured per graph")
+    ap.add_argument("--min-ms", type=float, default=3000.0,
+                    help="timed repeats of K steps continue until they span this long (at least 5 repeats)")
+    ap.add_argument("--configs", default="dec_group,long,enc_prefill",
+                    help="other workloads to time on rank 0 of a one-GPU run (comma list, or 'none')")
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=20.0)
     ap.add_argument("--attn-sweep", action="store_true",
                     help="print only the gather + attention batch sweep (rank 0, one GPU) and exit")
-    return ap.parse_args()
+    a = ap.parse_args()
+    a.configs = [] if a.configs in ("", "none") else [c for c in a.configs.split(",") if c]
+    return a
 
 
 # --------------------------------------------------------------------------- helpers
@@ -81,10 +90,16 @@ def bf16_peak() -> float:
     return FALLBACK_BF16_TFLOPS
 
 
-INDEX_SOURCES = ("index.cu", "common.cuh", "kernels.h")   # what builds the index kernels
+KERNEL_SOURCES = {   # what builds each entry point's kernels
+    "index_full": ("index.cu", "common.cuh", "kernels.h"),
+    "index_reindex": ("index.cu", "common.cuh", "kernels.h"),
+    "attn": ("attn.cu", "common.cuh", "kernels.h"),
+    "topk": ("topk_cluster.cu", "topk.cu", "common.cuh", "kernels.h"),
+    "append": ("append.cu", "common.cuh", "kernels.h"),
+}
 
 
-def source_sha(names=INDEX_SOURCES) -> str:
+def source_sha(names) -> str:
     """Hash of the sources a kernel is built from (first 16 hex digits)."""
     import hashlib
     src = os.path.join(ROOT, "fp4_kv_cache_append_b200", "csrc")
@@ -95,13 +110,14 @@ def source_sha(names=INDEX_SOURCES) -> str:
     return h.hexdigest()[:16]
 
 
-def ncu_traffic(kernel_tag: str):
-    """Per-launch DRAM bytes of a kernel from a committed ncu summary, if the
-    summary was taken on the current kernel source (else None)."""
-    summ = os.path.join(ROOT, "profiles", f"{kernel_tag}.md")
-    if not os.path.exists(summ):
+def ncu_traffic(kernel: str):
+    """Per-launch DRAM bytes of an entry point's kernel from the committed ncu
+    summary profiles/<kernel>_dec_full.md, if that summary was taken on the
+    current kernel source (else None)."""
+    summ = os.path.join(ROOT, "profiles", f"{kernel}_{WORKLOAD}.md")
+    if not os.path.exists(summ) or kernel not in KERNEL_SOURCES:
         return None
-    want = source_sha()
+    want = source_sha(KERNEL_SOURCES[kernel])
     sha = traffic = None
     with open(summ) as f:
         for line in f:
@@ -194,6 +210,108 @@ def job_throughput(world: int, steps: int, ms: float) -> float:
     return world * steps / (ms / 1e3)
 
 
+# --------------------------------------------------------------------------- timing helpers
+
+
+def capture_steps(st, n_steps, copies, events=None):
+    """A CUDA graph of exactly n_steps steps; step i uses cache copy i % copies."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(n_steps):
+            st.run(copy=i % copies, events=events, external_events=events is not None)
+    return g
+
+
+class StepGraphs:
+    """Exactly K steps per replay(): K // G replays of a G-step graph and one
+    replay of a (K mod G)-step graph (G a multiple of the copy count, so the
+    cache rotation continues across graphs)."""
+
+    def __init__(self, st, K, copies, max_graph=256):
+        import torch
+        self.K = K
+        G = min(K, max(copies, max_graph // copies * copies))
+        self.n_full, rem = divmod(K, G)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            st.run(copy=0)   # one eager call on the capture stream (per-device set-up)
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        self.g = capture_steps(st, G, copies) if self.n_full else None
+        self.r = capture_steps(st, rem, copies) if rem else None
+
+    def replay(self):
+        for _ in range(self.n_full):
+            self.g.replay()
+        if self.r is not None:
+            self.r.replay()
+
+
+def timed_repeats(replay, min_total_ms, min_repeats, barrier):
+    """Times `replay` again and again, each repeat bracketed by a barrier and a
+    device synchronisation, with CUDA events on the current stream; returns
+    the per-repeat milliseconds (at least min_repeats, spanning min_total_ms)."""
+    import torch
+    out = []
+    total = 0.0
+    while len(out) < min_repeats or total < min_total_ms:
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        replay()
+        e1.record()
+        torch.cuda.synchronize()
+        barrier()
+        ms = e0.elapsed_time(e1)
+        out.append(ms)
+        total += ms
+        if len(out) > 100000:
+            break
+    return out
+
+
+def breakdown(st, copies, n_steps, replays=3):
+    """Per entry-point durations: the same steps with events around every call
+    (events cut the launch overlap of consecutive kernels, so the sum is above
+    the headline step time); mean over the last replay's calls."""
+    import torch
+    events = {}
+    g = capture_steps(st, n_steps, copies, events=events)
+    for _ in range(replays):
+        g.replay()
+    torch.cuda.synchronize()
+    us = {k: statistics.mean(s.elapsed_time(e) for s, e in v) * 1e3 for k, v in events.items()}
+    calls = {k: len(v) / n_steps for k, v in events.items()}
+    del g
+    return us, calls
+
+
+def kernel_rooflines(st, kern_us, calls, hbm, fp8_peak=None):
+    """Achieved GB/s (and TFLOP/s) of each entry point per call against the
+    roofline: algorithmic bytes per call / its event-timed duration."""
+    alg = st.algorithmic_bytes()
+    flops = st.algorithmic_flops()
+    out = {}
+    for k, us in kern_us.items():
+        n = calls.get(k, 1.0)
+        if k not in alg or us <= 0:
+            continue
+        b = alg[k] / n
+        gbs = b / (us * 1e-6) / 1e9
+        d = {"us_per_call": round(us, 3), "bytes_per_call": int(b), "gbs": round(gbs, 1),
+             "frac_hbm": round(gbs / hbm, 4)}
+        if k in flops:
+            f = flops[k] / n
+            d["tflops"] = round(f / (us * 1e-6) / 1e12, 2)
+            if k.startswith("index") and fp8_peak:
+                d["frac_fp8_derived"] = round(d["tflops"] / fp8_peak, 4)
+        out[k] = d
+    return out
+
+
 # --------------------------------------------------------------------------- our arm
 
 
@@ -207,43 +325,21 @@ def run_ours(args, rank, world, dist):
     C.lib()   # fails loudly without the CUDA library
     dev = torch.device("cuda", torch.cuda.current_device())
     wl = I.WORKLOADS[WORKLOAD]
-    st = runner.Step(wl, seed=rank_seed(rank), copies=args.copies)
+    copies = args.copies
+    st = runner.Step(wl, seed=rank_seed(rank), copies=copies)
     st.prefill()
 
     # eager warm-up: initialises per-device state and every kernel
-    for i in range(args.copies):
+    for i in range(copies):
         st.run(copy=i)
     torch.cuda.synchronize()
     assert C.csa2_device_status() == 0
 
-    # ---- graphs of `rot` rotations over the cache copies: the headline graph
-    # has nothing between the calls (consecutive kernels overlap their launch
-    # with the previous kernel's tail); the breakdown graph records events
-    # around every call for the per-kernel durations and the roofline.
-    rot = max(1, args.graph_rotations)
-    steps_per_graph = rot * args.copies
-    side = torch.cuda.Stream()
-    side.wait_stream(torch.cuda.current_stream())
-    with torch.cuda.stream(side):
-        st.run(copy=0)   # one more eager call on the capture stream
-    torch.cuda.current_stream().wait_stream(side)
-    torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g):
-        for r in range(rot):
-            for cp in range(args.copies):
-                st.run(copy=cp)
-    events = {}
-    g_ev = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g_ev):
-        for r in range(rot):
-            for cp in range(args.copies):
-                st.run(copy=cp, events=events, external_events=True)
-    n_graph = max(1, round(args.steps / steps_per_graph))
-    K = n_graph * steps_per_graph
-    for _ in range(max(3, args.warmup)):
-        g.replay()
-        g_ev.replay()
+    K = max(1, args.steps)
+    graphs = StepGraphs(st, K, copies)
+    W = max(3, args.warmup)
+    for _ in range(W):
+        graphs.replay()
     torch.cuda.synchronize()
 
     gpu_id = None
@@ -258,61 +354,36 @@ def run_ours(args, rank, world, dist):
         if dist is not None:
             dist.barrier()
 
-    # ---- timed region (headline)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- timed region (headline): exactly K steps per repeat; repeats until
+    # they span min_ms (and at least 5); the median repeat is reported
     sampler = ClockSampler(gpu_id) if rank == 0 else None
     if sampler:
         sampler.__enter__()
-    barrier()
-    torch.cuda.synchronize()
-    t0.record()
-    for _ in range(n_graph):
-        g.replay()
-    t1.record()
-    torch.cuda.synchronize()
-    barrier()
+    reps = timed_repeats(graphs.replay, args.min_ms, 5, barrier)
     if sampler:
         sampler.__exit__()
-    ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
+    med = statistics.median(reps)
+    ms = max_over_ranks(med, dist, dev)
     assert C.csa2_device_status() == 0, "device status flagged during the timed region"
 
-    # ---- timed region (breakdown): same steps with events around every call;
-    # per-entry-point durations are the event pairs of its last replay
-    n_ev = max(1, n_graph // 4)
-    barrier()
-    torch.cuda.synchronize()
-    t2, t3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t2.record()
-    for _ in range(n_ev):
-        g_ev.replay()
-    t3.record()
-    torch.cuda.synchronize()
-    barrier()
-    ms_ev = t2.elapsed_time(t3) / (n_ev * steps_per_graph)
-    kern_us = {k: statistics.mean(s.elapsed_time(e) for s, e in v) * 1e3 for k, v in events.items()}
-    calls_per_step = {k: len(v) / steps_per_graph for k, v in events.items()}
+    # ---- per-call durations (events around every call)
+    steps_ev = 8 * copies
+    kern_us, calls = breakdown(st, copies, steps_ev)
+    ms_ev = None
 
-    # ---- timed region (dominant kernel): the Full scan alone, back to back over
-    # the rotating cache copies (cold), its query prepared by the step's append
+    # ---- the Full scan alone, back to back over the rotating cache copies (cold)
+    rot = 8
     g_dom = torch.cuda.CUDAGraph()
     scan = lambda cp: C.csa2_index_full_prepared(st.main[cp], st.q_pos, st.scores, st.n_valid, ws=st.ws_index)
     with torch.cuda.graph(g_dom):
         for r in range(rot):
-            for cp in range(args.copies):
+            for cp in range(copies):
                 scan(cp)
     for _ in range(3):
         g_dom.replay()
-    n_dom = max(4, n_graph // 8)
-    barrier()
-    torch.cuda.synchronize()
-    t4, t5 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t4.record()
-    for _ in range(n_dom):
-        g_dom.replay()
-    t5.record()
-    torch.cuda.synchronize()
-    barrier()
-    dom_us = t4.elapsed_time(t5) * 1e3 / (n_dom * steps_per_graph)
+    dom_reps = timed_repeats(g_dom.replay, 200.0, 5, barrier)
+    scan_us = statistics.median(dom_reps) * 1e3 / (rot * copies)
+    del g_dom
     assert C.csa2_device_status() == 0
 
     # ---- end to end through the public API: pinned host inputs in, result out, every step
@@ -323,45 +394,144 @@ def run_ours(args, rank, world, dist):
     steps_per_s = job_throughput(world, K, ms)
     B, n = wl.B, wl.entries
     alg = st.algorithmic_bytes()
-    step_bytes = sum(alg.values()) + B * (wl.D + wl.D) * 2 + B * (wl.D // 2 + wl.D // 16 + wl.dI + 4)
-    idx_bytes = B * n * (wl.dI + 4)                        # 132 B per visible entry
+    step_bytes = sum(alg.values())
     hbm, hbm_kind = peaks()
-    # dominant kernel = the one that moves the step's bytes (the Full scan:
-    # 132 B per visible entry, ~96% of the step's algorithmic bytes)
-    dom = "index_full"
-    dom_bytes = idx_bytes
+    fp8 = 2.0 * bf16_peak()
+    kr = kernel_rooflines(st, kern_us, calls, hbm, fp8)
+    kr["index_full"]["alone_us"] = round(scan_us, 3)
+    # the roofline object names the kernel with the largest share of the step
+    # time; its achieved rate uses the duration measured inside the step
+    # (events), except the Full scan, which is also timed alone back to back
+    shares = {k: kern_us[k] * calls[k] for k in kern_us}
+    dom = max(shares, key=shares.get)
+    dom_bytes = alg[dom] / calls[dom]
+    dom_us = scan_us if dom == "index_full" else kern_us[dom]
     achieved = dom_bytes / (dom_us * 1e-6) / 1e9
-    traffic = ncu_traffic(f"index_full_{WORKLOAD}")
     launches_per_step = st.launches_per_step()
     clocks = sampler.summary() if sampler else None
     return {
         "metric": METRIC, "value": steps_per_s, "unit": "steps/s", "n_gpus": world, "steps": K,
-        "warmup": max(3, args.warmup), "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
+        "warmup": W, "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "e4m3/e2m1 storage, fp8+fp16 mma, f32 acc", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: {WORKLOAD_DESC}", "global_batch": B * world, "seq_len": wl.n,
-                   "parallelism": f"dp{world} (independent batches, no collective)",
-                   "l2": f"inputs larger than L2: {args.copies} rotating cache copies",
-                   "timing": f"CUDA-graph replays of {steps_per_graph} steps"},
+        "config": config_dict(world, copies),
+        "repeats": len(reps), "timed_ms_total": sum(reps),
+        "ms_per_step_spread": [min(reps) / K, max(reps) / K],
         "tokens_per_s": steps_per_s * B,
         "step_bytes": step_bytes, "step_gbs": step_bytes * steps_per_s / world / 1e9,
         "step_frac_hbm": step_bytes * steps_per_s / world / 1e9 / hbm,
         "kernels_us": {k: round(v, 3) for k, v in kern_us.items()},
-        "ms_per_step_with_events": ms_ev,
+        "kernel_rooflines": kr,
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": hbm,
-                     "peak_kind": hbm_kind, "unit": "GB/s", "frac": achieved / hbm if achieved else None,
-                     "traffic": traffic, "bytes_per_launch": dom_bytes, "launch_us": dom_us,
-                     "per_unit": "132 B per visible entry (128 B E4M3 key + 4 B scale)",
-                     "timing": "prepared Full scans back to back in a CUDA graph over 4 rotating cache copies"},
-        "clocks": clocks, "e2e": e2e, "gpu_launches": launches_per_step * K,
+                     "peak_kind": hbm_kind, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": ncu_traffic(dom), "bytes_per_launch": dom_bytes, "launch_us": dom_us,
+                     "share_of_step": shares[dom] / sum(shares.values()),
+                     "per_unit": PER_UNIT[dom],
+                     "timing": ("prepared Full scans back to back in a CUDA graph over the rotating cache copies"
+                                if dom == "index_full" else "CUDA events around each call inside the step graph")},
+        "clocks": clocks, "e2e": e2e, "launches_per_step": launches_per_step,
+        "gpu_launches": launches_per_step * K * len(reps),
     }
 
 
+PER_UNIT = {
+    "index_full": "132 B per visible entry and sequence (128 B E4M3 key + 4 B scale) + the query rows",
+    "attn": "344,064 B per query row and layer: 512 x 288 B gathered FP4 entries + 128 x 512 B window rows "
+            "+ 64 KB q + 64 KB out",
+    "topk": "4 B per scored column read + 4 B per selected index / pool block written",
+    "append": "the new entries' kv rows + FP4 codes/scales + indexer key + window rows + W_IK",
+    "index_reindex": "132 B per pool column (P x 8 per row)",
+}
+
+
+def config_dict(world, copies):
+    return {"workload": f"{WORKLOAD}: {WORKLOAD_DESC}", "global_batch": 8 * world, "seq_len": 65536,
+            "parallelism": f"dp{world} (independent batches, no collective)",
+            "l2": f"inputs larger than L2: {copies} rotating cache copies (~{copies * 72} MB of step bytes)",
+            "timing": "CUDA-graph replays of exactly `steps` steps per repeat; median repeat"}
+
+
+OTHER_CONFIGS = {
+    # name: (cache copies rotated so a step's bytes are not L2-resident, steps per timed repeat)
+    "dec_group": (3, 24),
+    "long": (1, 8),
+    "enc_prefill": (1, 1),
+}
+
+
+def run_other_configs(args, hbm, barrier):
+    """The BASELINE configs other than the headline's, each timed as one
+    median over repeats of whole steps (CUDA graphs), with a per-call
+    breakdown and the dominant call's roofline fraction."""
+    import gc
+
+    import torch
+
+    from fp4_kv_cache_append_b200 import csa2 as C
+    from fp4_kv_cache_append_b200 import inputs as I
+    from fp4_kv_cache_append_b200 import runner
+    out = {}
+    fp8 = 2.0 * bf16_peak()
+    for name in args.configs:
+        copies, n_steps = OTHER_CONFIGS[name]
+        wl = I.WORKLOADS[name]
+        t0 = time.perf_counter()
+        st = runner.Step(wl, seed=0, copies=copies)
+        st.prefill()
+        for i in range(copies):
+            st.run(copy=i)
+        torch.cuda.synchronize()
+        assert C.csa2_device_status() == 0
+        graphs = StepGraphs(st, n_steps, copies)
+        for _ in range(3):
+            graphs.replay()
+        reps = timed_repeats(graphs.replay, 300.0, 5, barrier)
+        ms = statistics.median(reps) / n_steps
+        kern_us, calls = breakdown(st, copies, n_steps, replays=2)
+        alg = st.algorithmic_bytes()
+        flops = st.algorithmic_flops()
+        kr = kernel_rooflines(st, kern_us, calls, hbm, fp8)
+        shares = {k: kern_us[k] * calls[k] for k in kern_us}
+        dom = max(shares, key=shares.get)
+        steps_s = 1e3 / ms
+        d = {"workload": WORKLOAD_DESCS[name], "ms_per_step": ms, "steps_per_s": steps_s,
+             "tokens_per_s": steps_s * wl.B * wl.T, "repeats": len(reps), "steps_per_repeat": n_steps,
+             "bytes_per_step": int(sum(alg.values())), "flops_per_step": int(sum(flops.values())),
+             "step_gbs": sum(alg.values()) / (ms * 1e-3) / 1e9,
+             "step_frac_hbm": sum(alg.values()) / (ms * 1e-3) / 1e9 / hbm,
+             "kernels_us": {k: round(v, 3) for k, v in kern_us.items()}, "calls_per_step": calls,
+             "kernel_rooflines": kr, "dominant": dom, "dominant_share": shares[dom] / sum(shares.values()),
+             "l2": f"{copies} rotating cache copies" if copies > 1 else "a step's bytes exceed L2",
+             "setup_s": round(time.perf_counter() - t0, 1)}
+        if name == "enc_prefill":
+            d["index_full_fp8"] = {"tflops": kr["index_full"]["tflops"], "peak_tflops": fp8,
+                                   "peak_kind": "derived: 2 x the measured dense bf16 burst (no FP8 peak is measured)",
+                                   "frac": kr["index_full"]["tflops"] / fp8}
+        assert C.csa2_device_status() == 0
+        out[name] = d
+        del graphs, st
+        gc.collect()
+        torch.cuda.empty_cache()
+    return out
+
+
+WORKLOAD_DESCS = {
+    "dec_group": "decoder group Reindex + 3 Reuse: batch 16, context 262,144, m=1, 64 heads, KV dim 512 FP4, "
+                 "Reindex over the 2048 x 8 pool of an (untimed) Full scan, Top-512, window 128",
+    "long": "long-context decode: batch 4, context 1,048,576, m=1, Full scan -> 2048 x 8 pool -> Reindex + 3 Reuse, "
+            "64 heads, KV dim 512, Top-512, window 128, 512 planted keys",
+    "enc_prefill": "encoder prefill chunk: 8,192 new tokens over a 131,072-token prefix, m=2 -> 65,536 + 4,096 "
+                   "entries, Full + 5 Reuse, causal, 64 heads, KV dim 512, Top-512, window 128",
+}
+
+
 SWEEP_ROWS = (8, 16, 32, 64, 128)
+SWEEP_WINDOW_ONLY_ROWS = (8, 128)   # K = 0: the SWA-only layers
 
 
 def attn_batch_sweep(hbm, bf16_peak):
     """Gather + attention alone (csa2_sparse_attn_decode, dec_full shapes:
-    64 heads, D 512, Top-512 + a 128-row window) at 8 ... 128 query rows.
+    64 heads, D 512, Top-512 + a 128-row window) at 8 ... 128 query rows, and
+    the window-only form (K = 0, the SWA-only layers) at 8 and 128 rows.
     Each launch is timed on its own with CUDA events, after a 256 MB write
     that evicts the previous launch's lines from L2 (cold gathers).  Caches
     hold 16,384 random entries per sequence (the kernel reads only the 512
@@ -378,13 +548,13 @@ def attn_batch_sweep(hbm, bf16_peak):
     from fp4_kv_cache_append_b200 import inputs as I
     wl = I.WORKLOADS[WORKLOAD]
     n = 16384
-    per_row_bytes = wl.K * (wl.D // 2 + wl.D // 16) + wl.window * wl.D + 2 * wl.H * wl.D * 2
-    per_row_flops = (wl.K + wl.window) * wl.H * wl.D * 4
+    row_bytes = lambda K: K * (wl.D // 2 + wl.D // 16) + wl.window * wl.D + 2 * wl.H * wl.D * 2
+    row_flops = lambda K: (K + wl.window) * wl.H * wl.D * 4
     g = torch.Generator(device="cuda")
     g.manual_seed(20261202)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     res = []
-    for rows in SWEEP_ROWS:
+    for rows, K in [(r, wl.K) for r in SWEEP_ROWS] + [(r, 0) for r in SWEEP_WINDOW_ONLY_ROWS]:
         main = C.MainCache(rows, n, wl.D, wl.dI, 1)
         main.codes.random_(0, 256, generator=g)
         main.scales.random_(0x28, 0x49, generator=g)
@@ -393,10 +563,12 @@ def attn_batch_sweep(hbm, bf16_peak):
         swa.rows.random_(0, 0x7F, generator=g)
         q = torch.randn(rows, 1, wl.H, wl.D, generator=g, device="cuda").to(torch.bfloat16)
         q_pos = torch.full((rows, 1), n - 1, dtype=torch.int32, device="cuda")
-        idx = torch.rand(rows, n, generator=g, device="cuda").argsort(dim=1)[:, :wl.K]
-        idx = idx.to(torch.int32).reshape(rows, 1, wl.K).contiguous()
+        idx = None
+        if K:
+            idx = torch.rand(rows, n, generator=g, device="cuda").argsort(dim=1)[:, :K]
+            idx = idx.to(torch.int32).reshape(rows, 1, K).contiguous()
         out = torch.empty(rows, 1, wl.H, wl.D, dtype=torch.bfloat16, device="cuda")
-        ws = C.workspace(C.csa2_attn_workspace_size(rows, 1, wl.H, wl.D, wl.K, wl.window))
+        ws = C.workspace(C.csa2_attn_workspace_size(rows, 1, wl.H, wl.D, K, wl.window))
         call = lambda: C.csa2_sparse_attn_decode(main, swa, q, q_pos, idx, 1.0 / math.sqrt(wl.D), out, ws=ws)
         call()
         torch.cuda.synchronize()
@@ -411,14 +583,14 @@ def attn_batch_sweep(hbm, bf16_peak):
         torch.cuda.synchronize()
         us = sorted(a.elapsed_time(b) * 1e3 for a, b in times[4:])
         us = us[len(us) // 2]
-        gbs = rows * per_row_bytes / us / 1e3
-        tflops = rows * per_row_flops / us / 1e6
-        res.append({"rows": rows, "us": round(us, 2), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+        gbs = rows * row_bytes(K) / us / 1e3
+        tflops = rows * row_flops(K) / us / 1e6
+        res.append({"rows": rows, "K": K, "us": round(us, 2), "gbs": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
                     "tflops": round(tflops, 1), "frac_bf16": round(tflops / bf16_peak, 4)})
         assert C.csa2_device_status() == 0
         del main, swa, q, idx, out, ws
-    return {"per_row_bytes": per_row_bytes, "per_row_flops": per_row_flops, "timing": "median of 20 cold launches",
-            "points": res}
+    return {"per_row_bytes": row_bytes(wl.K), "per_row_bytes_window_only": row_bytes(0),
+            "per_row_flops": row_flops(wl.K), "timing": "median of 20 cold launches", "points": res}
 
 
 def run_e2e(st, n_steps):
@@ -467,92 +639,120 @@ def run_e2e(st, n_steps):
 # --------------------------------------------------------------------------- oracle (CPU) legs
 
 
-def oracle_sample(seconds: float, steps: int | None = None, warmup: int = 0):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+class OracleSample:
     """The oracle on a bounded sample of the workload: sequence 0's step
     (append of its token, Full scores over a contiguous slice of E of its n
-    entries, Top-K and pool over that slice, attention over K + 128 keys), run
-    by `threads` threads at once.  Throughput is extrapolated linearly in the
-    scanned slice to n entries and to the 8 sequences of a step."""
-    import concurrent.futures as cf
+    entries, Top-K and pool over that slice, attention over K + 128 keys).
+    measure(threads, ...) runs `threads` such samples at once per round;
+    throughput is extrapolated linearly in the scanned slice to n entries and
+    to the 8 sequences of a step."""
 
-    import numpy as np
+    def __init__(self):
+        import concurrent.futures as cf
 
-    import oracle
-    from fp4_kv_cache_append_b200 import inputs as I
+        import numpy as np
 
-    wl = I.WORKLOADS[WORKLOAD]
-    threads = min(wl.B, len(os.sched_getaffinity(0)))
-    n = wl.entries
-    cap = n
-    om = oracle.MainCache(1, cap, wl.D, wl.dI, 1)
-    kv = I.bits(I.context_kv(wl, 0, 0))
-    W = I.bits(I.w_ik(wl, 0))
-    first = wl.first_new
-    # untimed: fill the oracle cache (threads over disjoint token ranges)
-    parts = np.array_split(np.arange(first), threads)
+        import oracle
+        from fp4_kv_cache_append_b200 import inputs as I
 
-    def fill(rg):
-        if rg.size == 0:
-            return
-        sub = oracle.MainCache(1, cap, wl.D, wl.dI, 1)
-        sub.codes, sub.scales, sub.ik, sub.ik_scale = om.codes, om.scales, om.ik, om.ik_scale
-        oracle.append(sub, kv[None, rg[0]:rg[-1] + 1], None, W, None, None, np.array([rg[0]], np.int32), rg.size)
+        wl = self.wl = I.WORKLOADS[WORKLOAD]
+        self.cores = len(os.sched_getaffinity(0))
+        fill_threads = min(wl.B, self.cores)
+        n = self.n = wl.entries
+        om = self.om = oracle.MainCache(1, n, wl.D, wl.dI, 1)
+        kv = I.bits(I.context_kv(wl, 0, 0))
+        W = I.bits(I.w_ik(wl, 0))
+        first = wl.first_new
+        # untimed: fill the oracle cache (threads over disjoint token ranges)
+        parts = np.array_split(np.arange(first), fill_threads)
 
-    with cf.ThreadPoolExecutor(threads) as ex:
-        list(ex.map(fill, parts))
-    om.n_entries[0] = first
-    osw = oracle.SwaCache(1, wl.window, wl.D, window=wl.window)
-    rows = I.bits(I.window_kv(wl, 0, 0, 0))
-    lo = I.window_lo(wl)
-    oracle.append(None, None, None, None, osw, rows[None, : first - lo], np.array([lo], np.int32), first - lo)
-    qi, w = I.index_queries(wl, 0, 0, 0)
-    q = I.bits(I.queries(wl, 0, 0, 0)[0])
-    qi = I.bits(qi[0])
-    w = w[0].numpy()
-    kv_new = kv[None, first:first + 1]
-    rows_new = rows[None, first - lo:]
+        def fill(rg):
+            if rg.size == 0:
+                return
+            sub = oracle.MainCache(1, n, wl.D, wl.dI, 1)
+            sub.codes, sub.scales, sub.ik, sub.ik_scale = om.codes, om.scales, om.ik, om.ik_scale
+            oracle.append(sub, kv[None, rg[0]:rg[-1] + 1], None, W, None, None, np.array([rg[0]], np.int32),
+                          rg.size)
 
-    def one(E):
-        oracle.append(om, kv_new, None, W, osw, rows_new, np.array([first], np.int32), 1)
-        sc = oracle.index_scores(om, 0, qi, w, E)
-        top = oracle.topk(sc, wl.K)
-        oracle.block_pool(sc, wl.P)
-        oracle.attention(om, osw, 0, q, top, first, 1.0 / wl.D ** 0.5)
+        with cf.ThreadPoolExecutor(fill_threads) as ex:
+            list(ex.map(fill, parts))
+        om.n_entries[0] = first
+        osw = oracle.SwaCache(1, wl.window, wl.D, window=wl.window)
+        rows = I.bits(I.window_kv(wl, 0, 0, 0))
+        lo = I.window_lo(wl)
+        oracle.append(None, None, None, None, osw, rows[None, : first - lo], np.array([lo], np.int32), first - lo)
+        qi, w = I.index_queries(wl, 0, 0, 0)
+        q = I.bits(I.queries(wl, 0, 0, 0)[0])
+        qi = I.bits(qi[0])
+        w = w[0].numpy()
+        kv_new = kv[None, first:first + 1]
+        rows_new = rows[None, first - lo:]
 
-    # calibrate the slice so that one round of `threads` samples takes the budget
-    t = time.perf_counter()
-    one(4096)
-    t_small = time.perf_counter() - t
-    per_entry = max(t_small / 4096, 1e-9)
-    n_rounds = max(1, steps or 1)
-    E = int(min(n, max(4096, seconds / n_rounds / per_entry)))
-    for _ in range(warmup):
+        def one(E):
+            oracle.append(om, kv_new, None, W, osw, rows_new, np.array([first], np.int32), 1)
+            sc = oracle.index_scores(om, 0, qi, w, E)
+            top = oracle.topk(sc, wl.K)
+            oracle.block_pool(sc, wl.P)
+            oracle.attention(om, osw, 0, q, top, first, 1.0 / wl.D ** 0.5)
+
+        self.one = one
+        t = time.perf_counter()
+        one(4096)
+        self.per_entry = max((time.perf_counter() - t) / 4096, 1e-9)
+
+    def measure(self, threads: int, seconds: float, rounds: int = 1, warmup: int = 0):
+        import concurrent.futures as cf
+        wl, n = self.wl, self.n
+        E = int(min(n, max(4096, seconds / rounds / self.per_entry)))
         with cf.ThreadPoolExecutor(threads) as ex:
-            list(ex.map(lambda _: one(E), range(threads)))
-    t = time.perf_counter()
-    for _ in range(n_rounds):
-        with cf.ThreadPoolExecutor(threads) as ex:
-            list(ex.map(lambda _: one(E), range(threads)))
-    dt = (time.perf_counter() - t) / n_rounds       # one round: `threads` sequence-samples
-    seq_step_s = dt * (n / E)                         # one sequence, full scan (linear in the slice)
-    step_s = seq_step_s * wl.B / threads              # 8 sequences on `threads` cores
-    sample = (f"sequence 0 of {wl.B}: append 1 token + oracle scores over {E} of {n} entries + Top-{wl.K} + "
-              f"pool + attention; {threads} concurrent copies per round, {n_rounds} round(s); "
-              f"scaled by {n}/{E} and {wl.B}/{threads}")
-    return {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle", "sample": sample}
+            for _ in range(warmup):
+                list(ex.map(lambda _: self.one(E), range(threads)))
+            t = time.perf_counter()
+            for _ in range(rounds):
+                list(ex.map(lambda _: self.one(E), range(threads)))
+            dt = (time.perf_counter() - t) / rounds     # one round: `threads` sequence-samples at once
+        seq_step_s = dt * (n / E)                         # one sequence, full scan (linear in the slice)
+        step_s = seq_step_s * wl.B / threads              # 8 sequences on `threads` cores
+        sample = (f"sequence 0 of {wl.B}: append 1 token + oracle scores over {E} of {n} entries + Top-{wl.K} + "
+                  f"pool + attention; {threads} concurrent copies per round, {rounds} round(s); "
+                  f"scaled by {n}/{E} and {wl.B}/{threads}")
+        return {"value": 1.0 / step_s, "unit": "steps/s", "cores": threads, "kind": "oracle", "sample": sample}
+
+
+def cpu_baseline(seconds: float):
+    """The oracle on all host cores (up to one per sequence), and single-threaded."""
+    o = OracleSample()
+    mt = o.measure(min(o.wl.B, o.cores), seconds)
+    one = o.measure(1, seconds / 2)
+    mt.update({"value_1t": one["value"], "sample_1t": one["sample"], "cpu_model": cpu_model(),
+               "host_cores": o.cores})
+    return mt
 
 
 def run_reference(args):
     t0 = time.perf_counter()
+    o = OracleSample()
     # a few rounds of bounded samples, about a minute of oracle work in all
-    cb = oracle_sample(seconds=60.0, steps=min(max(args.steps, 1), 4), warmup=min(args.warmup, 1))
+    threads = min(o.wl.B, o.cores)
+    cb = o.measure(threads, 60.0, rounds=min(max(args.steps, 1), 4), warmup=min(args.warmup, 1))
+    cb.update({"cpu_model": cpu_model(), "host_cores": o.cores})
     wall = time.perf_counter() - t0
     return {
         "impl": "reference", "metric": METRIC, "value": cb["value"], "unit": "steps/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / cb["value"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64 (int64 FP8 dots)", "data": "synthetic",
-        "config": {"workload": f"{WORKLOAD}: {WORKLOAD_DESC}", "global_batch": 8, "seq_len": 65536,
-                   "parallelism": "host cores (oracle)"},
+        "config": config_dict(args.gpus, args.copies),
         "cpu_baseline": cb, "e2e": {"value": cb["value"], "unit": "steps/s", "h2d_bytes_per_step": 0,
                                     "d2h_bytes_per_step": 0},
         "wall_s": wall,
@@ -590,8 +790,10 @@ def main():
         res = run_ours(args, rank, world, dist)
         if rank == 0:
             res["attn_batch_sweep"] = attn_batch_sweep(peaks()[0], bf16_peak())
+            if world == 1 and args.configs:
+                res["configs"] = run_other_configs(args, peaks()[0], lambda: None)
             if world == 1 and not args.no_cpu_baseline:
-                res["cpu_baseline"] = oracle_sample(seconds=args.cpu_seconds)
+                res["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
             print(json.dumps(res), flush=True)
     finally:
         if dist is not None:

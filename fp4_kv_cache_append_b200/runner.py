@@ -224,4 +224,28 @@ class Step:
                 out["index_reindex"] = out.get("index_reindex", 0) + self.rows * wl.P * 8 * ik
             att = self.rows * (wl.K * entry + wl.window * D + 2 * 2 * wl.H * D)
             out["attn"] = out.get("attn", 0) + att
+            # append: new kv rows (+ gate), the entries' FP4 bytes and keys, window rows in and out
+            new_entries = B * wl.T // wl.m if kind == "full" else 0
+            app = B * wl.T * D * 2 * (1 if kind != "full" else (2 if wl.m == 1 else 3)) + B * wl.T * D \
+                + new_entries * (entry + ik) + (D * wl.dI * 2 if kind == "full" else 0)
+            out["append"] = out.get("append", 0) + app
+            if kind in ("full", "reindex"):
+                cols = self.cap if kind == "full" else wl.P * 8
+                out["topk"] = out.get("topk", 0) + self.rows * (cols * 4 + wl.K * 4) \
+                    + (self.rows * wl.P * 4 if kind == "full" and wl.P else 0)
+        return out
+
+    def algorithmic_flops(self) -> dict:
+        """FLOPs of the contractions per step: FP8 indexer q.k over the visible
+        entries (or pool columns) x heads x d_I x 2; attention S and P.V over
+        K + window keys x heads x D x 4 per layer."""
+        wl = self.wl
+        out = {}
+        for kind, _ in self.plan:
+            if kind == "full":
+                vis = sum(min(wl.entries, (wl.first_new + j + 1) // wl.m) for j in range(self.T_q))
+                out["index_full"] = wl.B * vis * wl.H_I * wl.dI * 2
+            if kind == "reindex":
+                out["index_reindex"] = self.rows * wl.P * 8 * wl.H_I * wl.dI * 2
+            out["attn"] = out.get("attn", 0) + self.rows * (wl.K + wl.window) * wl.H * wl.D * 4
         return out
