@@ -60,6 +60,8 @@ _SIGS = {
     "orc_index_key": (None, [_P, _P, _P, _I, _I, _P, _P]),
     "orc_append": (None, [_I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _P,
                           _P, _P, _P, _P, _I, _F, _P, _P, _I]),
+    "orc_project_kv": (None, [_P, _I, _P, _I, _P]),
+    "orc_append_project": (None, [_I, _I, _I, _I, _P, _P, _P, _P, _P, _P, _I, _P, _P, _P, _I]),
     "orc_n_visible": (_I, [_I, _I, _I]),
     "orc_index_scores": (None, [_P, _P, _I, _I, _P, _P, _I, _P]),
     "orc_index_scores_at": (None, [_P, _P, _P, _I, _I, _P, _P, _I, _P]),
@@ -242,6 +244,27 @@ def append(main: MainCache | None, kv, gate, W, swa: SwaCache | None, kv_swa, po
         _p(kv), _p(gate), _p(W),
         _p(swa.rows) if swa else None, swa.W_cap if swa else 0,
         swa.scale if swa else 1.0, _p(kv_swa), _p(pos0), int(T))
+
+
+def project_kv(h, W):
+    """The decoder entry of one token: kv = h W_KV rounded once to binary32."""
+    h = _c(h, np.uint16)
+    W = _c(W, np.uint16)
+    d, D = W.shape
+    kv = np.zeros(D, np.float32)
+    lib().orc_project_kv(_p(h), d, _p(W), D, _p(kv))
+    return kv
+
+
+def append_project(main: MainCache, H, W_kv, W_ik, pos0, T):
+    """Project T tokens per sequence (H [B][T][d]) into an m = 1 main cache."""
+    H = _c(H, np.uint16)
+    W_kv = _c(W_kv, np.uint16)
+    W_ik = _c(W_ik, np.uint16)
+    pos0 = _c(pos0, np.int32)
+    d = W_kv.shape[0]
+    lib().orc_append_project(main.B, main.cap, main.D, main.dI, _p(main.codes), _p(main.scales), _p(main.ik),
+                             _p(main.ik_scale), _p(main.n_entries), _p(H), d, _p(W_kv), _p(W_ik), _p(pos0), int(T))
 
 
 def n_visible(n_entries: int, t: int, m: int) -> int:

@@ -347,6 +347,60 @@ void orc_append(int B, int cap, int D, int dI, int m,
 }
 
 /* ------------------------------------------------------------------------ */
+/* CED decoder-KV projection  [jaehun "1) CED": the decoder's global KV is   */
+/* obtained by projecting the final encoder hidden state H_{L/2} with each   */
+/* decoder layer's W_KV^l (the flowchart edge names W_KV^l and W_Z^l; the     */
+/* equation itself was lost)].  Reading: the plainest linear projection,     */
+/* kv_t = H_t W_KV, with no bias and no normalisation.  W_Z can only enter   */
+/* as the gate of an m >= 2 pooling; the decoder's caches are m = 1, where a */
+/* softmax over one token is 1, so the decoder entry is kv_t itself.         */
+/* Value: the exact sum of the bf16 products rounded once to binary32.  The  */
+/* products are exact in binary64; the sum is carried in binary64 with       */
+/* Neumaier's compensated summation (error ~2^-106 relative to the sum of    */
+/* magnitudes, far below binary32's rounding) and then rounded to binary32.  */
+/* H: [d] bf16 (one token), W: [d][D] bf16, kv: [D].                         */
+/* ------------------------------------------------------------------------ */
+
+void orc_project_kv(const uint16_t *H, int d, const uint16_t *W, int D, float *kv)
+{
+    for (int c = 0; c < D; ++c) {
+        double s = 0.0, comp = 0.0;
+        for (int i = 0; i < d; ++i) {
+            double x = (double)orc_bf16_to_f32(H[i]) * (double)orc_bf16_to_f32(W[(size_t)i * D + c]);
+            double t = s + x;
+            if (fabs(s) >= fabs(x)) comp += (s - t) + x;
+            else comp += (x - t) + s;
+            s = t;
+        }
+        kv[c] = (float)(s + comp);
+    }
+}
+
+/* Append T projected tokens per sequence to an m = 1 main cache: token p =  */
+/* pos0[b] + tau is entry p; kv = H W_KV (above), then the FP4 entry and its */
+/* indexer key exactly as orc_append does; n_entries[b] = pos0[b] + T.       */
+/* H: [B][T][d] bf16.                                                        */
+void orc_append_project(int B, int cap, int D, int dI,
+                        uint8_t *codes, uint8_t *scales, uint8_t *ik, float *ik_scale, int32_t *n_entries,
+                        const uint16_t *H, int d, const uint16_t *W_kv, const uint16_t *W_ik,
+                        const int32_t *pos0, int T)
+{
+    float *x = (float *)malloc(sizeof(float) * D);
+    for (int b = 0; b < B; ++b) {
+        for (int tau = 0; tau < T; ++tau) {
+            int e = pos0[b] + tau;
+            if (e < 0 || e >= cap) continue;
+            orc_project_kv(H + ((size_t)b * T + tau) * d, d, W_kv, D, x);
+            size_t r = (size_t)b * cap + e;
+            orc_quant_fp4_row(x, D, codes + r * (D / 2), scales + r * (D / 16));
+            orc_index_key(codes + r * (D / 2), scales + r * (D / 16), W_ik, D, dI, ik + r * dI, ik_scale + r);
+        }
+        n_entries[b] = pos0[b] + T;
+    }
+    free(x);
+}
+
+/* ------------------------------------------------------------------------ */
 /* Visibility: entry e is complete for a query at token t iff m*e+m-1 <= t.  */
 /* n_vis = min(n_entries, floor((t+1)/m)).                                   */
 /* ------------------------------------------------------------------------ */
