@@ -45,6 +45,7 @@ _PM, _PS = ctypes.POINTER(MainCacheDesc), ctypes.POINTER(SwaCacheDesc)
 SIGNATURES = {
     "csa2_append_quant": (_I, [_PM, _P, _P, _P, _PS, _P, _P, _I, _P]),
     "csa2_append_quant_ex": (_I, [_PM, _P, _P, _P, _PS, _P, _P, _I, _P, _P, _I, _I, _P, _SZ, _P]),
+    "csa2_append_project": (_I, [_PM, _P, _I, _P, _P, _P, _I, _P]),
     "csa2_index_full": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _P, _SZ, _P]),
     "csa2_index_full_prepared": (_I, [_PM, _P, _I, _P, _I64, _P, _P, _SZ, _P]),
     "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
@@ -203,6 +204,14 @@ def csa2_append_quant_ex(main: MainCache, kv, gate, w_ik, swa: SwaCache | None, 
                                       _ptr(w_ik, torch.bfloat16), sd, _ptr(kv_swa, torch.bfloat16),
                                       _ptr(pos0, torch.int32), int(T), _ptr(q_idx, torch.bfloat16),
                                       _ptr(w, torch.float32), T_q, H_I, _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def csa2_append_project(main: MainCache, h, w_kv, w_ik, pos0, stream=None):
+    """Projected append (CED producer): h [B][T][d_model] bf16, w_kv [d_model][D]."""
+    T, d_model = h.shape[-2], h.shape[-1]
+    _check(lib().csa2_append_project(ctypes.byref(main.desc()), _ptr(h, torch.bfloat16), int(d_model),
+                                     _ptr(w_kv, torch.bfloat16), _ptr(w_ik, torch.bfloat16), _ptr(pos0, torch.int32),
+                                     int(T), _stream(stream)))
 
 
 def csa2_index_full_prepared(main: MainCache, q_pos, scores, n_valid=None, ws=None, stream=None):

@@ -100,6 +100,23 @@ csa2_status encode_ik_map(const csa2_main_cache *m, CUtensorMap *map, int box_ro
   return CSA2_OK;
 }
 
+// 2D map over a row-major bf16 matrix [rows][cols] with boxes of box_rows x 64
+// elements (128 bytes) in the 128B swizzle.
+csa2_status encode_bf16_map(const void *base, int64_t rows, int64_t cols, int box_rows, CUtensorMap *map) {
+  EncodeTiled enc = nullptr;
+  csa2_status st = get_encoder(&enc);
+  if (st != CSA2_OK) return st;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(CSA2_ERR_INVALID_ARG, "cuTensorMapEncodeTiled (bf16) failed (%d)", (int)r);
+  return CSA2_OK;
+}
+
 csa2_status check_main(const csa2_main_cache *m, bool need_pending) {
   if (!m) return fail(CSA2_ERR_INVALID_ARG, "main cache is NULL");
   if (!m->codes || !m->scales || !m->ik || !m->ik_scale || !m->n_entries)
@@ -239,6 +256,42 @@ csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uint16_t *kv
   p.q8 = static_cast<uint8_t *>(ws);
   p.wq = reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + (((size_t)rows * 64 * main->d_I + 15) & ~size_t(15)));
   return append_impl(main, kv, gate, w_ik, swa, kv_swa, pos0, T, &p, stream);
+}
+
+csa2_status csa2_append_project(const csa2_main_cache *main, const uint16_t *h, int d_model, const uint16_t *w_kv,
+                                const uint16_t *w_ik, const int32_t *pos0, int T, csa2_stream_t stream) {
+  t_err.clear();
+  csa2_status st;
+  if ((st = check_main(main, false)) != CSA2_OK) return st;
+  if (main->m != 1) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "the projected append serves m = 1 caches (m=%d)", main->m);
+  if (main->D % 256) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "D=%d must be a multiple of 256", main->D);
+  if (d_model < 64 || d_model > 32768 || d_model % 64)
+    return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "d_model=%d must be a multiple of 64 in [64, 32768]", d_model);
+  if (T < 0) return fail(CSA2_ERR_INVALID_ARG, "T=%d", T);
+  if (!pos0 || !aligned16(pos0)) return fail(CSA2_ERR_INVALID_ARG, "pos0 must be a 16-byte aligned device pointer");
+  if (T == 0) return CSA2_OK;
+  if (!h || !w_kv || !w_ik || !aligned16(h) || !aligned16(w_kv) || !aligned16(w_ik))
+    return fail(CSA2_ERR_INVALID_ARG, "h, w_kv and w_ik must be 16-byte aligned device pointers");
+  if ((int64_t)main->B * T >= (int64_t)1 << 31) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "B*T must be < 2^31");
+  DeviceState *d;
+  if ((st = device_state(&d)) != CSA2_OK) return st;
+  CUtensorMap hm, wm;
+  if ((st = encode_bf16_map(h, (int64_t)main->B * T, d_model, 128, &hm)) != CSA2_OK) return st;
+  if ((st = encode_bf16_map(w_kv, d_model, main->D, 64, &wm)) != CSA2_OK) return st;
+  ProjectArgs p{};
+  p.codes = main->codes; p.scales = main->scales; p.n_entries = main->n_entries;
+  p.B = main->B; p.cap = main->cap; p.D = main->D; p.pos0 = pos0; p.T = T; p.d = d_model; p.status = d->status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_project(hm, wm, p, s);
+  if (e != cudaSuccess) return cuda_fail(e, "projection launch");
+  AppendArgs a{};
+  a.codes = main->codes; a.scales = main->scales; a.ik = main->ik; a.ik_scale = main->ik_scale;
+  a.n_entries = main->n_entries; a.B = main->B; a.cap = main->cap; a.D = main->D; a.dI = main->d_I; a.m = 1;
+  a.w_ik = w_ik; a.pos0 = pos0; a.T = T; a.status = d->status;
+  a.entries_per_block = 8;
+  a.main_blocks_per_seq = (T + 7) / 8;
+  e = launch_append_keys(a, s);
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "key projection launch");
 }
 
 // Blocks per row of a scan: about four resident blocks per SM in one wave,

@@ -54,6 +54,60 @@ __device__ __forceinline__ float pool_pair(float ka, float kb, float za, float z
   return __fadd_rn(__fmul_rn(wa, ka), __fmul_rn(wb, kb));
 }
 
+// Indexer keys of entries e0 .. e0+count-1 (count <= 8) of sequence b from
+// their dequantised values xh [count][D] (shared memory), with W_ik staged in
+// shared memory as ws [D][dI]: k_i = sum_c x^_c W[c][i] as ONE fused
+// multiply-add chain per output, channels in ascending order from +0; then
+// per entry s_k = amax/448 and E4M3 codes of k/s_k.  Thread t owns output
+// i = t % dI of entries t / dI, t / dI + slots, ... (slots = blockDim / dI);
+// its chains share every W_ik element it reads.  Ends with the block's
+// threads past one barrier; every thread of the block must call it.
+__device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const float *xh, float *kbuf,
+                           const uint16_t *ws) {
+  const int t = threadIdx.x, D = a.D, dI = a.dI;
+  {
+    constexpr int kChains = 2;   // 8 entries over 4 (dI = 128) or 8 (dI = 64) slots of 512 threads
+    const int slots = (int)blockDim.x / dI;
+    const int i = t % dI, s0 = t / dI;
+    float acc[kChains];
+#pragma unroll
+    for (int k = 0; k < kChains; ++k) acc[k] = 0.0f;
+    if (s0 < count) {
+      const uint16_t *wcol = ws + i;
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) {
+        const float wv = bf16_to_f32(wcol[c * dI]);
+#pragma unroll
+        for (int k = 0; k < kChains; ++k) {
+          const int jj = s0 + k * slots;
+          if (jj < count) acc[k] = __fmaf_rn(xh[jj * D + c], wv, acc[k]);
+        }
+      }
+#pragma unroll
+      for (int k = 0; k < kChains; ++k) {
+        const int jj = s0 + k * slots;
+        if (jj < count) kbuf[jj * dI + i] = acc[k];
+      }
+    }
+  }
+  __syncthreads();
+  // ---- FP8 key per entry: warp jj takes entry jj
+  const int warp = t >> 5, lane = t & 31;
+  if (warp < count) {
+    const int jj = warp, e = e0 + jj;
+    float kmax = 0.0f;
+    for (int i = lane; i < dI; i += 32) kmax = fmaxf(kmax, fabsf(kbuf[jj * dI + i]));
+    for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
+    const float sk = __fdiv_rn(kmax, 448.0f);
+    if (e < a.cap) {
+      const size_t row = (size_t)b * a.cap + e;
+      for (int i = lane; i < dI; i += 32)
+        a.ik[row * dI + i] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(kbuf[jj * dI + i], sk)));
+      if (lane == 0) a.ik_scale[row] = sk;
+    }
+  }
+}
+
 // Entries j0 .. j0+count-1 (count <= kEntriesPerBlock) of sequence b.  The
 // projection reads each W_ik element once for all of the block's entries.
 __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
@@ -136,53 +190,7 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   }
   if (count <= 0) return;
 
-  // ---- indexer key: k_i = sum_c x^_c W[c][i] as ONE fused multiply-add
-  // chain per output, channels in ascending order from +0.  Thread t owns
-  // output i = t % dI of entries t / dI, t / dI + slots, ... (slots = 512 /
-  // dI entries per pass); its chains share every W_ik element it reads.
-  {
-    constexpr int kChains = 2;   // 8 entries over 4 (dI = 128) or 8 (dI = 64) slots
-    const int slots = (int)blockDim.x / dI;
-    const int i = t % dI, s0 = t / dI;
-    float acc[kChains];
-#pragma unroll
-    for (int k = 0; k < kChains; ++k) acc[k] = 0.0f;
-    if (s0 < count) {
-      const uint16_t *wcol = ws + i;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        const float wv = bf16_to_f32(wcol[c * dI]);
-#pragma unroll
-        for (int k = 0; k < kChains; ++k) {
-          const int jj = s0 + k * slots;
-          if (jj < count) acc[k] = __fmaf_rn(xh[jj * D + c], wv, acc[k]);
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kChains; ++k) {
-        const int jj = s0 + k * slots;
-        if (jj < count) kbuf[jj * dI + i] = acc[k];
-      }
-    }
-  }
-  __syncthreads();
-  // ---- FP8 key per entry: warp jj takes entry jj (s_k = amax/448, E4M3 codes)
-  {
-    const int warp = t >> 5, lane = t & 31;
-    if (warp < count) {
-      const int jj = warp, e = p0 / m + j0 + jj;
-      float kmax = 0.0f;
-      for (int i = lane; i < dI; i += 32) kmax = fmaxf(kmax, fabsf(kbuf[jj * dI + i]));
-      for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
-      const float sk = __fdiv_rn(kmax, 448.0f);
-      if (e < a.cap) {
-        const size_t row = (size_t)b * a.cap + e;
-        for (int i = lane; i < dI; i += 32)
-          a.ik[row * dI + i] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(kbuf[jj * dI + i], sk)));
-        if (lane == 0) a.ik_scale[row] = sk;
-      }
-    }
-  }
+  entry_keys(a, b, p0 / m + j0, count, xh, kbuf, ws);
 }
 
 __device__ void append_window_row(const AppendArgs &a, int b, int r) {
@@ -348,6 +356,54 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
     }
   }
   if (c == 0 && t == 0) a.n_entries[b] = p0 + 1;
+}
+
+// Indexer keys of entries already stored as FP4 (the projected append writes
+// codes and scales first): one 512-thread block per group of up to 8 new
+// entries of a sequence; the entries are dequantised exactly (E2M1 x E4M3)
+// and projected by entry_keys, the same arithmetic as a token append.
+__global__ void __launch_bounds__(512) append_keys_kernel(const AppendArgs a) {
+  extern __shared__ float sm[];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int t = threadIdx.x, D = a.D, dI = a.dI;
+  const int b = blockIdx.x / a.main_blocks_per_seq;
+  const int j0 = (blockIdx.x % a.main_blocks_per_seq) * a.entries_per_block;
+  const int p0 = a.pos0[b];
+  if (p0 < 0) return;   // flagged by the projection kernel
+  int count = a.T - j0;
+  if (count > a.entries_per_block) count = a.entries_per_block;
+  if (count <= 0) return;
+  float *xh = sm;
+  float *kbuf = xh + a.entries_per_block * D;
+  uint16_t *ws = reinterpret_cast<uint16_t *>(kbuf + a.entries_per_block * dI + 32);
+  {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.w_ik);
+    uint4 *dst = reinterpret_cast<uint4 *>(ws);
+    for (int i = t; i < D * dI / 8; i += blockDim.x) dst[i] = src[i];
+  }
+  for (int i = t; i < count * D; i += blockDim.x) {
+    const int jj = i / D, c = i % D, e = p0 + j0 + jj;
+    float v = 0.0f;
+    if (e < a.cap) {
+      const size_t row = (size_t)b * a.cap + e;
+      const uint32_t code = (a.codes[row * (D / 2) + c / 2] >> ((c & 1) * 4)) & 0xFu;
+      v = __fmul_rn(e2m1_to_f32(code), e4m3_to_f32(a.scales[row * (D / 16) + c / 16]));
+    }
+    xh[jj * D + c] = v;
+  }
+  __syncthreads();
+  entry_keys(a, b, p0 + j0, count, xh, kbuf, ws);
+}
+
+cudaError_t launch_append_keys(const AppendArgs &a, cudaStream_t s) {
+  const int blocks = a.B * a.main_blocks_per_seq;
+  if (blocks == 0) return cudaSuccess;
+  const size_t smem = sizeof(float) * ((size_t)a.entries_per_block * (a.D + a.dI) + 32) +
+                      sizeof(uint16_t) * (size_t)a.D * a.dI;
+  cudaError_t e = cudaFuncSetAttribute(append_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(append_keys_kernel, dim3(blocks), dim3(512), smem, s, dim3(1, 1, 1), a);
 }
 
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s) {

@@ -43,6 +43,21 @@ struct AppendArgs {
   QueryPrep prep;          // optional: the following scan's query, 8 blocks per row
 };
 cudaError_t launch_append(const AppendArgs &a, cudaStream_t s);
+// Indexer keys of entries already stored as FP4 (after the projected append):
+// one block per group of entries_per_block new entries of a sequence.
+cudaError_t launch_append_keys(const AppendArgs &a, cudaStream_t s);
+
+// CED decoder-KV producer: codes/scales of kv = H W_KV (m = 1), token row
+// r = b * T + t -> entry pos0[b] + t.
+struct ProjectArgs {
+  uint8_t *codes, *scales;
+  int32_t *n_entries;
+  int B, cap, D;
+  const int32_t *pos0;
+  int T, d;              // tokens per sequence, d_model
+  unsigned int *status;
+};
+cudaError_t launch_project(const CUtensorMap &h_map, const CUtensorMap &w_map, const ProjectArgs &a, cudaStream_t s);
 
 struct IndexArgs {
   const float *ik_scale;

@@ -145,6 +145,31 @@ CSA2_API csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uin
                               int T_q, int H_I, void *ws, size_t ws_bytes, csa2_stream_t stream);
 
 /*
+ * 1c. Projected append: the CED decoder-KV producer  [jaehun "1) CED": the
+ *     decoder's global KV is the final encoder hidden state projected by each
+ *     decoder layer's W_KV^l (the flowchart edge "project W_KV^l, W_Z^l"; the
+ *     equation was lost, so this is the plain linear projection; W_Z can only
+ *     gate an m >= 2 pooling and the decoder caches are m = 1)].
+ *  main   m = 1 cache, D a multiple of 256
+ *  h      [B][T][d_model] bf16 hidden states of the new tokens
+ *  w_kv   [d_model][D] bf16 projection W_KV^l
+ *  w_ik   [D][d_I] bf16 indexer projection
+ *  pos0   [B] i32 DEVICE: position (= entry) of each sequence's first new token
+ * kv = h W_kv is accumulated in fp32 on the tensor cores and quantised in the
+ * same kernel to the FP4 entry (scale = E4M3(amax/6), codes = E2M1(x/scale));
+ * the indexer key of each new entry then follows from the stored bytes as in
+ * csa2_append_quant, and n_entries[b] becomes pos0[b] + T.  No window rows
+ * (a layer's window KV is appended with csa2_append_quant, main = NULL).
+ * The fp32 accumulation order is the tensor core's: an FP4 byte can differ
+ * from the correctly rounded projection's only where that value lies within
+ * the accumulation error of a rounding boundary of the quantiser.
+ * Supported: 64 <= d_model <= 32768, d_model a multiple of 64.
+ */
+CSA2_API csa2_status csa2_append_project(const csa2_main_cache *main, const uint16_t *h, int d_model,
+                                         const uint16_t *w_kv, const uint16_t *w_ik, const int32_t *pos0, int T,
+                                         csa2_stream_t stream);
+
+/*
  * 2. Full indexer scoring  [jaehun "2) CSA2": a Full layer scores all entries
  *    with its own indexer; score_j = sum_h w_h ReLU(q_h . k_j) as an FP8
  *    contraction].

@@ -20,7 +20,8 @@ def declared():
 
 def test_header_declares_the_five_entry_points():
     names = declared()
-    for n in ("csa2_append_quant", "csa2_index_full", "csa2_index_reindex", "csa2_topk", "csa2_sparse_attn_decode"):
+    for n in ("csa2_append_quant", "csa2_index_full", "csa2_index_reindex", "csa2_topk", "csa2_sparse_attn_decode",
+              "csa2_append_project"):
         assert n in names
 
 
@@ -151,6 +152,22 @@ def test_binding_marshals_every_entry_point_without_a_gpu():
     for call in calls:
         with pytest.raises(C.Csa2Error):
             call()
+
+
+def test_projected_append_host_validation():
+    """csa2_append_project: m = 1 caches only, d_model a multiple of 64,
+    aligned pointers; T = 0 enqueues nothing."""
+    L = C.lib()
+    p = ctypes.c_void_p(16)
+    m1 = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 2, 128, 512, 128, 1)
+    m2 = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 2, 128, 512, 128, 2)
+    d128 = C.MainCacheDesc(16, 16, 16, 16, 16, 16, 16, 2, 128, 128, 64, 1)
+    assert L.csa2_append_project(ctypes.byref(m2), p, 4096, p, p, p, 8, None) == 2      # m = 2
+    assert L.csa2_append_project(ctypes.byref(d128), p, 4096, p, p, p, 8, None) == 2    # D = 128
+    assert L.csa2_append_project(ctypes.byref(m1), p, 100, p, p, p, 8, None) == 2       # d_model % 64
+    assert L.csa2_append_project(ctypes.byref(m1), ctypes.c_void_p(24), 4096, p, p, p, 8, None) == 1
+    assert L.csa2_append_project(ctypes.byref(m1), p, 4096, p, p, None, 8, None) == 1   # pos0
+    assert L.csa2_append_project(ctypes.byref(m1), p, 4096, p, p, p, 0, None) == 0      # nothing to do
 
 
 def test_window_only_attention_host_validation():

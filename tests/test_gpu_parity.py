@@ -176,6 +176,85 @@ def _check_scores(got, ref):
     assert np.all(err <= SCORE_RTOL * np.abs(ref) + atol), f"max err {err.max()} (max ref {np.abs(ref).max()})"
 
 
+# ------------------------------------------------------------------ projected append (CED producer)
+
+
+def _robust_groups(kv_exact, eps, D):
+    """Per (row, 16-channel group): whether every value within +-eps of the
+    exact projection gives the same E4M3 scale and the same E2M1 codes (the
+    quantiser is monotone, so the interval's two ends decide)."""
+    rows = kv_exact.shape[0]
+    x = kv_exact.reshape(rows, D // 16, 16)
+    e = eps.reshape(rows, D // 16, 16)
+    a_lo = np.maximum(np.abs(x) - e, 0).max(axis=2)
+    a_hi = (np.abs(x) + e).max(axis=2)
+    s_lo = oracle.e4m3_encode((a_lo / 6).astype(np.float32))
+    s_hi = oracle.e4m3_encode((a_hi / 6).astype(np.float32))
+    robust = s_lo == s_hi
+    sv = np.vectorize(oracle.e4m3_value)(s_lo.astype(np.int64))
+    sv = np.where(sv == 0, 1.0, sv)
+    c_lo = oracle.e2m1_encode(((x - e) / sv[..., None]).astype(np.float32))
+    c_hi = oracle.e2m1_encode(((x + e) / sv[..., None]).astype(np.float32))
+    return robust & (c_lo == c_hi).all(axis=2)
+
+
+@pytest.mark.parametrize("B,T,d,D,dI,pos", [(2, 300, 1024, 512, 128, [0, 100]), (1, 129, 256, 256, 64, [7]),
+                                            (3, 8, 4096, 512, 128, [5, 0, 60])])
+def test_append_project_vs_oracle(B, T, d, D, dI, pos):
+    """kv = H W_KV in fp32 on the tensor cores, FP4-quantised in the epilogue,
+    against the oracle's correctly rounded projection: every 16-channel group
+    whose quantisation is decided the same way everywhere within the fp32
+    accumulation bound (d x 2^-22 x sum |h w|) is bit-exact; the rest (the
+    exact value within that bound of a rounding boundary) must be rare and
+    dequantise within one quantisation step.  Indexer keys follow from the
+    stored bytes bit-exactly."""
+    g = gen(d + D + T)
+    cap = 512
+    H = torch.randn(B, T, d, generator=g).to(torch.bfloat16)
+    Wkv = (torch.randn(d, D, generator=g) / math.sqrt(d)).to(torch.bfloat16)
+    Wik = (torch.randn(D, dI, generator=g) / math.sqrt(D)).to(torch.bfloat16)
+    pos0 = np.array(pos, np.int32)
+    gm = C.MainCache(B, cap, D, dI, 1)
+    C.csa2_append_project(gm, H.cuda(), Wkv.cuda(), Wik.cuda(), torch.from_numpy(pos0).cuda())
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    om = oracle.MainCache(B, cap, D, dI, 1)
+    oracle.append_project(om, bits(H), bits(Wkv), bits(Wik), pos0, T)
+    np.testing.assert_array_equal(gm.n_entries.cpu().numpy(), pos0 + T)
+    codes, scales = gm.codes.cpu().numpy(), gm.scales.cpu().numpy()
+    ik, iks = gm.ik.cpu().numpy(), gm.ik_scale.cpu().numpy()
+    Hd, Wd = H.double().numpy(), Wkv.double().numpy()
+    n_fragile = n_groups = 0
+    for b in range(B):
+        rows = slice(pos0[b], pos0[b] + T)
+        exact = Hd[b] @ Wd
+        eps = d * 2.0 ** -22 * (np.abs(Hd[b]) @ np.abs(Wd))
+        robust = _robust_groups(exact, eps, D)
+        gc, oc = codes[b, rows].reshape(T, D // 16, 8), om.codes[b, rows].reshape(T, D // 16, 8)
+        gs, os_ = scales[b, rows], om.scales[b, rows]
+        same = (gc == oc).all(axis=2) & (gs == os_)
+        assert same[robust].all(), "a robust group differs from the oracle"
+        n_fragile += int((~robust).sum())
+        n_groups += robust.size
+        # every group dequantises within one quantisation step (+ the bound) of the exact value
+        dq = np.stack([oracle.fp4_dequant_row(codes[b, e], scales[b, e], D) for e in range(pos0[b], pos0[b] + T)])
+        step = np.repeat(np.vectorize(oracle.e4m3_value)(gs.astype(np.int64)), 16, axis=1)
+        assert np.all(np.abs(dq - exact) <= step + eps)
+        # indexer keys: from the stored bytes, exactly as the oracle forms them
+        for t in range(T):
+            e = pos0[b] + t
+            if same[t].all():
+                ref_ik, ref_s = om.ik[b, e], om.ik_scale[b, e]
+            else:
+                ref_ik, ref_s = oracle.index_key(codes[b, e], scales[b, e], bits(Wik))
+            np.testing.assert_array_equal(ik[b, e], ref_ik)
+            assert iks[b, e].view(np.uint32) == np.float32(ref_s).view(np.uint32)
+    assert n_fragile <= 0.01 * n_groups, f"{n_fragile} of {n_groups} groups near a rounding boundary"
+    # entries outside the appended range are untouched
+    for b in range(B):
+        assert not codes[b, :pos0[b]].any() and not codes[b, pos0[b] + T:].any()
+
+
 @pytest.mark.parametrize("D,dI,H_I,n,T_q,m", [(128, 64, 4, 1000, 1, 1), (512, 128, 64, 2047, 3, 1),
                                               (256, 128, 17, 700, 2, 1), (512, 128, 64, 900, 4, 2)])
 def test_index_full_vs_oracle(D, dI, H_I, n, T_q, m):
