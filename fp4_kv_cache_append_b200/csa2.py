@@ -48,6 +48,8 @@ SIGNATURES = {
     "csa2_append_project": (_I, [_PM, _P, _I, _P, _P, _P, _I, _P]),
     "csa2_index_full": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _P, _SZ, _P]),
     "csa2_index_full_prepared": (_I, [_PM, _P, _I, _P, _I64, _P, _P, _SZ, _P]),
+    "csa2_index_topk": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _I, _P, _I, _P, _P, _SZ, _P]),
+    "csa2_index_topk_workspace_size": (_SZ, [_I, _I, _I]),
     "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "csa2_index_workspace_size": (_SZ, [_I, _I]),
     "csa2_topk": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P, _SZ, _P]),
@@ -245,6 +247,23 @@ def csa2_index_full(main: MainCache, q_idx, w, q_pos, scores, n_valid=None, ws=N
                                  _ptr(q_pos, torch.int32), T_q, H_I, _ptr(scores, torch.float32),
                                  scores.shape[-1], _ptr(n_valid, torch.int32), _ptr(ws), _nbytes(ws),
                                  _stream(stream)))
+
+
+def csa2_index_topk_workspace_size(rows: int, cap: int, d_I: int) -> int:
+    return int(lib().csa2_index_topk_workspace_size(rows, cap, d_I))
+
+
+def csa2_index_topk(main: MainCache, q_idx, w, q_pos, scores, K: int, out_idx, n_valid=None, P_out: int = 0,
+                    out_pool=None, ws=None, stream=None):
+    """Full scan fused with the first selection level, then Top-K and pool.
+    q_idx and w None: the query was prepared in ws by csa2_append_quant_ex."""
+    T_q = q_pos.shape[-1]
+    H_I = q_idx.shape[-2] if q_idx is not None else 64
+    ws = _ws_or_alloc(ws, csa2_index_topk_workspace_size(main.B * T_q, main.cap, main.d_I), scores.device)
+    _check(lib().csa2_index_topk(ctypes.byref(main.desc()), _ptr(q_idx, torch.bfloat16), _ptr(w, torch.float32),
+                                 _ptr(q_pos, torch.int32), T_q, H_I, _ptr(scores, torch.float32), scores.shape[-1],
+                                 _ptr(n_valid, torch.int32), int(K), _ptr(out_idx, torch.int32), int(P_out),
+                                 _ptr(out_pool, torch.int32), _ptr(ws), _nbytes(ws), _stream(stream)))
 
 
 def csa2_index_reindex(main: MainCache, q_idx, w, q_pos, pool_blocks, pool_scores, ws=None, stream=None):

@@ -337,7 +337,8 @@ size_t csa2_index_workspace_size(int rows, int d_I) {
 
 static csa2_status index_full_impl(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                                    const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
-                                   int32_t *n_valid, void *ws, size_t ws_bytes, bool prepared, csa2_stream_t stream) {
+                                   int32_t *n_valid, void *ws, size_t ws_bytes, bool prepared, csa2_stream_t stream,
+                                   float *bmax = nullptr, int64_t ld_b = 0) {
   IndexArgs a;
   CUtensorMap map;
   csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, scores, ws, ws_bytes, &a, &map, 128, prepared);
@@ -347,6 +348,7 @@ static csa2_status index_full_impl(const csa2_main_cache *main, const uint16_t *
   DeviceState *d;
   if ((st = device_state(&d)) != CSA2_OK) return st;
   a.ld = ld; a.n_valid = n_valid; a.status = d->status;
+  a.bmax = bmax; a.ld_b = ld_b;
   a.tiles_per_row = main->cap / 128;
   const int R = index_rows_per_block(T_q, false);
   if (R == 1) {
@@ -375,6 +377,55 @@ csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const int32_t 
   t_err.clear();
   return index_full_impl(main, nullptr, nullptr, q_pos, T_q, 64, scores, ld, n_valid, const_cast<void *>(ws),
                          ws_bytes, true, stream);
+}
+
+// Workspace of csa2_index_topk: the prepared query (as for csa2_index_full),
+// then the block maxima [rows][cap/8] f32, then n_valid [rows] i32.
+static size_t index_topk_offsets(int rows, int cap, int d_I, size_t *off_b, size_t *off_nv) {
+  const size_t q = (index_workspace_bytes(rows, d_I) + 15) & ~size_t(15);
+  const size_t b = ((size_t)rows * (cap / 8) * 4 + 15) & ~size_t(15);
+  *off_b = q;
+  *off_nv = q + b;
+  return q + b + (((size_t)rows * 4 + 15) & ~size_t(15));
+}
+
+size_t csa2_index_topk_workspace_size(int rows, int cap, int d_I) {
+  if (rows <= 0 || cap <= 0 || cap % 128 || (d_I != 64 && d_I != 128)) return 0;
+  size_t ob, onv;
+  return index_topk_offsets(rows, cap, d_I, &ob, &onv);
+}
+
+csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
+                            const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld, int32_t *n_valid,
+                            int K, int32_t *out_idx, int P_out, int32_t *out_pool, void *ws, size_t ws_bytes,
+                            csa2_stream_t stream) {
+  t_err.clear();
+  csa2_status st;
+  if ((st = check_main(main, false)) != CSA2_OK) return st;
+  const bool prepared = !q_idx && !w;
+  if (main->cap > kTopkBmaxMaxBlocks * 8)
+    return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "cap=%d above %d (use csa2_index_full + csa2_topk)", main->cap,
+                kTopkBmaxMaxBlocks * 8);
+  if (K < 1 || K > 2048) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "K=%d not in [1,2048]", K);
+  if (P_out < 0 || P_out > 4096) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "P_out=%d not in [0,4096]", P_out);
+  if (!out_idx || !aligned16(out_idx)) return fail(CSA2_ERR_INVALID_ARG, "out_idx must be a 16-byte aligned device pointer");
+  if (P_out > 0 && (!out_pool || !aligned16(out_pool))) return fail(CSA2_ERR_INVALID_ARG, "out_pool needed");
+  if (ld % 4) return fail(CSA2_ERR_INVALID_ARG, "ld=%lld must be a multiple of 4", (long long)ld);
+  if (T_q <= 0 || (int64_t)main->B * T_q > 65535) return fail(CSA2_ERR_INVALID_ARG, "T_q=%d", T_q);
+  const int rows = main->B * T_q;
+  size_t off_b, off_nv;
+  const size_t need = index_topk_offsets(rows, main->cap, main->d_I, &off_b, &off_nv);
+  if (!ws || ws_bytes < need || !aligned16(ws))
+    return fail(CSA2_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, ws_bytes);
+  uint8_t *wb = static_cast<uint8_t *>(ws);
+  float *bmax = reinterpret_cast<float *>(wb + off_b);
+  int32_t *nv = n_valid ? n_valid : reinterpret_cast<int32_t *>(wb + off_nv);
+  st = index_full_impl(main, q_idx, w, q_pos, T_q, prepared ? 64 : H_I, scores, ld, nv, ws, ws_bytes, prepared,
+                       stream, bmax, main->cap / 8);
+  if (st != CSA2_OK) return st;
+  TopkBmaxArgs t{scores, ld, bmax, main->cap / 8, rows, main->cap, nv, K, out_idx, P_out, out_pool};
+  cudaError_t e = launch_topk_bmax(t, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "topk_bmax launch");
 }
 
 csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,

@@ -5,24 +5,30 @@
 //   FP8 window KV.  All query heads share one KV (K = V).
 //
 // One block per (query row, key split); keys in tiles of 128 (the selected
-// entries first, then the window rows).  Per tile:
-//   1. every thread issues all of its gather loads at once (FP4 codes +
-//      scales, or E4M3 rows) and dequantises them exactly into fp16 with the
-//      hardware E2M1/E4M3 -> f16x2 converts (E2M1 x E4M3 products and E4M3
-//      values are exact in fp16), laid out in shared memory as a K-major
-//      128B-swizzled operand;
-//   2. S^T = K^ Q^T on tcgen05 (kind::f16, M = 128 keys, N = 64 heads,
-//      K = D): TMEM lane = key, column = head;
-//   3. all 8 warps (TMEM lane quarter x 32-head half) form the per-head
-//      maxima and sums over the 128 keys and write P (fp16) row by row as an
-//      MN-major operand [key][head];
-//   4. O^T += V^T P^T on tcgen05 (M = 128 channels per TMEM block, N = 64
-//      heads, K = 128 keys).  V^T is the same shared-memory tile as K^, read
-//      as an MN-major operand, so the tile is dequantised once.
-// The softmax reference max of a head moves only when a tile raises it by more
-// than 2^8 (then O^T and the running sum are rescaled in place), so P stays
-// within fp16 range and rescaling is rare.  Window rows keep their raw E4M3
-// values; the layer's window scale multiplies their logits and their P.
+// entries first, then the window rows).  Three warp roles run as a pipeline
+// over 64-channel chunks of a tile, handing work over through mbarriers:
+//   warps 0-7   gather + dequantise: thread (key slot r, half h) loads its
+//               key's 32-channel piece of every chunk (FP4 codes + their two
+//               E4M3 scales, or E4M3 window bytes), all loads of the tile in
+//               flight at once, and writes them exactly as fp16 (hardware
+//               E2M1/E4M3 -> f16x2 converts; E2M1 x E4M3 is exact in fp16)
+//               into the K-major 128B-swizzled K^ tile, chunk by chunk; a
+//               chunk is overwritten only after the previous tile's O^T MMAs
+//               that read it completed
+//   warp 12     tcgen05.mma issuer: S^T = K^ Q^T chunk by chunk as chunks
+//               land (M = 128 keys, N = 64 heads, K = 16, kind::f16), then,
+//               once P is written, O^T += V^T P^T per 128-channel block (V^T
+//               is the same K^ tile read MN-major) and the row sums
+//               L += 1 P^T with an all-ones A operand held in TMEM
+//   warps 8-11  softmax: thread = key (TMEM lane), 64 head logits; the
+//               reference max of a head moves only when a tile raises it by
+//               more than 2^8 (O^T and L are then rescaled in TMEM), so P =
+//               2^(s - m) stays within fp16 range; P is written as the MN-
+//               major B operand [key][head]
+// So the dequantisation of chunk k+1 overlaps the S MMAs of chunk k, and the
+// next tile's dequantisation overlaps this tile's O^T MMAs.  Window rows keep
+// their raw E4M3 values; the layer's window scale multiplies their logits and
+// their P.
 // The splits of one row form a thread-block cluster: each writes O / l per
 // head (fp16, [head][channel]) and its (max, sum) per head to the workspace, and
 // after one cluster barrier each split merges a slice of the channels from all
@@ -30,12 +36,9 @@
 // Launch shape (plan_attn): the split count minimises waves x (tiles per split
 // + merge cost) with one block per SM; at small batch each split is a pair of
 // blocks (grid z) that both compute S and P and each issue the O^T MMAs of,
-// write and merge half of the channels.  A block that runs several tiles has
-// L2 fetch the next tile's rows during the current tile's MMAs and skips the
-// per-head max reduction while the reference max holds.
-// Each block runs its code about once, from a cold instruction cache, so the
-// unrolled size of the straight-line parts (merge, maxima) is kept down:
-// fetching code costs as much as executing it here.
+// write and merge half of the channels.
+// Every wait is bounded: one that gives up flags the device status and stops
+// every role; issued MMAs are drained and TMEM freed before the block exits.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -43,16 +46,20 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kTile = 128;         // keys per tile (M of S^T)
-constexpr int kHeads = 64;         // heads padded to 64 (N)
+constexpr int kDqWarps = 8;                  // gather + dequantise
+constexpr int kSmWarp0 = 8;                  // softmax warps 8..11
+constexpr int kMmaWarp = 12;
+constexpr int kThreads = 13 * 32;
+constexpr int kDq = kDqWarps * 32;           // dequantise threads
+constexpr int kTile = 128;                   // keys per tile (M of S^T)
+constexpr int kHeads = 64;                   // heads padded to 64 (N)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLazy = 8.0f;      // log2 headroom before the reference max moves
+constexpr float kLazy = 8.0f;                // log2 headroom before the reference max moves
 constexpr uint32_t kWaitLimit = 1u << 22;
-// Merge items (head, 8 channels) per thread whose loads are in flight
-// together.  Each block runs the merge once, from a cold instruction cache,
-// so its unrolled size matters: 2 items keep one round of L2 reads for a
-// dec_full split (448 items) at 10 KB less code than 4.
+constexpr int kSmBar = 1;                    // named barrier of the softmax warps
+// TMEM columns: S^T [0, 64), O^T blocks [64, 64 + 64 MT), L [320, 384), ones [384, 416)
+constexpr uint32_t kColS = 0, kColO = 64, kColL = 320, kColOnes = 384, kTmemCols = 512;
+// Merge items (head, 8 channels) per thread whose loads are in flight together.
 constexpr int kMergeItems = 2;
 
 template <int D>
@@ -60,13 +67,13 @@ struct AttnSmem {
   alignas(1024) uint8_t kh[(D / 64) * kTile * 128];   // K^ tile: D/64 chunks of [128 keys x 128 B]
   alignas(1024) uint8_t q[(D / 64) * kHeads * 128];   // Q: D/64 chunks of [64 heads x 128 B]
   alignas(1024) uint8_t p[kTile * 128];               // P: [128 keys][64 heads] fp16, MN-major
-  int key_ent[2][kTile];                              // entry id or window slot, -1 = masked
+  float m_ref[kHeads], alpha[kHeads], lsum[kHeads];
   float red[4][kHeads];
-  float m_ref[kHeads], l_run[kHeads], alpha[kHeads];
   float wgt[8][kHeads];                               // merge weights of the splits
-  uint64_t sbar, obar;
+  uint64_t chunk_full[D / 64], o_done[D / 128], s_full, p_full, fin;
   uint32_t tmem_base;
-  int rescale;
+  int abort;
+  int rescale_at;                                     // tile whose softmax moved a reference max
 };
 
 // Byte offset of 16-byte piece `pc` (8 fp16 elements) of row `r` in a
@@ -116,7 +123,6 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
-
 // f32 (max, sum) per (row, split, head), after the fp16 partials.
 __device__ __forceinline__ float *partial_stats(const AttnArgs &a, size_t nrows) {
   return reinterpret_cast<float *>(reinterpret_cast<uint8_t *>(a.ws) + nrows * a.nsplit * (size_t)a.D * kHeads * 2);
@@ -130,55 +136,45 @@ __device__ __forceinline__ void prefetch_l2(const void *p) {
   asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-// Key ids of tile c (threads 0..127): entry ids of the selected entries, or
-// ring slots of the window rows; -1 = masked.  With `warm`, each thread also
-// asks L2 for its key's bytes (codes and scales, or the window row), so the
-// tile's gather, issued a few thousand cycles later, finds them there.
-template <int D>
-__device__ __forceinline__ void load_key_ids(const AttnArgs &a, int row, int b, int c, int n_fp4_tiles, int wlo,
-                                             int nwin, int *dst, int tid, bool warm) {
-  if (tid >= kTile) return;
-  int id = -1;
-  if (c < n_fp4_tiles) {
-    const int k = c * kTile + tid;
-    if (k < a.K) {
-      const int e = a.idx[(size_t)row * a.K + k];
-      if (e >= a.cap) flag(a.status, CSA2_DEV_INDEX_RANGE);
-      id = (e >= 0 && e < a.cap) ? e : -1;
-    }
-    if (warm && id >= 0) {
-      const size_t er = (size_t)b * a.cap + id;
-#pragma unroll
-      for (int o = 0; o < D / 2; o += 128) prefetch_l2(a.codes + er * (D / 2) + o);
-      prefetch_l2(a.scales + er * (D / 16));
-    }
-  } else {
-    const int j = (c - n_fp4_tiles) * kTile + tid;
-    id = j < nwin ? (wlo + j) % a.W_cap : -1;
-    if (warm && id >= 0) {
-#pragma unroll
-      for (int o = 0; o < D; o += 128) prefetch_l2(a.swa_rows + ((size_t)b * a.W_cap + id) * D + o);
-    }
+// Bounded wait that also gives up early once another role raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
+  for (uint32_t i = 0; i < kWaitLimit; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((i & 255u) == 255u && *abort) return false;
   }
-  dst[tid] = id;
+  *abort = 1;
+  return false;
+}
+
+// Key slot `slot` of tile c: the entry id of a selected entry or the ring slot
+// of a window row; -1 = masked.
+__device__ __forceinline__ int key_id(const AttnArgs &a, int row, int c, int n_fp4_tiles, int wlo, int nwin,
+                                      int slot) {
+  if (c < n_fp4_tiles) {
+    const int k = c * kTile + slot;
+    if (k >= a.K) return -1;
+    const int e = a.idx[(size_t)row * a.K + k];
+    return (e >= 0 && e < a.cap) ? e : -1;
+  }
+  const int j = (c - n_fp4_tiles) * kTile + slot;
+  return j < nwin ? (wlo + j) % a.W_cap : -1;
 }
 
 }  // namespace
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
+  constexpr int NCH = D / 64;                      // 64-channel chunks of a tile
   constexpr int MT = D / 128;                      // O^T TMEM blocks of 128 channels
-  constexpr int QI = kHeads * (D / 8) / kThreads;  // 16-byte pieces of Q per thread
-  constexpr int GF = D / 64;                       // FP4 items (32 channels) per thread and tile
-  constexpr int GW = D / 32;                       // window items (16 channels) per thread and tile
-  constexpr uint32_t kCols = D == 128 ? 128u : (D == 256 ? 256u : 512u);
+  constexpr int QI = kHeads * (D / 8) / kDq;       // 16-byte pieces of Q per dequantise thread
   constexpr uint32_t kIdS = mma_idesc(128, kHeads, 0u /*f16*/, 0u /*f16*/);
   constexpr uint32_t kIdO = kIdS | (1u << 15) | (1u << 16);   // A (V^T) and B (P^T) MN-major
+  constexpr uint32_t kIdL = kIdS | (1u << 16);                // A (ones, TMEM) K-major, B (P^T) MN-major
   extern __shared__ uint8_t smem_raw[];
   AttnSmem<D> &S = *reinterpret_cast<AttnSmem<D> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                                    ~uintptr_t(1023));
+  volatile int *abort = &S.abort;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int quarter = warp & 3, half = warp >> 2;   // TMEM lane quarter, 32-head half
   const int row = blockIdx.x;   // b * T_q + query
   const int split = blockIdx.y;
   const int b = row / a.T_q;
@@ -187,14 +183,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
 
   // ---- set-up that touches no global memory overlaps the previous kernel
   if (tid == 0) {
-    mbar_init(&S.sbar, 1);
-    mbar_init(&S.obar, 1);
-    S.rescale = 0;
+    for (int k = 0; k < NCH; ++k) mbar_init(&S.chunk_full[k], kDqWarps);
+    for (int m = 0; m < MT; ++m) mbar_init(&S.o_done[m], 1);
+    mbar_init(&S.s_full, 1);
+    mbar_init(&S.p_full, 4);
+    mbar_init(&S.fin, 1);
+    S.abort = 0;
+    S.rescale_at = -1;
     fence_barrier_init();
   }
-  if (warp == 4) {
-    tmem_alloc(&S.tmem_base, kCols);
+  if (tid < kHeads) { S.m_ref[tid] = -INFINITY; S.alpha[tid] = 1.f; }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&S.tmem_base, kTmemCols);
     tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = S.tmem_base;
+  if (warp >= kSmWarp0 && warp < kSmWarp0 + 4) {   // the all-ones A operand of the row-sum MMA
+    uint32_t ones[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) ones[j] = 0x3C003C00u;
+    tmem_st_x32(tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kColOnes, ones);
+    tmem_wait_st();
   }
   pdl_wait();
   const int t = a.q_pos[row];
@@ -208,65 +220,27 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   const int c_begin = split * a.chunks_per_split;
   int c_end = c_begin + a.chunks_per_split;
   if (c_end > total) c_end = total;
-
-  // ---- Q loads and the first tile's key ids are issued together
-  uint4 qraw[QI];
-  {
-    const uint16_t *qrow = a.q + (size_t)row * a.H * D;
-#pragma unroll
-    for (int u = 0; u < QI; ++u) {
-      const int i = tid + u * kThreads;
-      const int h = i / (D / 8), pc = i % (D / 8);
-      qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
-    }
-  }
-  if (c_begin < c_end) load_key_ids<D>(a, row, b, c_begin, n_fp4_tiles, wlo, nwin, S.key_ent[c_begin & 1], tid, false);
-  if (tid < kHeads) { S.m_ref[tid] = -INFINITY; S.l_run[tid] = 0.f; S.alpha[tid] = 1.f; }
+  const int n_tiles = c_end > c_begin ? c_end - c_begin : 0;
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();   // the ones are in TMEM before any MMA
   tc_fence_after();
-  const uint32_t tmem = S.tmem_base;
-  const uint32_t kh_base = smem_u32(S.kh), q_base = smem_u32(S.q), p_base = smem_u32(S.p);
 
-  bool aborted = false;
-  int n_done = 0;   // tiles whose O^T MMAs were issued
-#pragma unroll 1
-  for (int c = c_begin; c < c_end; ++c) {
-    const bool is_win = c >= n_fp4_tiles;
-    const int *ids = S.key_ent[c & 1];
-    // ---- 1a. gather loads, all issued before any is used: FP4 item = 32
-    // channels (16 code bytes + 2 scale bytes), window item = 16 E4M3 bytes
-    uint4 raw[GW];
-    uint32_t sc[GF];
-    if (!is_win) {
-#pragma unroll
-      for (int u = 0; u < GF; ++u) {
-        const int i = tid + u * kThreads;
-        const int r = i / (D / 32), g = i % (D / 32);
-        const int id = ids[r];
-        raw[u] = make_uint4(0, 0, 0, 0);
-        sc[u] = 0u;
-        if (id >= 0) {
-          const size_t er = (size_t)b * a.cap + id;
-          raw[u] = __ldg(reinterpret_cast<const uint4 *>(a.codes + er * (D / 2)) + g);
-          sc[u] = __ldg(reinterpret_cast<const uint16_t *>(a.scales + er * (D / 16)) + g);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < GW; ++u) {
-        const int i = tid + u * kThreads;
-        const int r = i / (D / 16), g = i % (D / 16);
-        const int id = ids[r];
-        raw[u] = id >= 0 ? __ldg(reinterpret_cast<const uint4 *>(a.swa_rows + ((size_t)b * a.W_cap + id) * D) + g)
-                         : make_uint4(0, 0, 0, 0);
-      }
-    }
-    // ---- Q: bf16 -> fp16 into the B-operand layout (first tile only)
-    if (c == c_begin) {
+  if (warp < kDqWarps) {
+    // ================================================ gather + dequantise
+    const int r = tid >> 1, hf = tid & 1;   // key slot, 32-channel half of each chunk
+    // Q: bf16 -> fp16 into the B-operand layout (before chunk 0 of the first tile)
+    if (n_tiles > 0) {
+      const uint16_t *qrow = a.q + (size_t)row * a.H * D;
+      uint4 qraw[QI];
 #pragma unroll
       for (int u = 0; u < QI; ++u) {
-        const int i = tid + u * kThreads;
+        const int i = tid + u * kDq;
+        const int h = i / (D / 8), pc = i % (D / 8);
+        qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < QI; ++u) {
+        const int i = tid + u * kDq;
         const int h = i / (D / 8), pc = i % (D / 8);
         const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
         uint32_t o[4];
@@ -278,223 +252,295 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
         *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
-    // the previous tile's O^T MMAs read K^ and P: wait before overwriting
-    bool ok = true;
-    if (n_done > 0) ok = mbar_wait_bounded(&S.obar, (n_done - 1) & 1, kWaitLimit);
-    if (__syncthreads_or(!ok)) { aborted = true; break; }
-
-    // ---- 1b. dequantise (hardware converts, exact) into the swizzled K^ tile
-    if (!is_win) {
-#pragma unroll
-      for (int u = 0; u < GF; ++u) {
-        const int i = tid + u * kThreads;
-        const int r = i / (D / 32), g = i % (D / 32);
-        const uint32_t s2 = e4m3x2_to_f16x2(sc[u]);   // scales of channels 32g.. and 32g+16..
-        const __half2 slo = __low2half2(*reinterpret_cast<const __half2 *>(&s2));
-        const __half2 shi = __high2half2(*reinterpret_cast<const __half2 *>(&s2));
-        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {   // 8 channels -> one 16-byte piece
-          uint32_t h[4];
-          e2m1x8_to_f16x2(w[k], h);
-          const __half2 sk = k < 2 ? slo : shi;
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h[e]), sk);
-            h[e] = *reinterpret_cast<const uint32_t *>(&v);
-          }
-          *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 4 * g + k, kTile)) = make_uint4(h[0], h[1], h[2], h[3]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int u = 0; u < GW; ++u) {
-        const int i = tid + u * kThreads;
-        const int r = i / (D / 16), g = i % (D / 16);
-        uint32_t h[8];
-        e4m3x4_to_f16x2(raw[u].x, h);
-        e4m3x4_to_f16x2(raw[u].y, h + 2);
-        e4m3x4_to_f16x2(raw[u].z, h + 4);
-        e4m3x4_to_f16x2(raw[u].w, h + 6);
-        *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 2 * g, kTile)) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 2 * g + 1, kTile)) = make_uint4(h[4], h[5], h[6], h[7]);
-      }
-    }
-    fence_proxy_async();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- 2. S^T = K^ Q^T
-    if (tid == 128) {
-      // descriptors advance by (byte offset >> 4) in their start-address field
-      tc_fence_after();
-      const uint64_t da = smem_desc_kmajor(kh_base, 128), db = smem_desc_kmajor(q_base, 128);
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (uint32_t)((ks & 3) * 32);
-        tc_mma_f16(tmem, da + (((ks >> 2) * (kTile * 128) + off) >> 4), db + (((ks >> 2) * (kHeads * 128) + off) >> 4),
-                   kIdS, ks > 0 ? 1u : 0u);
-      }
-      tc_commit(&S.sbar);
-    }
-    // the next tile's key ids (the other buffer) while the MMAs run
-    if (c + 1 < c_end) load_key_ids<D>(a, row, b, c + 1, n_fp4_tiles, wlo, nwin, S.key_ent[(c + 1) & 1], tid, true);
-    ok = mbar_wait_bounded(&S.sbar, (c - c_begin) & 1, kWaitLimit);
-    if (__syncthreads_or(!ok)) { aborted = true; break; }
-    tc_fence_after();
-
-    // ---- 3. softmax: warp (quarter, half) holds keys 32*quarter + lane,
-    // heads 32*half .. 32*half + 31
-    const float lsc = a.scale * (is_win ? a.s_swa : 1.0f) * kLog2e;
-    const float psc = is_win ? a.s_swa : 1.0f;
-    const bool first = (c == c_begin);
-    const int r = 32 * quarter + lane;
-    float sv[32];
-    const bool valid = ids[r] >= 0;
-    auto load_logits = [&]() {
-      uint32_t rv[32];
-      tmem_ld_x32(tmem + ((uint32_t)(32 * quarter) << 16) + 32 * half, rv);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) sv[j] = valid ? __uint_as_float(rv[j]) * lsc : -INFINITY;
-    };
-    load_logits();
-    // After the first tile the reference max usually holds: the per-head
-    // maxima are needed only when some logit exceeds it by more than 2^8.
-    bool need_max = first;
-    if (!first) {
-      const float4 *mp = reinterpret_cast<const float4 *>(&S.m_ref[32 * half]);
-      bool over = false;
-#pragma unroll
-      for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 m4 = mp[j4];
-        over |= (sv[4 * j4] > m4.x + kLazy) | (sv[4 * j4 + 1] > m4.y + kLazy) | (sv[4 * j4 + 2] > m4.z + kLazy) |
-                (sv[4 * j4 + 3] > m4.w + kLazy);
-      }
-      need_max = __syncthreads_or(over);
-    }
-    if (need_max) {
-      // per-head maxima of this warp's 32 keys (the butterfly consumes sv;
-      // the logits are read from TMEM again afterwards)
-      reduce_scatter32_max(sv, lane);
-      S.red[quarter][32 * half + lane] = sv[0];
-      __syncthreads();
-      load_logits();
-    }
-    if (need_max && tid < kHeads) {   // new reference max of head tid
-      const float m_old = S.m_ref[tid];
-      const float mt = fmaxf(fmaxf(S.red[0][tid], S.red[1][tid]), fmaxf(S.red[2][tid], S.red[3][tid]));
-      float al = 1.f;
-      if (mt != -INFINITY) {
-        if (m_old == -INFINITY) {
-          S.m_ref[tid] = mt;
-          al = 0.f;
-        } else if (mt > m_old + kLazy) {
-          S.m_ref[tid] = mt;
-          al = exp2f(m_old - mt);
-          if (!first) S.rescale = 1;
-        }
-      }
-      S.alpha[tid] = al;
-      S.l_run[tid] *= al;
-    }
-    if (need_max) __syncthreads();
-    // P = 2^(s - m_ref): row r of the P operand (fp16, window rows scaled)
-    {
-      const float4 *mp = reinterpret_cast<const float4 *>(&S.m_ref[32 * half]);
-      uint32_t ph[16];
-#pragma unroll
-      for (int j4 = 0; j4 < 8; ++j4) {
-        const float4 m4 = mp[j4];
-        const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int j = 4 * j4 + k;
-          sv[j] = (sv[j] == -INFINITY || mm[k] == -INFINITY) ? 0.f : ex2_approx(sv[j] - mm[k]);
-        }
-        const __half2 h0 = __floats2half2_rn(sv[4 * j4] * psc, sv[4 * j4 + 1] * psc);
-        const __half2 h1 = __floats2half2_rn(sv[4 * j4 + 2] * psc, sv[4 * j4 + 3] * psc);
-        ph[2 * j4] = *reinterpret_cast<const uint32_t *>(&h0);
-        ph[2 * j4 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-        *reinterpret_cast<uint4 *>(S.p + r * 128 + (((4 * half + i) ^ (r & 7)) << 4)) =
-            make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
-      reduce_scatter32(sv, lane);   // sv[0] = sum over this warp's keys of head 32*half + lane
-    }
-    S.red[quarter][32 * half + lane] = sv[0];   // the max readers finished before the last barrier
-    __syncthreads();
-    if (tid < kHeads) S.l_run[tid] += (S.red[0][tid] + S.red[1][tid]) + (S.red[2][tid] + S.red[3][tid]);
-    // rare: a head's reference max moved -> rescale its O^T column
-    if (S.rescale) {
+    int id = n_tiles > 0 ? key_id(a, row, c_begin, n_fp4_tiles, wlo, nwin, r) : -1;
 #pragma unroll 1
-      for (int mt = mt_lo; mt < mt_hi; ++mt) {
-        const uint32_t taddr = tmem + ((uint32_t)(32 * quarter) << 16) + kHeads + mt * kHeads + 32 * half;
-        uint32_t o[32];
-        tmem_ld_x32(taddr, o);
+    for (int it = 0; it < n_tiles; ++it) {
+      const int c = c_begin + it;
+      const bool is_win = c >= n_fp4_tiles;
+      // all of this tile's loads in flight at once: FP4 = 16 code bytes + 2
+      // scale bytes per chunk, window = 32 E4M3 bytes per chunk
+      uint4 raw[2 * NCH];
+      uint32_t sc[NCH];
+      if (!is_win) {
+        const size_t er = (size_t)b * a.cap + (id >= 0 ? id : 0);
+        const uint4 *cp = reinterpret_cast<const uint4 *>(a.codes + er * (D / 2)) + hf;
+        const uint16_t *sp = reinterpret_cast<const uint16_t *>(a.scales + er * (D / 16)) + hf;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          raw[k] = id >= 0 ? __ldg(cp + 2 * k) : make_uint4(0, 0, 0, 0);
+          sc[k] = id >= 0 ? (uint32_t)__ldg(sp + 2 * k) : 0u;
+        }
+      } else {
+        const uint4 *wp = reinterpret_cast<const uint4 *>(a.swa_rows + ((size_t)b * a.W_cap + (id >= 0 ? id : 0)) * D) + 2 * hf;
+#pragma unroll
+        for (int k = 0; k < NCH; ++k) {
+          raw[2 * k] = id >= 0 ? __ldg(wp + 4 * k) : make_uint4(0, 0, 0, 0);
+          raw[2 * k + 1] = id >= 0 ? __ldg(wp + 4 * k + 1) : make_uint4(0, 0, 0, 0);
+        }
+      }
+      // the next tile's key and an L2 prefetch of its bytes
+      int id_next = -1;
+      if (it + 1 < n_tiles) {
+        id_next = key_id(a, row, c + 1, n_fp4_tiles, wlo, nwin, r);
+        if (id_next >= 0) {
+          if (c + 1 < n_fp4_tiles) {
+            const size_t er = (size_t)b * a.cap + id_next;
+            prefetch_l2(a.codes + er * (D / 2) + hf * (D / 4));
+            if (hf == 0) prefetch_l2(a.scales + er * (D / 16));
+          } else {
+            prefetch_l2(a.swa_rows + ((size_t)b * a.W_cap + id_next) * D + hf * (D / 2));
+          }
+        }
+      }
+      bool ok = true;
+#pragma unroll
+      for (int k = 0; k < NCH; ++k) {
+        // chunks 2m, 2m+1 are read by the previous tile's O^T block m
+        if (it > 0 && (k & 1) == 0) {
+          int w_ok = 1;
+          if (lane == 0) w_ok = wait_or_abort(&S.o_done[k >> 1], (it - 1) & 1, abort);
+          if (!__shfl_sync(0xffffffffu, w_ok, 0)) { ok = false; break; }
+        }
+        uint32_t h[16];
+        if (!is_win) {
+          const uint32_t s2 = e4m3x2_to_f16x2(sc[k]);   // scales of the piece's two 16-channel groups
+          const __half2 slo = __low2half2(*reinterpret_cast<const __half2 *>(&s2));
+          const __half2 shi = __high2half2(*reinterpret_cast<const __half2 *>(&s2));
+          const uint32_t w[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            e2m1x8_to_f16x2(w[q4], h + 4 * q4);
+            const __half2 sk = q4 < 2 ? slo : shi;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __half2 v = __hmul2(*reinterpret_cast<const __half2 *>(&h[4 * q4 + e]), sk);
+              h[4 * q4 + e] = *reinterpret_cast<const uint32_t *>(&v);
+            }
+          }
+        } else {
+          e4m3x4_to_f16x2(raw[2 * k].x, h);
+          e4m3x4_to_f16x2(raw[2 * k].y, h + 2);
+          e4m3x4_to_f16x2(raw[2 * k].z, h + 4);
+          e4m3x4_to_f16x2(raw[2 * k].w, h + 6);
+          e4m3x4_to_f16x2(raw[2 * k + 1].x, h + 8);
+          e4m3x4_to_f16x2(raw[2 * k + 1].y, h + 10);
+          e4m3x4_to_f16x2(raw[2 * k + 1].z, h + 12);
+          e4m3x4_to_f16x2(raw[2 * k + 1].w, h + 14);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 8 * k + 4 * hf + j, kTile)) =
+              make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
+        fence_proxy_async();   // generic stores -> visible to the tensor core
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.chunk_full[k]);
+      }
+      if (!ok) break;
+      id = id_next;
+    }
+  } else if (warp < kSmWarp0 + 4) {
+    // ================================================ softmax
+    const int q = warp & 3;                 // TMEM lane quarter
+    const int r = 32 * q + lane;            // key slot = TMEM lane
+    const int st = tid - kSmWarp0 * 32;     // 0..127
+    const uint32_t srow = tmem + ((uint32_t)(32 * q) << 16);
+#pragma unroll 1
+    for (int it = 0; it < n_tiles; ++it) {
+      const int c = c_begin + it;
+      const bool is_win = c >= n_fp4_tiles;
+      int id = key_id(a, row, c, n_fp4_tiles, wlo, nwin, r);
+      if (c < n_fp4_tiles && c * kTile + r < a.K) {   // flag selected entries outside the cache
+        const int e = a.idx[(size_t)row * a.K + c * kTile + r];
+        if (e >= a.cap) flag(a.status, CSA2_DEV_INDEX_RANGE);
+      }
+      const bool valid = id >= 0;
+      int w_ok = 1;
+      if (lane == 0) w_ok = wait_or_abort(&S.s_full, it & 1, abort);
+      if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
+      tc_fence_after();
+      const float lsc = a.scale * (is_win ? a.s_swa : 1.0f) * kLog2e;
+      const float psc = is_win ? a.s_swa : 1.0f;
+      const bool first = it == 0;
+      float sv[64];
+      auto load_logits = [&]() {
+        uint32_t rv[64];
+        tmem_ld_x32(srow + kColS, rv);
+        tmem_ld_x32(srow + kColS + 32, rv + 32);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * S.alpha[32 * half + j]);
-        tmem_st_x32(taddr, o);
+        for (int j = 0; j < 64; ++j) sv[j] = valid ? __uint_as_float(rv[j]) * lsc : -INFINITY;
+      };
+      load_logits();
+      // after the first tile the reference max usually holds: the per-head
+      // maxima are needed only when a logit exceeds it by more than 2^8
+      bool over = first;
+      if (!first) {
+        const float4 *mp = reinterpret_cast<const float4 *>(S.m_ref);
+#pragma unroll
+        for (int j4 = 0; j4 < 16; ++j4) {
+          const float4 m4 = mp[j4];
+          over |= (sv[4 * j4] > m4.x + kLazy) | (sv[4 * j4 + 1] > m4.y + kLazy) | (sv[4 * j4 + 2] > m4.z + kLazy) |
+                  (sv[4 * j4 + 3] > m4.w + kLazy);
+        }
       }
-      tmem_wait_st();
+      const bool need_max = named_bar_or(kSmBar, 128, over);
+      if (need_max) {
+        reduce_scatter32_max(sv, lane);        // heads 0..31 (consumes sv[0..31])
+        S.red[q][lane] = sv[0];
+        reduce_scatter32_max(sv + 32, lane);   // heads 32..63
+        S.red[q][32 + lane] = sv[32];
+        named_bar(kSmBar, 128);
+        if (st < kHeads) {   // new reference max of head st
+          const float m_old = S.m_ref[st];
+          const float mt = fmaxf(fmaxf(S.red[0][st], S.red[1][st]), fmaxf(S.red[2][st], S.red[3][st]));
+          float al = 1.f;
+          if (mt != -INFINITY) {
+            if (m_old == -INFINITY) {
+              S.m_ref[st] = mt;
+              al = 0.f;
+            } else if (mt > m_old + kLazy) {
+              S.m_ref[st] = mt;
+              al = exp2f(m_old - mt);
+              if (!first) S.rescale_at = it;
+            }
+          }
+          S.alpha[st] = al;
+        }
+        named_bar(kSmBar, 128);
+        load_logits();
+      }
+      // P = 2^(s - m_ref): row r of the P operand (fp16, window rows scaled)
+      {
+        const float4 *mp = reinterpret_cast<const float4 *>(S.m_ref);
+        uint32_t ph[32];
+#pragma unroll
+        for (int j4 = 0; j4 < 16; ++j4) {
+          const float4 m4 = mp[j4];
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int j = 4 * j4 + k;
+            sv[j] = (sv[j] == -INFINITY || mm[k] == -INFINITY) ? 0.f : ex2_approx(sv[j] - mm[k]);
+          }
+          const __half2 h0 = __floats2half2_rn(sv[4 * j4] * psc, sv[4 * j4 + 1] * psc);
+          const __half2 h1 = __floats2half2_rn(sv[4 * j4 + 2] * psc, sv[4 * j4 + 3] * psc);
+          ph[2 * j4] = *reinterpret_cast<const uint32_t *>(&h0);
+          ph[2 * j4 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          *reinterpret_cast<uint4 *>(S.p + r * 128 + ((i ^ (r & 7)) << 4)) =
+              make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
+      }
+      // rare: a head's reference max moved -> rescale its O^T and L columns
+      // (the previous tile's O^T MMAs completed before S of this tile did)
+      if (need_max && S.rescale_at == it) {
+#pragma unroll 1
+        for (int blk = 0; blk <= MT; ++blk) {
+          if (blk < MT && (blk < mt_lo || blk >= mt_hi)) continue;
+          const uint32_t base = srow + (blk < MT ? kColO + 64 * blk : kColL);
+#pragma unroll 1
+          for (int hh = 0; hh < 2; ++hh) {
+            uint32_t o[32];
+            tmem_ld_x32(base + 32 * hh, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * S.alpha[32 * hh + j]);
+            tmem_st_x32(base + 32 * hh, o);
+          }
+        }
+        tmem_wait_st();
+      }
+      fence_proxy_async();   // P (generic stores) -> visible to the tensor core
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.p_full);
     }
-    fence_proxy_async();   // P (generic stores) -> visible to the tensor core
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) S.rescale = 0;
-
-    // ---- 4. O^T += V^T P^T
-    if (tid == 128) {
+  } else if (lane == 0) {
+    // ================================================ MMA issuer
+    const uint32_t kh_base = smem_u32(S.kh), q_base = smem_u32(S.q), p_base = smem_u32(S.p);
+    const uint64_t dq0 = smem_desc_kmajor(q_base, 128), dk0 = smem_desc_kmajor(kh_base, 128);
+    const uint64_t dv0 = smem_desc_mnmajor_sw128(kh_base, kTile * 128, 1024);
+    const uint64_t dp0 = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
+    bool ok = true;
+#pragma unroll 1
+    for (int it = 0; it < n_tiles && ok; ++it) {
+      // S^T = K^ Q^T, chunk by chunk as the chunks land
+#pragma unroll 1
+      for (int k = 0; k < NCH; ++k) {
+        if (!wait_or_abort(&S.chunk_full[k], it & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)   // descriptors advance by (byte offset >> 4)
+          tc_mma_f16(tmem + kColS, dk0 + ((k * (kTile * 128) + kk * 32) >> 4),
+                     dq0 + ((k * (kHeads * 128) + kk * 32) >> 4), kIdS, (k > 0 || kk > 0) ? 1u : 0u);
+      }
+      if (!ok) break;
+      tc_commit(&S.s_full);
+      if (!wait_or_abort(&S.p_full, it & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      const uint64_t da = smem_desc_mnmajor_sw128(kh_base, kTile * 128, 1024);
-      const uint64_t db = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
+      const uint32_t acc0 = it > 0 ? 1u : 0u;
+      // L^T += 1 P^T (every lane gets the per-head sums of P)
+#pragma unroll
+      for (int ks = 0; ks < kTile / 16; ++ks)
+        tc_mma_f16_ta(tmem + kColL, tmem + kColOnes, dp0 + (((2 * ks) * 1024) >> 4), kIdL, (ks > 0) ? 1u : acc0);
+      // O^T += V^T P^T per 128-channel block; each block's commit frees its two K^ chunks
 #pragma unroll
       for (int mt = 0; mt < MT; ++mt) {
-        if (mt < mt_lo || mt >= mt_hi) continue;
+        if (mt >= mt_lo && mt < mt_hi) {
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
-          tc_mma_f16(tmem + kHeads + mt * kHeads, da + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
-                     db + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0 || !first) ? 1u : 0u);
+          for (int ks = 0; ks < kTile / 16; ++ks)
+            tc_mma_f16(tmem + kColO + mt * kHeads, dv0 + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
+                       dp0 + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0) ? 1u : acc0);
+        }
+        tc_commit(&S.o_done[mt]);
       }
-      tc_commit(&S.obar);
     }
-    ++n_done;
+    tc_commit(&S.fin);   // arrives once every MMA issued above is done
   }
 
   // ---- epilogue: O^T (TMEM lane = channel within a 128-channel block)
-  bool ok = !aborted;
-  if (ok && n_done > 0) ok = mbar_wait_bounded(&S.obar, (n_done - 1) & 1, kWaitLimit);
-  const bool failed = __syncthreads_or(!ok);
+  bool ok = *abort == 0;
+  if (ok && n_tiles > 0 && tid < kDq) ok = wait_or_abort(&S.fin, 0, abort);
+  const bool failed = __syncthreads_or(!ok) || *abort != 0;
+  const size_t nrows = (size_t)a.B * a.T_q;
   if (failed) {
     if (tid == 0) flag(a.status, CSA2_DEV_TIMEOUT);
-    if (tid == 128 && n_done > 0) {   // let every issued MMA finish before TMEM is freed
-      mbar_init(&S.sbar, 1);
-      fence_barrier_init();
-      tc_commit(&S.sbar);
-      mbar_wait_bounded(&S.sbar, 0, kWaitLimit);
-    }
-  } else {
+    if (warp == kMmaWarp && lane == 0) mbar_wait_bounded(&S.fin, 0, kWaitLimit);   // every issued MMA done
+  } else if (tid < kDq) {
     tc_fence_after();
-    const size_t nrows = (size_t)a.B * a.T_q;
+    const int quarter = warp & 3, half = warp >> 2;   // TMEM lane quarter, 32-head half
+    const uint32_t lrow = tmem + ((uint32_t)(32 * quarter) << 16);
+    float linv[32];
+    {
+      uint32_t lv[32];
+      if (n_tiles > 0) {
+        tmem_ld_x32(lrow + kColL + 32 * half, lv);
+        tmem_wait_ld();
+      } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) lv[j] = 0u;
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const float l = __uint_as_float(lv[j]);
+        linv[j] = l > 0.f ? 1.f / l : 0.f;
+      }
+      if (quarter == 0 && lane == 0) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) S.lsum[32 * half + j] = __uint_as_float(lv[j]);
+      }
+    }
     // O / l per head.  One split: bf16, staged head-major [64 heads][D] in
     // the K^ tile (free once the last O^T MMA completed), then written out in
-    // 16-byte pieces.  Several splits: fp16 partials straight from registers
-    // (a channel per lane; staging measured slower on this latency-bound path).
-    float linv[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float l = S.l_run[32 * half + j];
-      linv[j] = l > 0.f ? 1.f / l : 0.f;
-    }
+    // 16-byte pieces.  Several splits: fp16 partials straight from registers.
     uint16_t *ob = reinterpret_cast<uint16_t *>(S.kh);
 #pragma unroll 1
     for (int mt = mt_lo; mt < mt_hi; ++mt) {
       const int ch = mt * 128 + 32 * quarter + lane;
       uint32_t o[32];
-      if (n_done > 0) {
-        tmem_ld_x32(tmem + ((uint32_t)(32 * quarter) << 16) + kHeads + mt * kHeads + 32 * half, o);
+      if (n_tiles > 0) {
+        tmem_ld_x32(lrow + kColO + mt * kHeads + 32 * half, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -512,32 +558,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
         for (int j = 0; j < 32; ++j) po[(size_t)(32 * half + j) * D] = __float2half_rn(__uint_as_float(o[j]) * linv[j]);
       }
     }
+  }
+  __syncthreads();
+  if (!failed) {
     if (a.nsplit == 1) {
-      __syncthreads();
-      const uint4 *src = reinterpret_cast<const uint4 *>(ob);
+      const uint4 *src = reinterpret_cast<const uint4 *>(S.kh);
       uint4 *dst = reinterpret_cast<uint4 *>(a.out + (size_t)row * a.H * D);
       const int n16 = a.H * (D / 8);
 #pragma unroll 4
       for (int i = tid; i < n16; i += kThreads) dst[i] = src[i];
-    }
-    if (a.nsplit > 1 && tid < kHeads) {
+    } else if (tid < kHeads) {
       float *pm = partial_stats(a, nrows) + ((size_t)row * a.nsplit + split) * kHeads;
       float *pl = pm + nrows * a.nsplit * kHeads;
       pm[tid] = S.m_ref[tid];
-      pl[tid] = S.l_run[tid];
+      pl[tid] = S.lsum[tid];
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, kCols);
+    tmem_dealloc(tmem, kTmemCols);
   }
 
   // ---- merge of the splits (the row's blocks form one cluster)
   if (a.nsplit > 1) {
     cluster_sync_all();   // every split's partials are written
-    const size_t nrows = (size_t)a.B * a.T_q;
     const float *pm = partial_stats(a, nrows) + (size_t)row * a.nsplit * kHeads;
     const float *pl = pm + nrows * a.nsplit * kHeads;
     if (tid < kHeads) {   // all 2 x nsplit loads in flight together
@@ -621,9 +667,9 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   const int nc = (K + kTile - 1) / kTile + (window + kTile - 1) / kTile;
   // One block per SM at a time (shared memory), so a launch takes
   // ceil(blocks / SMs) waves; a block costs one unit per key tile, plus
-  // about 0.8 for writing and merging split partials, plus 0.2 of set-up
-  // (measured per-phase cycle counts).  Take the split count of least cost
-  // (at most 8: the splits of a row form one cluster).
+  // about 0.8 for writing and merging split partials, plus 0.2 of set-up.
+  // Take the split count of least cost (at most 8: the splits of a row form
+  // one cluster).
   int nsplit = 1, cps = nc;
   double best = 1e30;
   for (int ns = 1; ns <= 8 && ns <= nc; ++ns) {
@@ -649,8 +695,7 @@ static cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(attn_kernel<D>, dim3(a.B * a.T_q, a.nsplit, a.csplit), dim3(kThreads), smem, s,
-                    dim3(1, (unsigned)a.nsplit, 1),
-                    a);
+                    dim3(1, (unsigned)a.nsplit, 1), a);
 }
 
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s) {

@@ -51,10 +51,6 @@ struct IndexSmem {
   int n_issued, n_mma;
 };
 
-__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 // Bounded wait that also gives up early once another role raised `abort`.
 __device__ __forceinline__ bool wait_or_abort(uint64_t *bar, uint32_t parity, volatile int *abort) {
   for (uint32_t i = 0; i < kWaitLimit; ++i) {
@@ -278,6 +274,13 @@ __global__ void __launch_bounds__(kThreads, 4) index_kernel(const __grid_constan
       float *out = a.scores + (size_t)row * a.ld;
       if (REINDEX) out[tile * kTileRows + r] = valid ? sum * sk : -INFINITY;
       else if (valid) out[e] = sum * sk;
+      if (!REINDEX && a.bmax) {   // the maximum of each block of 8 entries (8 consecutive lanes)
+        float m = valid ? sum * sk : -INFINITY;
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+        if ((r & 7) == 0 && e < n_vis) a.bmax[(size_t)row * a.ld_b + (e >> 3)] = m;
+      }
     }
   }
 
@@ -490,8 +493,15 @@ __global__ void __launch_bounds__(multi_threads<R>(), 1) index_multi_kernel(cons
           }
           head_reduce_reg<kMultiChunk>(s4, &wr[k][c * kMultiChunk], acc);
         }
-        if (e < nv_mine[k])
-          a.scores[(size_t)(row0 + my_row + k) * a.ld + e] = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * sk;
+        const float sc = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * sk;
+        if (e < nv_mine[k]) a.scores[(size_t)(row0 + my_row + k) * a.ld + e] = sc;
+        if (a.bmax) {   // the maximum of each block of 8 entries (8 consecutive lanes)
+          float m = e < nv_mine[k] ? sc : -INFINITY;
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+          m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+          if ((r & 7) == 0 && e < nv_mine[k]) a.bmax[(size_t)(row0 + my_row + k) * a.ld_b + (e >> 3)] = m;
+        }
       }
     }
   }

@@ -74,6 +74,8 @@ struct IndexArgs {
   int P;
   int tiles_per_row;      // reindex: P/16; full: cap/128 (the visible count is found in the kernel)
   int ctas_per_row;       // blocks sharing one row's tiles
+  float *bmax;            // full mode, optional: [B*T_q][ld_b] maximum score of each block of 8 entries
+  int64_t ld_b;
   uint8_t *q8;            // workspace: [B*T_q][64*dI] prepared FP8 query (MMA layout)
   float *wq;              // workspace: [B*T_q][64] w_h * s_q,h
   bool prepared;          // q8/wq already hold the query (no preparation kernel)
@@ -135,6 +137,22 @@ TopkPlan plan_topk(int rows, int n_cols, int K, int P_out);
 cudaError_t launch_topk(const TopkArgs &a, const TopkPlan &p, cudaStream_t s);
 bool topk_cluster_fits(int n_cols);                              // one cluster per row, no workspace
 cudaError_t launch_topk_cluster(const TopkArgs &a, cudaStream_t s);
+
+// Top-K and pool from the block maxima a Full scan wrote (one block per row).
+struct TopkBmaxArgs {
+  const float *scores;    // [rows][ld]
+  int64_t ld;
+  const float *bmax;      // [rows][ld_b]
+  int64_t ld_b;
+  int rows, n_cols;
+  const int32_t *n_valid; // [rows] or nullptr
+  int K;
+  int32_t *out_idx;       // [rows][K]
+  int P_out;
+  int32_t *out_pool;      // [rows][P_out]
+};
+constexpr int kTopkBmaxMaxBlocks = 16384;   // blocks of 8 columns per row (131,072 columns)
+cudaError_t launch_topk_bmax(const TopkBmaxArgs &a, cudaStream_t s);
 
 struct AttnArgs {
   const uint8_t *codes, *scales;

@@ -201,6 +201,31 @@ CSA2_API csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const
                               const void *ws, size_t ws_bytes, csa2_stream_t stream);
 
 /*
+ * 2c. Full scoring fused with the first level of the Top-K and pool selection
+ *     [jaehun "2) CSA2": the Full layer scans every entry, keeps the Top-512
+ *     and builds the 2,048 blocks x 8 positions pool (paper sec. 2.3.2,
+ *     Fig. 5)].  The scan's epilogue writes, with the scores, the maximum of
+ *     every block of 8 entries; the selection reads those maxima (not the
+ *     scores) to pick the pool and the K-th largest block maximum tau, and
+ *     then only the scores of the blocks whose maximum is >= tau (every Top-K
+ *     entry lies in one).  Results are those of csa2_index_full followed by
+ *     csa2_topk(scores, ..., n_valid, NULL, K, out_idx, P_out, out_pool).
+ *  q_idx, w  as for csa2_index_full; both NULL: the query was prepared in ws
+ *            by csa2_append_quant_ex (then ws starts with that preparation)
+ *  scores [B*T_q][ld] f32 out (ld >= cap, a multiple of 4), n_valid as for
+ *            csa2_index_full (may be NULL)
+ *  K, out_idx, P_out, out_pool as for csa2_topk
+ *  ws, ws_bytes: csa2_index_topk_workspace_size(B*T_q, cap, d_I) bytes
+ * Supported: cap <= 131,072 (rows of more entries: csa2_index_full +
+ * csa2_topk), 1 <= K <= 2048, 0 <= P_out <= 4096.
+ */
+CSA2_API csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
+                                     const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
+                                     int32_t *n_valid, int K, int32_t *out_idx, int P_out, int32_t *out_pool,
+                                     void *ws, size_t ws_bytes, csa2_stream_t stream);
+CSA2_API size_t csa2_index_topk_workspace_size(int rows, int cap, int d_I);
+
+/*
  * 3. Reindex scoring  [jaehun "2) CSA2": later Reindex layers rescore only the
  *    <= 2,048 blocks x 8 positions pool built by the first Full layer; the toy
  *    example: KV reused, indices recomputed with the layer's own indexer Q].

@@ -360,6 +360,64 @@ def _ref_topk_rows(s, n_valid, K):
     return np.stack([oracle.topk(s[r, :n_valid[r]].astype(np.float64), K) for r in range(s.shape[0])])
 
 
+@pytest.mark.parametrize("B,n,T_q,m,K,P,mode", [(8, 20000, 1, 1, 512, 2048, "plain"),
+                                                 (4, 65536, 1, 1, 512, 2048, "prepared"),
+                                                 (2, 131072, 1, 1, 512, 2048, "plain"),
+                                                 (1, 9000, 8, 2, 512, 0, "plain"),
+                                                 (2, 3000, 4, 1, 512, 256, "plain"),
+                                                 (3, 500, 1, 1, 512, 2048, "plain"),
+                                                 (2, 12000, 1, 1, 100, 64, "constant")])
+def test_index_topk_equals_scan_then_topk(B, n, T_q, m, K, P, mode):
+    """csa2_index_topk (block maxima from the scan's epilogue, selection from
+    them) gives bit for bit the scores, n_valid, Top-K and pool of
+    csa2_index_full followed by csa2_topk -- on ordinary rows, on a short
+    context (fewer blocks than K), with several query rows per sequence, and
+    on a cache of identical entries (every block ties: the whole-row path)."""
+    D, dI, H_I = 256, 128, 64
+    cap = (n // m + 127) // 128 * 128
+    g = gen(n + K + T_q)
+    gm = C.MainCache(B, cap, D, dI, m)
+    if mode == "constant":
+        kv = torch.randn(1, 1, D, generator=g).to(torch.bfloat16).expand(B, n, D).contiguous()
+    else:
+        kv = torch.randn(B, n, D, generator=g).to(torch.bfloat16)
+    gate = torch.randn(B, n, D, generator=g).to(torch.bfloat16) if m == 2 else None
+    W = (torch.randn(D, dI, generator=g) / math.sqrt(D)).to(torch.bfloat16)
+    C.csa2_append_quant(gm, kv.cuda(), gate.cuda() if gate is not None else None, W.cuda(), None, None,
+                        torch.zeros(B, dtype=torch.int32).cuda(), n)
+    qi = torch.randn(B, T_q, H_I, dI, generator=g).to(torch.bfloat16).cuda()
+    w = torch.rand(B, T_q, H_I, generator=g).cuda()
+    qpos = torch.tensor(np.stack([np.arange(n - T_q, n) - 3 * b for b in range(B)]), dtype=torch.int32).cuda()
+    rows = B * T_q
+    s1 = torch.full((rows, cap), float("nan"), device="cuda")
+    nv1 = torch.empty(rows, dtype=torch.int32, device="cuda")
+    i1 = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    p1 = torch.empty(rows, max(P, 1), dtype=torch.int32, device="cuda")
+    C.csa2_index_full(gm, qi, w, qpos, s1, nv1)
+    wst = C.workspace(C.csa2_topk_workspace_size(rows, cap, K, P))
+    C.csa2_topk(s1, cap, K, i1, n_valid=nv1, P_out=P, out_pool=p1 if P else None, ws=wst)
+    s2 = torch.full((rows, cap), float("nan"), device="cuda")
+    nv2 = torch.empty(rows, dtype=torch.int32, device="cuda")
+    i2 = torch.full((rows, K), -7, dtype=torch.int32, device="cuda")
+    p2 = torch.full((rows, max(P, 1)), -7, dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_index_topk_workspace_size(rows, cap, dI))
+    if mode == "prepared":
+        C.csa2_append_quant_ex(gm, None, None, None, None, None, torch.full((B,), n, dtype=torch.int32).cuda(), 0,
+                               qi, w, ws)
+        C.csa2_index_topk(gm, None, None, qpos, s2, K, i2, n_valid=nv2, P_out=P, out_pool=p2 if P else None, ws=ws)
+    else:
+        C.csa2_index_topk(gm, qi, w, qpos, s2, K, i2, n_valid=nv2, P_out=P, out_pool=p2 if P else None, ws=ws)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    assert torch.equal(nv1, nv2)
+    for r in range(rows):
+        k = int(nv1[r])
+        assert torch.equal(s1[r, :k].view(torch.int32), s2[r, :k].view(torch.int32))
+    assert torch.equal(i1, i2)
+    if P:
+        assert torch.equal(p1, p2)
+
+
 @pytest.mark.parametrize("rows,n,K,P,levels", [(3, 4096, 64, 2048, None), (2, 65536, 512, 2048, None),
                                                (4, 20000, 512, 2048, 50), (2, 300, 512, 2048, None),
                                                (1, 262144, 512, 2048, None), (2, 9000, 2048, 0, 3),
