@@ -57,6 +57,7 @@ SIGNATURES = {
     "csa2_topk_noalloc": (_I, [_P, _I, _I64, _I, _P, _P, _I, _P, _I, _P, _P]),
     "csa2_sparse_attn_decode": (_I, [_PM, _PS, _P, _P, _I, _I, _P, _I, _F, _P, _P, _SZ, _P]),
     "csa2_attn_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "csa2_debug_inject_timeout": (None, [ctypes.c_uint32]),
     "csa2_last_error": (ctypes.c_char_p, []),
     "csa2_device_status": (_I, [_P, ctypes.POINTER(ctypes.c_uint32), _I]),
     "csa2_version": (_I, []),
@@ -325,6 +326,12 @@ def csa2_device_status(clear: bool = True, stream=None) -> int:
     if st not in (CSA2_OK, 4):
         _check(st)
     return int(v.value)
+
+
+def csa2_debug_inject_timeout(polls: int):
+    """Diagnostic: later indexer scans wait `polls` polls on a barrier nothing
+    arrives on and take the give-up path (0 switches it off)."""
+    lib().csa2_debug_inject_timeout(int(polls))
 
 
 def csa2_version() -> int:

@@ -1,10 +1,13 @@
 // C ABI of libcsa2 (declared in include/csa2.h): argument validation, TMA
 // descriptor encoding, launch planning.  Nothing here allocates device memory.
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
+
+#include <nvtx3/nvToolsExt.h>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -17,6 +20,14 @@ __device__ unsigned int g_status;
 namespace {
 
 thread_local std::string t_err;
+std::atomic<uint32_t> g_inject_polls{0};
+
+// An NVTX range named after the entry point for the duration of the call
+// (host side: validation and launches), visible in Nsight timelines.
+struct NvtxRange {
+  explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 
 csa2_status fail(csa2_status st, const char *fmt, ...) {
   char buf[512];
@@ -150,6 +161,8 @@ csa2_status check_swa(const csa2_swa_cache *s) {
 
 void set_last_error_message(const char *msg) { t_err = msg; }
 
+uint32_t injected_timeout_polls() { return g_inject_polls.load(std::memory_order_relaxed); }
+
 }  // namespace csa2
 
 using namespace csa2;
@@ -159,6 +172,8 @@ extern "C" {
 int csa2_version(void) { return (1 << 16) | 0; }
 
 const char *csa2_last_error(void) { return t_err.c_str(); }
+
+void csa2_debug_inject_timeout(uint32_t polls) { g_inject_polls.store(polls, std::memory_order_relaxed); }
 
 csa2_status csa2_device_status(csa2_stream_t stream, uint32_t *flags, int clear) {
   if (!flags) return fail(CSA2_ERR_INVALID_ARG, "flags is NULL");
@@ -233,6 +248,7 @@ csa2_status csa2_append_quant(const csa2_main_cache *main, const uint16_t *kv, c
                               const uint16_t *w_ik, const csa2_swa_cache *swa, const uint16_t *kv_swa,
                               const int32_t *pos0, int T, csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_append_quant");
   return append_impl(main, kv, gate, w_ik, swa, kv_swa, pos0, T, nullptr, stream);
 }
 
@@ -241,6 +257,7 @@ csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uint16_t *kv
                                  const int32_t *pos0, int T, const uint16_t *q_idx, const float *w, int T_q,
                                  int H_I, void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_append_quant_ex");
   if (!main) return fail(CSA2_ERR_INVALID_ARG, "preparing a scan's query needs the main cache (its d_I)");
   if (!q_idx || !w || !aligned16(q_idx) || !aligned16(w))
     return fail(CSA2_ERR_INVALID_ARG, "q_idx and w must be 16-byte aligned device pointers");
@@ -261,6 +278,7 @@ csa2_status csa2_append_quant_ex(const csa2_main_cache *main, const uint16_t *kv
 csa2_status csa2_append_project(const csa2_main_cache *main, const uint16_t *h, int d_model, const uint16_t *w_kv,
                                 const uint16_t *w_ik, const int32_t *pos0, int T, csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_append_project");
   csa2_status st;
   if ((st = check_main(main, false)) != CSA2_OK) return st;
   if (main->m != 1) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "the projected append serves m = 1 caches (m=%d)", main->m);
@@ -327,6 +345,7 @@ static csa2_status index_common(const csa2_main_cache *main, const uint16_t *q_i
   a->B = main->B; a->cap = main->cap; a->m = main->m; a->dI = main->d_I;
   a->q_idx = q_idx; a->w = w; a->q_pos = q_pos; a->T_q = T_q; a->H_I = H_I; a->scores = scores;
   a->prepared = prepared;
+  a->inject_polls = injected_timeout_polls();
   return CSA2_OK;
 }
 
@@ -368,6 +387,7 @@ csa2_status csa2_index_full(const csa2_main_cache *main, const uint16_t *q_idx, 
                             const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
                             int32_t *n_valid, void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_index_full");
   return index_full_impl(main, q_idx, w, q_pos, T_q, H_I, scores, ld, n_valid, ws, ws_bytes, false, stream);
 }
 
@@ -375,6 +395,7 @@ csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const int32_t 
                                      int64_t ld, int32_t *n_valid, const void *ws, size_t ws_bytes,
                                      csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_index_full_prepared");
   return index_full_impl(main, nullptr, nullptr, q_pos, T_q, 64, scores, ld, n_valid, const_cast<void *>(ws),
                          ws_bytes, true, stream);
 }
@@ -400,6 +421,7 @@ csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, 
                             int K, int32_t *out_idx, int P_out, int32_t *out_pool, void *ws, size_t ws_bytes,
                             csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_index_topk");
   csa2_status st;
   if ((st = check_main(main, false)) != CSA2_OK) return st;
   const bool prepared = !q_idx && !w;
@@ -432,6 +454,7 @@ csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_id
                                const int32_t *q_pos, int T_q, int H_I, const int32_t *pool_blocks, int P,
                                float *pool_scores, void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_index_reindex");
   IndexArgs a;
   CUtensorMap map;
   csa2_status st = index_common(main, q_idx, w, q_pos, T_q, H_I, pool_scores, ws, ws_bytes, &a, &map, 8);
@@ -456,6 +479,7 @@ csa2_status csa2_topk(const float *scores, int rows, int64_t ld, int n_cols, con
                       const int32_t *pool_blocks, int K, int32_t *out_idx, int P_out, int32_t *out_pool,
                       void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_topk");
   if (!scores || !out_idx || !aligned16(scores) || !aligned16(out_idx))
     return fail(CSA2_ERR_INVALID_ARG, "scores/out_idx must be 16-byte aligned device pointers");
   if (rows <= 0 || rows > 65535) return fail(CSA2_ERR_INVALID_ARG, "rows=%d", rows);
@@ -487,6 +511,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
                                     float softmax_scale, uint16_t *out, void *ws, size_t ws_bytes,
                                     csa2_stream_t stream) {
   t_err.clear();
+  NvtxRange nvtx("csa2_sparse_attn_decode");
   csa2_status st;
   if ((st = check_main(main, false)) != CSA2_OK) return st;
   if (!swa) return fail(CSA2_ERR_INVALID_ARG, "window cache is NULL");

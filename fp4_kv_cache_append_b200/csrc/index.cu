@@ -45,7 +45,7 @@ struct IndexSmem {
   alignas(1024) uint8_t tile[kStages][kTileRows * DI];   // A operand ring (K-major, swizzled)
   alignas(1024) uint8_t q8[kHeads * DI];                 // B operand (K-major, swizzled)
   alignas(16) float wq[kHeads];                          // w_h * s_q,h
-  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain, qbar;
+  uint64_t full[kStages], empty[kStages], tfull[2], tempty[2], drain, qbar, never;
   uint32_t tmem_base;
   int abort;
   int n_issued, n_mma;
@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 4) index_kernel(const __grid_constan
     for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 4); }
     mbar_init(&S.drain, 1);
     mbar_init(&S.qbar, 1);
+    mbar_init(&S.never, 1);   // nothing arrives on it (diagnostic timeout)
     S.abort = 0;
     S.n_issued = 0;
     S.n_mma = 0;
@@ -201,7 +202,8 @@ __global__ void __launch_bounds__(kThreads, 4) index_kernel(const __grid_constan
     // ------------------------------------------------ MMA issuer
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(S.q8);
-      const bool qok = wait_or_abort(&S.qbar, 0, abort);
+      if (a.inject_polls && !mbar_wait_bounded(&S.never, 0, a.inject_polls)) *abort = 1;
+      const bool qok = !*abort && wait_or_abort(&S.qbar, 0, abort);
       for (int i = 0; i < ntiles && qok; ++i) {
         const int s = i % kStages, ab = i & 1;
         if (!wait_or_abort(&S.full[s], (i / kStages) & 1, abort)) break;
@@ -338,7 +340,7 @@ struct MultiSmem {
   alignas(1024) uint8_t tile[kMultiStages][kTileRows * DI];
   alignas(1024) uint8_t q8[R * kHeads * DI];
   alignas(16) float wq[R][kHeads];
-  uint64_t full[kMultiStages], empty[kMultiStages], tfull[2], tempty[2], drain, qbar;
+  uint64_t full[kMultiStages], empty[kMultiStages], tfull[2], tempty[2], drain, qbar, never;
   uint32_t tmem_base;
   int abort;
   int n_issued, n_mma;
@@ -364,6 +366,7 @@ __global__ void __launch_bounds__(multi_threads<R>(), 1) index_multi_kernel(cons
     for (int x = 0; x < 2; ++x) { mbar_init(&S.tfull[x], 1); mbar_init(&S.tempty[x], 4 * R / kMultiRpw); }
     mbar_init(&S.drain, 1);
     mbar_init(&S.qbar, 1);
+    mbar_init(&S.never, 1);   // nothing arrives on it (diagnostic timeout)
     S.abort = 0;
     S.n_issued = 0;
     S.n_mma = 0;
@@ -431,7 +434,8 @@ __global__ void __launch_bounds__(multi_threads<R>(), 1) index_multi_kernel(cons
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t q_addr = smem_u32(S.q8);
-      const bool qok = wait_or_abort(&S.qbar, 0, abort);
+      if (a.inject_polls && !mbar_wait_bounded(&S.never, 0, a.inject_polls)) *abort = 1;
+      const bool qok = !*abort && wait_or_abort(&S.qbar, 0, abort);
       for (int i = 0; i < ntiles && qok; ++i) {
         const int s = i % kMultiStages, ab = i & 1;
         if (!wait_or_abort(&S.full[s], (i / kMultiStages) & 1, abort)) break;

@@ -80,7 +80,10 @@ struct IndexArgs {
   float *wq;              // workspace: [B*T_q][64] w_h * s_q,h
   bool prepared;          // q8/wq already hold the query (no preparation kernel)
   unsigned int *status;
+  uint32_t inject_polls;  // diagnostic: > 0 makes the MMA issuer first wait this many polls on a
+                          // barrier nothing arrives on (a wait that runs out, then the abort path)
 };
+uint32_t injected_timeout_polls();   // csa2_debug_inject_timeout's setting (0 = off)
 size_t index_workspace_bytes(int rows, int dI);
 int index_rows_per_block(int T_q, bool reindex);   // query rows sharing one scan block (1, 2 or 4)
 cudaError_t launch_index(const CUtensorMap &ik_map, const IndexArgs &a, bool reindex, int sms,

@@ -30,6 +30,8 @@
 #include <cstdio>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -83,11 +85,25 @@ csa2_status scratch_address(void **out) {
 
 using namespace csa2;
 
+static csa2_status topk_noalloc_impl(const float *scores, int rows, int64_t ld, int n_cols, const int32_t *n_valid,
+                                     const int32_t *pool_blocks, int K, int32_t *out_idx, int P_out,
+                                     int32_t *out_pool, csa2_stream_t stream);
+
 extern "C" CSA2_API csa2_status csa2_topk_noalloc(const float *scores, int rows, int64_t ld, int n_cols,
                                                   const int32_t *n_valid, const int32_t *pool_blocks, int K,
                                                   int32_t *out_idx, int P_out, int32_t *out_pool,
                                                   csa2_stream_t stream) {
   set_last_error_message("");
+  nvtxRangePushA("csa2_topk_noalloc");
+  const csa2_status st = topk_noalloc_impl(scores, rows, ld, n_cols, n_valid, pool_blocks, K, out_idx, P_out, out_pool,
+                                           stream);
+  nvtxRangePop();
+  return st;
+}
+
+static csa2_status topk_noalloc_impl(const float *scores, int rows, int64_t ld, int n_cols, const int32_t *n_valid,
+                                     const int32_t *pool_blocks, int K, int32_t *out_idx, int P_out,
+                                     int32_t *out_pool, csa2_stream_t stream) {
   if (!scores || !out_idx || !noalloc_aligned16(scores) || !noalloc_aligned16(out_idx))
     return noalloc_fail(CSA2_ERR_INVALID_ARG, "scores/out_idx must be 16-byte aligned device pointers");
   if (rows <= 0 || rows > 65535) return noalloc_fail(CSA2_ERR_INVALID_ARG, "rows=%d", rows);

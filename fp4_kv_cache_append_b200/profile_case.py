@@ -42,10 +42,11 @@ def main():
             ms = sorted(s_.elapsed_time(e_) for s_, e_ in pairs)
             print(f"{name:14s} {len(pairs) // args.time} call(s) per step, {sum(ms) / len(ms):9.3f} ms per call "
                   f"(min {ms[0]:.3f})")
-        if "index_full" in events:
-            ms = min(s_.elapsed_time(e_) for s_, e_ in events["index_full"])
+        scan = "index_topk" if "index_topk" in events else "index_full"
+        if scan in events:
+            ms = min(s_.elapsed_time(e_) for s_, e_ in events[scan])
             flop = 2.0 * wl.H_I * wl.dI * float(st.n_valid.sum().item())
-            print(f"index_full: {flop / 1e12:.2f} TFLOP of FP8 MMA per call, {flop / (ms * 1e-3) / 1e12:.1f} TFLOP/s "
+            print(f"{scan}: {flop / 1e12:.2f} TFLOP of FP8 MMA per call, {flop / (ms * 1e-3) / 1e12:.1f} TFLOP/s "
                   f"at the fastest call")
     flags = C.csa2_device_status()
     print(f"profile_case {args.workload}: {args.steps} steps done, device status {flags:#x}")

@@ -101,7 +101,12 @@ class Step:
         ws_at = C.csa2_attn_workspace_size(B, self.T_q, wl.H, D, wl.K, wl.window)
         self.ws_topk = C.workspace(max(ws_full, ws_re), dev)
         self.ws_attn = C.workspace(ws_at, dev)
-        self.ws_index = C.workspace(C.csa2_index_workspace_size(self.rows, wl.dI), dev)
+        # Full layers of contexts up to 131,072 entries select from the block
+        # maxima their scan writes (csa2_index_topk); longer ones scan, then select
+        self.fused = wl.mode in ("full", "prefill") and self.cap <= 131072
+        ws_i = (C.csa2_index_topk_workspace_size(self.rows, self.cap, wl.dI) if self.fused
+                else C.csa2_index_workspace_size(self.rows, wl.dI))
+        self.ws_index = C.workspace(ws_i, dev)
 
     # ------------------------------------------------------------------ set-up (untimed)
 
@@ -173,11 +178,17 @@ class Step:
                 timed("append", lambda: C.csa2_append_quant_ex(main, self.kv_new, self.gate_new, self.w_ik, swa[l],
                                                                self.kv_swa_new[l], self.pos0, wl.T, self.q_idx[l],
                                                                self.w[l], self.ws_index))
-                timed("index_full", lambda: C.csa2_index_full_prepared(main, self.q_pos, self.scores, self.n_valid,
-                                                                       ws=self.ws_index))
-                timed("topk", lambda: C.csa2_topk(self.scores, self.cap, wl.K, self.idx, n_valid=self.n_valid,
-                                                  P_out=wl.P, out_pool=self.pool if wl.P else None,
-                                                  ws=self.ws_topk))
+                if self.fused:
+                    timed("index_topk", lambda: C.csa2_index_topk(main, None, None, self.q_pos, self.scores, wl.K,
+                                                                  self.idx, n_valid=self.n_valid, P_out=wl.P,
+                                                                  out_pool=self.pool if wl.P else None,
+                                                                  ws=self.ws_index))
+                else:
+                    timed("index_full", lambda: C.csa2_index_full_prepared(main, self.q_pos, self.scores,
+                                                                           self.n_valid, ws=self.ws_index))
+                    timed("topk", lambda: C.csa2_topk(self.scores, self.cap, wl.K, self.idx, n_valid=self.n_valid,
+                                                      P_out=wl.P, out_pool=self.pool if wl.P else None,
+                                                      ws=self.ws_topk))
             elif kind == "reindex":
                 timed("append", lambda: C.csa2_append_quant(None, None, None, None, swa[l], self.kv_swa_new[l],
                                                             self.pos0, wl.T))
@@ -196,15 +207,17 @@ class Step:
 
     def launches_per_step(self) -> int:
         """libcsa2 kernel launches one step enqueues (append 1, which also
-        prepares a Full scan's query; Full scan 1; Reindex 2 = query prep +
-        scan; Top-K 1 for rows of up to 65,536 columns else 4; attention 1)."""
+        prepares a Full scan's query; Full scan with the fused selection 2, or
+        scan 1 + Top-K; Reindex 2 = query prep + scan; Top-K 1 for rows of up
+        to 65,536 columns else 4 (1 for >= 128 rows of up to 131,072 without
+        a pool); attention 1)."""
         wl = self.wl
-        topk = lambda n_cols: 1 if n_cols <= 65536 else 4
+        topk = lambda n_cols: 1 if n_cols <= 65536 or (self.rows >= 128 and n_cols <= 131072 and not wl.P) else 4
         n = 0
         for kind, _ in self.plan:
             n += 1 + 1   # append, attention
             if kind == "full":
-                n += 1 + topk(self.cap)
+                n += 2 if self.fused else 1 + topk(self.cap)
             elif kind == "reindex":
                 n += 2 + topk(wl.P * 8)
         return n
@@ -233,6 +246,10 @@ class Step:
                 cols = self.cap if kind == "full" else wl.P * 8
                 out["topk"] = out.get("topk", 0) + self.rows * (cols * 4 + wl.K * 4) \
                     + (self.rows * wl.P * 4 if kind == "full" and wl.P else 0)
+        if self.fused:   # the scan's bytes plus the selection's: block maxima out and in, the candidates' scores
+            nb = (wl.entries + 7) // 8
+            out["index_topk"] = out.pop("index_full") + self.rows * (2 * nb * 4 + 8 * wl.K * 4 + wl.K * 4 + wl.P * 4)
+            out.pop("topk")
         return out
 
     def algorithmic_flops(self) -> dict:
@@ -244,7 +261,7 @@ class Step:
         for kind, _ in self.plan:
             if kind == "full":
                 vis = sum(min(wl.entries, (wl.first_new + j + 1) // wl.m) for j in range(self.T_q))
-                out["index_full"] = wl.B * vis * wl.H_I * wl.dI * 2
+                out["index_topk" if self.fused else "index_full"] = wl.B * vis * wl.H_I * wl.dI * 2
             if kind == "reindex":
                 out["index_reindex"] = self.rows * wl.P * 8 * wl.H_I * wl.dI * 2
             out["attn"] = out.get("attn", 0) + self.rows * (wl.K + wl.window) * wl.H * wl.D * 4

@@ -313,6 +313,15 @@ CSA2_API csa2_status csa2_topk_noalloc(const float *scores, int rows, int64_t ld
                                        int32_t *out_idx, int P_out, int32_t *out_pool,
                                        csa2_stream_t stream);
 
+/* Diagnostic: with polls > 0, the MMA-issuing warp of every later indexer
+ * scan (csa2_index_full, _prepared, _topk, _reindex) first waits `polls`
+ * polls on a barrier that nothing arrives on.  That wait runs out, and the
+ * scan takes the path of any wait that gives up: it sets CSA2_DEV_TIMEOUT,
+ * stops every role, waits (bounded) for its issued copies and MMAs, frees its
+ * tensor memory and returns, leaving its scores incomplete.  polls = 0 (the
+ * default) switches it off.  Process-wide; for tests of the give-up path. */
+CSA2_API void csa2_debug_inject_timeout(uint32_t polls);
+
 /* Thread-local description of the last error of this thread ("" if none). */
 CSA2_API const char *csa2_last_error(void);
 

@@ -319,6 +319,40 @@ def test_index_full_prepared_by_the_append(D, dI, H_I, T_q):
     assert C.csa2_device_status() == 0
 
 
+@pytest.mark.parametrize("T_q", [1, 4])
+def test_index_scan_wait_that_runs_out_flags_and_recovers(T_q):
+    """Failure detection without a fault: with csa2_debug_inject_timeout the
+    scan's MMA issuer waits on a barrier that nothing arrives on; the wait
+    runs out, the scan sets CSA2_DEV_TIMEOUT, stops every role, drains its
+    copies and MMAs, frees its tensor memory and returns.  The context stays
+    usable: the next scans give the reference scores again."""
+    B, n, D, dI, H_I = 2, 3000, 256, 128, 64
+    gm, _, om, _, _ = build_pair(B=B, cap=3072, D=D, dI=dI, m=1, T=n, pos0=[0, 0], seed=91, swa=False)
+    g = gen(92)
+    qi = torch.randn(B, T_q, H_I, dI, generator=g).to(torch.bfloat16).cuda()
+    w = torch.rand(B, T_q, H_I, generator=g).cuda()
+    qpos = torch.tensor(np.stack([np.arange(n - T_q, n)] * B), dtype=torch.int32).cuda()
+    ref = torch.zeros(B * T_q, 3072, device="cuda")
+    C.csa2_index_full(gm, qi, w, qpos, ref)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    bad = torch.zeros_like(ref)
+    C.csa2_debug_inject_timeout(64)
+    try:
+        C.csa2_index_full(gm, qi, w, qpos, bad)
+        torch.cuda.synchronize()
+    finally:
+        C.csa2_debug_inject_timeout(0)
+    assert C.csa2_device_status(clear=True) & C.DEV_TIMEOUT
+    assert not torch.equal(bad, ref)   # the scan gave up before writing its scores
+    again = torch.zeros_like(ref)
+    for _ in range(2):
+        C.csa2_index_full(gm, qi, w, qpos, again)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    assert torch.equal(again, ref)
+
+
 @pytest.mark.parametrize("T_q,m", [(8, 1), (6, 1), (4, 2)])
 def test_index_full_row_groups_match_single_rows(T_q, m):
     """T_q a multiple of 4 (or 2) takes the multi-row scan, which puts 4 (or 2)
