@@ -48,7 +48,9 @@ SIGNATURES = {
     "csa2_append_project": (_I, [_PM, _P, _I, _P, _P, _P, _I, _P]),
     "csa2_index_full": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _P, _SZ, _P]),
     "csa2_index_full_prepared": (_I, [_PM, _P, _I, _P, _I64, _P, _P, _SZ, _P]),
-    "csa2_index_topk": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _I, _P, _I, _P, _P, _SZ, _P]),
+    "csa2_index_topk": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I64, _P, _I, _P, _I, _P, _P, _P, _P, _SZ, _P]),
+    "csa2_topk_merge": (_I, [_P, _P, _I, _I, _I, ctypes.POINTER(ctypes.c_int32), _I, _P, _P, _P]),
+    "csa2_gather_entries": (_I, [_PM, _I, _P, _I, _P, _P, _I, _P, _P]),
     "csa2_index_topk_workspace_size": (_SZ, [_I, _I, _I]),
     "csa2_index_reindex": (_I, [_PM, _P, _P, _P, _I, _I, _P, _I, _P, _P, _SZ, _P]),
     "csa2_index_workspace_size": (_SZ, [_I, _I]),
@@ -255,7 +257,7 @@ def csa2_index_topk_workspace_size(rows: int, cap: int, d_I: int) -> int:
 
 
 def csa2_index_topk(main: MainCache, q_idx, w, q_pos, scores, K: int, out_idx, n_valid=None, P_out: int = 0,
-                    out_pool=None, ws=None, stream=None):
+                    out_pool=None, out_scores=None, out_pool_scores=None, ws=None, stream=None):
     """Full scan fused with the first selection level, then Top-K and pool.
     q_idx and w None: the query was prepared in ws by csa2_append_quant_ex."""
     T_q = q_pos.shape[-1]
@@ -264,7 +266,24 @@ def csa2_index_topk(main: MainCache, q_idx, w, q_pos, scores, K: int, out_idx, n
     _check(lib().csa2_index_topk(ctypes.byref(main.desc()), _ptr(q_idx, torch.bfloat16), _ptr(w, torch.float32),
                                  _ptr(q_pos, torch.int32), T_q, H_I, _ptr(scores, torch.float32), scores.shape[-1],
                                  _ptr(n_valid, torch.int32), int(K), _ptr(out_idx, torch.int32), int(P_out),
-                                 _ptr(out_pool, torch.int32), _ptr(ws), _nbytes(ws), _stream(stream)))
+                                 _ptr(out_pool, torch.int32), _ptr(out_scores, torch.float32),
+                                 _ptr(out_pool_scores, torch.float32), _ptr(ws), _nbytes(ws), _stream(stream)))
+
+
+def csa2_topk_merge(scores, ids, seg_base, K: int, out_ids, out_scores=None, stream=None):
+    """scores, ids [G][rows][n_seg] device tensors; seg_base: G ints (host)."""
+    G, rows, n_seg = scores.shape
+    base = (ctypes.c_int32 * G)(*[int(x) for x in seg_base])
+    _check(lib().csa2_topk_merge(_ptr(scores, torch.float32), _ptr(ids, torch.int32), G, rows, n_seg, base, int(K),
+                                 _ptr(out_ids, torch.int32), _ptr(out_scores, torch.float32), _stream(stream)))
+
+
+def csa2_gather_entries(shard: MainCache, lo: int, ids, out_codes, out_scales, out_pos=None, stream=None):
+    """ids [B][K]; out_codes [B][out_cap][D/2], out_scales [B][out_cap][D/16]."""
+    K = ids.shape[-1]
+    _check(lib().csa2_gather_entries(ctypes.byref(shard.desc()), int(lo), _ptr(ids, torch.int32), K,
+                                     _ptr(out_codes, torch.uint8), _ptr(out_scales, torch.uint8),
+                                     out_codes.shape[1], _ptr(out_pos, torch.int32), _stream(stream)))
 
 
 def csa2_index_reindex(main: MainCache, q_idx, w, q_pos, pool_blocks, pool_scores, ws=None, stream=None):

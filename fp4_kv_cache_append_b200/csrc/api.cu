@@ -418,8 +418,8 @@ size_t csa2_index_topk_workspace_size(int rows, int cap, int d_I) {
 
 csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                             const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld, int32_t *n_valid,
-                            int K, int32_t *out_idx, int P_out, int32_t *out_pool, void *ws, size_t ws_bytes,
-                            csa2_stream_t stream) {
+                            int K, int32_t *out_idx, int P_out, int32_t *out_pool, float *out_scores,
+                            float *out_pool_scores, void *ws, size_t ws_bytes, csa2_stream_t stream) {
   t_err.clear();
   NvtxRange nvtx("csa2_index_topk");
   csa2_status st;
@@ -433,6 +433,8 @@ csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, 
   if (!out_idx || !aligned16(out_idx)) return fail(CSA2_ERR_INVALID_ARG, "out_idx must be a 16-byte aligned device pointer");
   if (P_out > 0 && (!out_pool || !aligned16(out_pool))) return fail(CSA2_ERR_INVALID_ARG, "out_pool needed");
   if (ld % 4) return fail(CSA2_ERR_INVALID_ARG, "ld=%lld must be a multiple of 4", (long long)ld);
+  if ((out_scores && !aligned16(out_scores)) || (out_pool_scores && !aligned16(out_pool_scores)))
+    return fail(CSA2_ERR_INVALID_ARG, "out_scores / out_pool_scores must be 16-byte aligned");
   if (T_q <= 0 || (int64_t)main->B * T_q > 65535) return fail(CSA2_ERR_INVALID_ARG, "T_q=%d", T_q);
   const int rows = main->B * T_q;
   size_t off_b, off_nv;
@@ -445,9 +447,51 @@ csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, 
   st = index_full_impl(main, q_idx, w, q_pos, T_q, prepared ? 64 : H_I, scores, ld, nv, ws, ws_bytes, prepared,
                        stream, bmax, main->cap / 8);
   if (st != CSA2_OK) return st;
-  TopkBmaxArgs t{scores, ld, bmax, main->cap / 8, rows, main->cap, nv, K, out_idx, P_out, out_pool};
+  TopkBmaxArgs t{scores, ld, bmax, main->cap / 8, rows, main->cap, nv, K, out_idx, P_out, out_pool,
+                 out_scores, P_out > 0 ? out_pool_scores : nullptr};
   cudaError_t e = launch_topk_bmax(t, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "topk_bmax launch");
+}
+
+csa2_status csa2_topk_merge(const float *scores, const int32_t *ids, int G, int rows, int n_seg,
+                            const int32_t *seg_base, int K, int32_t *out_ids, float *out_scores,
+                            csa2_stream_t stream) {
+  t_err.clear();
+  NvtxRange nvtx("csa2_topk_merge");
+  if (!scores || !ids || !out_ids || !aligned16(scores) || !aligned16(ids) || !aligned16(out_ids))
+    return fail(CSA2_ERR_INVALID_ARG, "scores/ids/out_ids must be 16-byte aligned device pointers");
+  if (out_scores && !aligned16(out_scores)) return fail(CSA2_ERR_INVALID_ARG, "out_scores alignment");
+  if (!seg_base) return fail(CSA2_ERR_INVALID_ARG, "seg_base (host array of G ints) is NULL");
+  if (G < 1 || G > kMergeMaxShards) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "G=%d not in [1,%d]", G, kMergeMaxShards);
+  if (rows < 1 || rows > 65535 || n_seg < 1) return fail(CSA2_ERR_INVALID_ARG, "rows=%d n_seg=%d", rows, n_seg);
+  if ((int64_t)G * n_seg > kTopkBmaxMaxBlocks)
+    return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "G*n_seg=%lld above %d", (long long)G * n_seg, kTopkBmaxMaxBlocks);
+  if (K < 1 || K > 4096) return fail(CSA2_ERR_UNSUPPORTED_SHAPE, "K=%d not in [1,4096]", K);
+  TopkMergeArgs a{};
+  a.scores = scores; a.ids = ids; a.G = G; a.rows = rows; a.n_seg = n_seg;
+  for (int g = 0; g < G; ++g) a.seg_base[g] = seg_base[g];
+  a.K = K; a.out_ids = out_ids; a.out_scores = out_scores;
+  cudaError_t e = launch_topk_merge(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "topk_merge launch");
+}
+
+csa2_status csa2_gather_entries(const csa2_main_cache *shard, int lo, const int32_t *ids, int K,
+                                uint8_t *out_codes, uint8_t *out_scales, int out_cap, int32_t *out_pos,
+                                csa2_stream_t stream) {
+  t_err.clear();
+  NvtxRange nvtx("csa2_gather_entries");
+  csa2_status st;
+  if ((st = check_main(shard, false)) != CSA2_OK) return st;
+  if (!ids || !out_codes || !out_scales || !aligned16(ids) || !aligned16(out_codes) || !aligned16(out_scales))
+    return fail(CSA2_ERR_INVALID_ARG, "ids/out_codes/out_scales must be 16-byte aligned device pointers");
+  if (out_pos && !aligned16(out_pos)) return fail(CSA2_ERR_INVALID_ARG, "out_pos alignment");
+  if (lo < 0) return fail(CSA2_ERR_INVALID_ARG, "lo=%d", lo);
+  if (K < 1 || K > 4096 || out_cap < K) return fail(CSA2_ERR_INVALID_ARG, "K=%d out_cap=%d", K, out_cap);
+  GatherArgs a{};
+  a.codes = shard->codes; a.scales = shard->scales; a.B = shard->B; a.cap = shard->cap; a.D = shard->D; a.lo = lo;
+  a.ids = ids; a.K = K; a.out_codes = out_codes; a.out_scales = out_scales; a.out_cap = out_cap; a.out_pos = out_pos;
+  cudaError_t e = launch_gather_entries(a, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "gather_entries launch");
 }
 
 csa2_status csa2_index_reindex(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,

@@ -27,8 +27,9 @@
 //               major B operand [key][head]
 // So the dequantisation of chunk k+1 overlaps the S MMAs of chunk k, and the
 // next tile's dequantisation overlaps this tile's O^T MMAs.  Window rows keep
-// their raw E4M3 values; the layer's window scale multiplies their logits and
-// their P.
+// their raw E4M3 values: the layer's window scale multiplies their logits, and
+// O^T (not L) is divided by it when the window tiles start and multiplied by it
+// at the end, so their values count scaled and their P unscaled.
 // The splits of one row form a thread-block cluster: each writes O / l per
 // head (fp16, [head][channel]) and its (max, sum) per head to the workspace, and
 // after one cluster barrier each split merges a slice of the channels from all
@@ -359,7 +360,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       if (!__shfl_sync(0xffffffffu, w_ok, 0)) break;
       tc_fence_after();
       const float lsc = a.scale * (is_win ? a.s_swa : 1.0f) * kLog2e;
-      const float psc = is_win ? a.s_swa : 1.0f;
       const bool first = it == 0;
       float sv[64];
       auto load_logits = [&]() {
@@ -422,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
             const int j = 4 * j4 + k;
             sv[j] = (sv[j] == -INFINITY || mm[k] == -INFINITY) ? 0.f : ex2_approx(sv[j] - mm[k]);
           }
-          const __half2 h0 = __floats2half2_rn(sv[4 * j4] * psc, sv[4 * j4 + 1] * psc);
-          const __half2 h1 = __floats2half2_rn(sv[4 * j4 + 2] * psc, sv[4 * j4 + 3] * psc);
+          const __half2 h0 = __floats2half2_rn(sv[4 * j4], sv[4 * j4 + 1]);
+          const __half2 h1 = __floats2half2_rn(sv[4 * j4 + 2], sv[4 * j4 + 3]);
           ph[2 * j4] = *reinterpret_cast<const uint32_t *>(&h0);
           ph[2 * j4 + 1] = *reinterpret_cast<const uint32_t *>(&h1);
         }
@@ -432,20 +432,29 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
           *reinterpret_cast<uint4 *>(S.p + r * 128 + ((i ^ (r & 7)) << 4)) =
               make_uint4(ph[4 * i], ph[4 * i + 1], ph[4 * i + 2], ph[4 * i + 3]);
       }
-      // rare: a head's reference max moved -> rescale its O^T and L columns
-      // (the previous tile's O^T MMAs completed before S of this tile did)
-      if (need_max && S.rescale_at == it) {
+      // rare: a head's reference max moved -> rescale its O^T and L columns;
+      // and at the first window tile after FP4 tiles, O^T is divided by the
+      // window scale (window rows enter O^T unscaled; the epilogue multiplies
+      // the O of a block that saw window tiles by the scale).  The previous
+      // tile's MMAs completed before S of this tile did.
+      const bool moved = need_max && S.rescale_at == it;
+      const bool to_win = is_win && c == n_fp4_tiles && it > 0;
+      if (moved || to_win) {
+        const float inv_s = to_win ? 1.0f / a.s_swa : 1.0f;
 #pragma unroll 1
         for (int blk = 0; blk <= MT; ++blk) {
           if (blk < MT && (blk < mt_lo || blk >= mt_hi)) continue;
+          if (blk == MT && !moved) continue;
           const uint32_t base = srow + (blk < MT ? kColO + 64 * blk : kColL);
+          const float f = blk < MT ? inv_s : 1.0f;
 #pragma unroll 1
           for (int hh = 0; hh < 2; ++hh) {
             uint32_t o[32];
             tmem_ld_x32(base + 32 * hh, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * S.alpha[32 * hh + j]);
+            for (int j = 0; j < 32; ++j)
+              o[j] = __float_as_uint(__uint_as_float(o[j]) * ((moved ? S.alpha[32 * hh + j] : 1.0f) * f));
             tmem_st_x32(base + 32 * hh, o);
           }
         }
@@ -521,10 +530,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) lv[j] = 0u;
       }
+      // window rows entered O^T unscaled: a block that saw window tiles scales its O
+      const float osc = c_end > n_fp4_tiles && n_tiles > 0 ? a.s_swa : 1.0f;
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const float l = __uint_as_float(lv[j]);
-        linv[j] = l > 0.f ? 1.f / l : 0.f;
+        linv[j] = l > 0.f ? osc / l : 0.f;
       }
       if (quarter == 0 && lane == 0) {
 #pragma unroll

@@ -153,9 +153,37 @@ struct TopkBmaxArgs {
   int32_t *out_idx;       // [rows][K]
   int P_out;
   int32_t *out_pool;      // [rows][P_out]
+  float *out_scores;      // [rows][K] or nullptr: the selected entries' scores
+  float *out_pool_scores; // [rows][P_out] or nullptr: the pool blocks' maxima
 };
 constexpr int kTopkBmaxMaxBlocks = 16384;   // blocks of 8 columns per row (131,072 columns)
 cudaError_t launch_topk_bmax(const TopkBmaxArgs &a, cudaStream_t s);
+
+// Merge of G per-shard selections of one row each (see topk_merge_kernel).
+constexpr int kMergeMaxShards = 16;
+struct TopkMergeArgs {
+  const float *scores;    // [G][rows][n_seg]
+  const int32_t *ids;     // [G][rows][n_seg]
+  int G, rows, n_seg;
+  int seg_base[kMergeMaxShards];
+  int K;
+  int32_t *out_ids;       // [rows][K]
+  float *out_scores;      // [rows][K] or nullptr
+};
+cudaError_t launch_topk_merge(const TopkMergeArgs &a, cudaStream_t s);
+
+// Copies of selected entries of a context shard (entries lo .. lo + cap - 1
+// of each sequence) into a compact cache of one row per sequence.
+struct GatherArgs {
+  const uint8_t *codes, *scales;   // shard planes [B][cap][D/2], [B][cap][D/16]
+  int B, cap, D, lo;
+  const int32_t *ids;              // [B][K] global entry ids, -1 = none
+  int K;
+  uint8_t *out_codes, *out_scales; // [B][out_cap][D/2], [B][out_cap][D/16]
+  int out_cap;
+  int32_t *out_pos;                // [B][K] k where ids >= 0, else -1 (or nullptr)
+};
+cudaError_t launch_gather_entries(const GatherArgs &a, cudaStream_t s);
 
 struct AttnArgs {
   const uint8_t *codes, *scales;

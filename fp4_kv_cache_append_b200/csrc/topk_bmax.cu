@@ -42,6 +42,10 @@ __device__ __forceinline__ uint32_t skey(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+__device__ __forceinline__ float kval(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // Final rule of a selection: take key if key > kthr, or key == kthr and its
 // rank among the keys equal to kthr (in column order) is below take_eq.
 struct SelRule {
@@ -265,11 +269,17 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
       const bool tk = strictly_taken(key, pr) || (tie(key, pr) && tb < pr.take_eq);
       tb += tie(key, pr);
       if (tk) {
-        if (pos < a.P_out) op[pos] = tid * kBpt + i;
+        if (pos < a.P_out) {
+          op[pos] = tid * kBpt + i;
+          if (a.out_pool_scores) a.out_pool_scores[(size_t)row * a.P_out + pos] = kval(key);
+        }
         ++pos;
       }
     }
-    for (int i = n_pool + tid; i < a.P_out; i += kT) op[i] = -1;
+    for (int i = n_pool + tid; i < a.P_out; i += kT) {
+      op[i] = -1;
+      if (a.out_pool_scores) a.out_pool_scores[(size_t)row * a.P_out + i] = -INFINITY;
+    }
   }
 
   // ---- candidate blocks: maximum >= tau (every block when fewer than K are present)
@@ -318,7 +328,10 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
       const bool tk = strictly_taken(key, rule) || (tie(key, rule) && tb < rule.take_eq);
       tb += tie(key, rule);
       if (tk) {
-        if (pos < a.K) out[pos] = sh.cand_col[tid * kCpt + i];
+        if (pos < a.K) {
+          out[pos] = sh.cand_col[tid * kCpt + i];
+          if (a.out_scores) a.out_scores[(size_t)row * a.K + pos] = kval(key);
+        }
         ++pos;
       }
     }
@@ -334,12 +347,81 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
       const bool tk = strictly_taken(key, rule) || (tie(key, rule) && tb < rule.take_eq);
       tb += tie(key, rule);
       if (tk) {
-        if (pos < a.K) out[pos] = tid * rk.npt + i;
+        if (pos < a.K) {
+          out[pos] = tid * rk.npt + i;
+          if (a.out_scores) a.out_scores[(size_t)row * a.K + pos] = kval(key);
+        }
         ++pos;
       }
     });
   }
-  for (int i = K_take + tid; i < a.K; i += kT) out[i] = -1;
+  for (int i = K_take + tid; i < a.K; i += kT) {
+    out[i] = -1;
+    if (a.out_scores) a.out_scores[(size_t)row * a.K + i] = -INFINITY;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Merge of per-shard selections (a context split over several GPUs): row r's
+// candidates are G segments of n_seg (score, id) pairs, segment g at
+// [g][rows][n_seg]; candidate (g, i) stands for entry ids[g][r][i] +
+// seg_base[g] (ids < 0: none).  The K best by (score desc, entry asc), listed
+// ascending, -1 / -inf padded.  Each segment's ids ascend and the segments'
+// entry ranges ascend with g, so candidate order is entry order and the
+// selection's column tie rule is the entry tie rule.
+__global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkMergeArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  SelSmem &sel = *reinterpret_cast<SelSmem *>(smem_raw);
+  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  pdl_launch_dependents();
+  pdl_wait();
+  const int n = a.G * a.n_seg;
+  uint32_t key[kBpt];
+  int32_t gid[kBpt];
+#pragma unroll
+  for (int i = 0; i < kBpt; ++i) {
+    const int j = tid * kBpt + i;
+    key[i] = 0u;
+    gid[i] = -1;
+    if (j < n) {
+      const int g = j / a.n_seg, c = j % a.n_seg;
+      const size_t at = ((size_t)g * a.rows + row) * a.n_seg + c;
+      const int id = a.ids[at];
+      if (id >= 0) {
+        key[i] = skey(a.scores[at]);
+        gid[i] = id + a.seg_base[g];
+      }
+    }
+  }
+  const RegKeys<kBpt> ks{key};
+  const int k[1] = {a.K};
+  radix_select<1>(ks, k, sel, tid, lane, warp);
+  const SelRule rule = sel.rule[0];
+  const int K_take = min(sel.n_present, a.K);
+  int pos, tb;
+  taken_offsets(ks, rule, sel.red, lane, warp, pos, tb);
+  int32_t *out = a.out_ids + (size_t)row * a.K;
+#pragma unroll
+  for (int i = 0; i < kBpt; ++i) {
+    const bool tk = strictly_taken(key[i], rule) || (tie(key[i], rule) && tb < rule.take_eq);
+    tb += tie(key[i], rule);
+    if (tk) {
+      if (pos < a.K) {
+        out[pos] = gid[i];
+        if (a.out_scores) a.out_scores[(size_t)row * a.K + pos] = kval(key[i]);
+      }
+      ++pos;
+    }
+  }
+  for (int i = K_take + tid; i < a.K; i += kT) {
+    out[i] = -1;
+    if (a.out_scores) a.out_scores[(size_t)row * a.K + i] = -INFINITY;
+  }
+}
+
+cudaError_t launch_topk_merge(const TopkMergeArgs &a, cudaStream_t s) {
+  const size_t smem = sizeof(SelSmem);
+  return launch_pdl(topk_merge_kernel, dim3(a.rows), dim3(kT), smem, s, dim3(1, 1, 1), a);
 }
 
 size_t topk_bmax_smem() { return sizeof(Smem); }

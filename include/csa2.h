@@ -215,6 +215,10 @@ CSA2_API csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const
  *  scores [B*T_q][ld] f32 out (ld >= cap, a multiple of 4), n_valid as for
  *            csa2_index_full (may be NULL)
  *  K, out_idx, P_out, out_pool as for csa2_topk
+ *  out_scores [B*T_q][K] f32 out (may be NULL): the score of each selected
+ *            entry (-inf where out_idx is -1); out_pool_scores [B*T_q][P_out]
+ *            (may be NULL): each pool block's maximum (-inf padded) -- what a
+ *            context shard sends to the merge (entry 2d)
  *  ws, ws_bytes: csa2_index_topk_workspace_size(B*T_q, cap, d_I) bytes
  * Supported: cap <= 131,072 (rows of more entries: csa2_index_full +
  * csa2_topk), 1 <= K <= 2048, 0 <= P_out <= 4096.
@@ -222,8 +226,51 @@ CSA2_API csa2_status csa2_index_full_prepared(const csa2_main_cache *main, const
 CSA2_API csa2_status csa2_index_topk(const csa2_main_cache *main, const uint16_t *q_idx, const float *w,
                                      const int32_t *q_pos, int T_q, int H_I, float *scores, int64_t ld,
                                      int32_t *n_valid, int K, int32_t *out_idx, int P_out, int32_t *out_pool,
-                                     void *ws, size_t ws_bytes, csa2_stream_t stream);
+                                     float *out_scores, float *out_pool_scores, void *ws, size_t ws_bytes,
+                                     csa2_stream_t stream);
 CSA2_API size_t csa2_index_topk_workspace_size(int rows, int cap, int d_I);
+
+/*
+ * 2d. Context sharding across GPUs  [jaehun "2) CSA2" and Fig. 2: a long
+ *     context's decode cost is the Full scan over all entries, which splits by
+ *     entry range; the selection keeps <= 512 entries and 2,048 blocks].  With
+ *     a sequence's entries split by contiguous ranges over G GPUs, each rank
+ *     runs csa2_index_topk on its range (with out_scores / out_pool_scores),
+ *     the ranks exchange those (score, id) lists (an all-gather), and
+ *     csa2_topk_merge selects the global Top-K (and, with block ids, the pool)
+ *     from them: every global Top-K entry is in its own range's Top-K, so the
+ *     merge is exact.  csa2_gather_entries then copies, on each rank, the
+ *     merged selection's entries that rank holds into a compact cache (zeros
+ *     for the others); the ranks' buffers summed bytewise (one contributor
+ *     per slot) form the cache the attention runs on.
+ *
+ * csa2_topk_merge: per row, the K best of G segments of n_seg candidates.
+ *  scores, ids [G][rows][n_seg] f32 / i32 (DEVICE): segment g of row r is
+ *         rank g's list; candidate (g, i) is entry ids[g][r][i] + seg_base[g]
+ *         (ids < 0: none).  Each segment's ids ascend, and the segments'
+ *         entry ranges ascend with g (so ties go to the smaller entry).
+ *  seg_base [G] i32 HOST array: first entry of each rank's range
+ *  out_ids [rows][K] i32 out: the K best entries (score desc, entry asc),
+ *         ascending, -1 padded; out_scores [rows][K] f32 out (may be NULL)
+ * Supported: 1 <= G <= 16, G * n_seg <= 16,384, 1 <= K <= 4096.
+ */
+CSA2_API csa2_status csa2_topk_merge(const float *scores, const int32_t *ids, int G, int rows, int n_seg,
+                                     const int32_t *seg_base, int K, int32_t *out_ids, float *out_scores,
+                                     csa2_stream_t stream);
+
+/*
+ * csa2_gather_entries: the selected entries a shard holds, in selection order.
+ *  shard  the rank's main cache: its entry e is entry lo + e of the sequence
+ *  ids    [B][K] i32 global entry ids of the merged selection (-1 = none)
+ *  out_codes [B][out_cap][D/2], out_scales [B][out_cap][D/16] u8 out: slot k
+ *         holds entry ids[b][k] when lo <= ids[b][k] < lo + cap, else zeros
+ *  out_pos [B][K] i32 out (may be NULL): k where ids[b][k] >= 0, else -1 --
+ *         the selection as slots of the compact cache
+ * Supported: K <= out_cap, K <= 4096.
+ */
+CSA2_API csa2_status csa2_gather_entries(const csa2_main_cache *shard, int lo, const int32_t *ids, int K,
+                                         uint8_t *out_codes, uint8_t *out_scales, int out_cap, int32_t *out_pos,
+                                         csa2_stream_t stream);
 
 /*
  * 3. Reindex scoring  [jaehun "2) CSA2": later Reindex layers rescore only the
