@@ -10,10 +10,17 @@
 //
 // One 1024-thread block per row.  Thread t holds the keys of blocks
 // 16t .. 16t+15 (order-preserving 32-bit keys of the block maxima, 0 =
-// absent).  Two radix selections run side by side over them, 8 key bits per
-// round (histograms in shared memory, warp-aggregated atomics):
+// absent).  Two selections run side by side over them:
 //   * the pool: the P_out blocks with the largest maxima;
 //   * tau: the K-th largest block maximum.
+// A selection bins the keys by VALUE, linearly between the smallest and the
+// largest present value (256 bins, shared-memory atomics: values spread over
+// the bins, so few atomics collide), finds the bin holding the k-th largest
+// key, and ranks that bin's keys exactly (key desc, column asc) -- scores of
+// a row sit in a few binades, so binning by key bits would put nearly all of
+// them in one bin.  A bin of more than kColl keys (heavy ties, or one huge
+// outlier squeezing the rest into one bin) is resolved by a radix selection on
+// the key bits instead.
 // There are at least K distinct entries scoring >= tau (one per block whose
 // maximum is >= tau), so the K-th largest score s_K >= tau, and every entry
 // of the Top-K lies in a block whose maximum is >= s_K >= tau.  The entries
@@ -46,11 +53,16 @@ __device__ __forceinline__ float kval(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Final rule of a selection: take key if key > kthr, or key == kthr and its
-// rank among the keys equal to kthr (in column order) is below take_eq.
+constexpr int kColl = 2048;        // largest value bin ranked exactly
+
+// Final rule of a selection: take key if key > kthr, or key == kthr and
+// (cmode: its column <= cthr; else: its rank among the keys equal to kthr, in
+// column order, is below take_eq).
 struct SelRule {
   uint32_t kthr;
+  int cthr;
   int take_eq;
+  int cmode;
 };
 
 struct SelSmem {
@@ -60,13 +72,16 @@ struct SelSmem {
   SelRule rule[2];
   unsigned long long red[kW];
   int n_present;
+  uint32_t kmin, kmax;               // smallest / largest present key
+  int vbin_ok;                       // the value range gives usable bins
+  int T[2], cnt[2], n_coll[2], fallback[2];
+  uint2 coll[2][kColl];              // (key, column) of the threshold bin
 };
 
 struct Smem {
   SelSmem sel;
   uint32_t cand_key[kCap];
   int32_t cand_col[kCap];
-  int n_cand_blocks;
 };
 
 // Exclusive block scan of v; afterwards red[kW-1] holds the block total.
@@ -98,6 +113,8 @@ __device__ __forceinline__ unsigned long long block_scan(unsigned long long v, u
 template <int N>
 struct RegKeys {
   const uint32_t *k;
+  int t;
+  __device__ __forceinline__ int col(int i) const { return t * N + i; }
   template <typename F>
   __device__ __forceinline__ void each(F f) const {
 #pragma unroll
@@ -110,6 +127,7 @@ struct RegKeys {
 struct RowKeys {
   const float *row;
   int n, npt, t;
+  __device__ __forceinline__ int col(int i) const { return t * npt + i; }
   template <typename F>
   __device__ __forceinline__ void each(F f) const {
 #pragma unroll 1
@@ -136,7 +154,9 @@ __device__ void radix_select(const Keys &keys, const int *k, SelSmem &sm, int ti
     sm.need[tid] = k[tid];
     sm.done[tid] = present <= k[tid];
     sm.rule[tid].kthr = 0u;        // take every present key
+    sm.rule[tid].cthr = 0;
     sm.rule[tid].take_eq = 0;
+    sm.rule[tid].cmode = 0;
     if (tid == 0) sm.n_present = present;
   }
   __syncthreads();
@@ -190,10 +210,12 @@ __device__ void radix_select(const Keys &keys, const int *k, SelSmem &sm, int ti
         if ((int)cnt == need2) {            // every key of the bin is taken
           sm.rule[s].kthr = prefix;
           sm.rule[s].take_eq = 0x7FFFFFFF;
+          sm.rule[s].cmode = 0;
           sm.done[s] = 1;
         } else if (shift == 0) {            // one key value: need2 of its ties, in column order
           sm.rule[s].kthr = prefix;
           sm.rule[s].take_eq = need2;
+          sm.rule[s].cmode = 0;
           sm.done[s] = 1;
         }
       }
@@ -202,8 +224,12 @@ __device__ void radix_select(const Keys &keys, const int *k, SelSmem &sm, int ti
   }
 }
 
-__device__ __forceinline__ bool strictly_taken(uint32_t key, const SelRule &r) { return key != 0u && key > r.kthr; }
-__device__ __forceinline__ bool tie(uint32_t key, const SelRule &r) { return key != 0u && key == r.kthr; }
+// Keys taken whatever their rank among ties, and keys among which the rank
+// decides (ties of a take_eq rule).
+__device__ __forceinline__ bool strictly_taken(uint32_t key, int col, const SelRule &r) {
+  return key != 0u && (key > r.kthr || (r.cmode && key == r.kthr && col <= r.cthr));
+}
+__device__ __forceinline__ bool tie(uint32_t key, const SelRule &r) { return !r.cmode && key != 0u && key == r.kthr; }
 
 // Output positions of this thread's taken keys: the number of taken keys in
 // earlier columns.  Returns (position of my first taken key, ties before me).
@@ -211,13 +237,161 @@ template <typename Keys>
 __device__ void taken_offsets(const Keys &keys, const SelRule &rule, unsigned long long *red, int lane, int warp,
                               int &pos, int &ties_before) {
   int st = 0, tt = 0;
-  keys.each([&](uint32_t key, int) {
-    st += strictly_taken(key, rule);
+  keys.each([&](uint32_t key, int i) {
+    st += strictly_taken(key, keys.col(i), rule);
     tt += tie(key, rule);
   });
   const unsigned long long ex = block_scan(((unsigned long long)tt << 32) | (unsigned long long)st, red, lane, warp);
   ties_before = (int)(ex >> 32);
   pos = (int)(ex & 0xFFFFFFFFull) + min(ties_before, rule.take_eq);
+}
+
+// Visits this thread's taken keys in column order: f(key, i, position).
+template <typename Keys, typename F>
+__device__ void for_taken(const Keys &keys, const SelRule &rule, unsigned long long *red, int lane, int warp, F f) {
+  int pos, tb;
+  taken_offsets(keys, rule, red, lane, warp, pos, tb);
+  keys.each([&](uint32_t key, int i) {
+    const bool tk = strictly_taken(key, keys.col(i), rule) || (tie(key, rule) && tb < rule.take_eq);
+    tb += tie(key, rule);
+    if (tk) f(key, i, pos++);
+  });
+}
+
+__device__ __forceinline__ int vbin(uint32_t key, float vlo, float inv) {
+  const int b = (int)((kval(key) - vlo) * inv);
+  return b < 0 ? 0 : (b > 255 ? 255 : b);
+}
+
+// NS selections over the same keys (see the file comment): selection s finds
+// the k[s]-th largest present key; afterwards sm.rule[s] decides every key.
+template <int NS, typename Keys>
+__device__ void vselect(const Keys &keys, const int *k, SelSmem &sm, int tid, int lane, int warp) {
+  // present count, smallest and largest key
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  int mine = 0;
+  keys.each([&](uint32_t key, int) {
+    if (key) { mn = min(mn, key); mx = max(mx, key); ++mine; }
+  });
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; }
+  block_scan((unsigned long long)mine, sm.red, lane, warp);   // its barriers order the resets above
+  if (lane == 0) { atomicMin(&sm.kmin, mn); atomicMax(&sm.kmax, mx); }
+  if (tid < 256 * NS) (&sm.hist[0][0])[tid] = 0u;
+  if (tid < NS) {
+    const int present = (int)sm.red[kW - 1];
+    sm.done[tid] = present <= k[tid];
+    sm.rule[tid].kthr = 0u;        // take every present key
+    sm.rule[tid].cthr = 0;
+    sm.rule[tid].take_eq = 0;
+    sm.rule[tid].cmode = 0;
+    sm.fallback[tid] = 0;
+    sm.n_coll[tid] = 0;
+    if (tid == 0) sm.n_present = present;
+  }
+  __syncthreads();
+  if (sm.done[0] && (NS == 1 || sm.done[1])) return;
+  const float vlo = kval(sm.kmin), span = kval(sm.kmax) - vlo;
+  const float inv = 256.0f / span;
+  const bool ok = span > 0.f && isfinite(span) && isfinite(inv);
+  if (ok) {   // value-bin histogram
+    keys.each([&](uint32_t key, int) {
+      if (key) {
+        const int bb = vbin(key, vlo, inv);
+#pragma unroll
+        for (int s = 0; s < NS; ++s)
+          if (!sm.done[s]) atomicAdd(&sm.hist[s][bb], 1u);
+      }
+    });
+  }
+  __syncthreads();
+  if (warp < NS && !sm.done[warp]) {   // warp s: the value bin holding the k-th largest key
+    const int s = warp;
+    if (!ok) {
+      if (lane == 0) sm.fallback[s] = 1;
+    } else {
+      uint32_t v[8], lsum = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { v[i] = sm.hist[s][255 - 8 * lane - i]; lsum += v[i]; }
+      uint32_t cum = lsum;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, cum, o);
+        if (lane >= o) cum += y;
+      }
+      const int need = k[s];
+      const uint32_t before = cum - lsum;
+      if ((int)before < need && (int)cum >= need) {
+        uint32_t acc = before;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if ((int)(acc + v[i]) >= need) {
+            sm.T[s] = 255 - 8 * lane - i;
+            sm.cnt[s] = (int)v[i];
+            sm.need[s] = need - (int)acc;   // 1 <= need <= cnt
+            sm.fallback[s] = (int)v[i] > kColl;
+            break;
+          }
+          acc += v[i];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // collect the threshold bin's (key, column) pairs
+  if (ok) {
+    keys.each([&](uint32_t key, int i) {
+      if (key) {
+        const int bb = vbin(key, vlo, inv);
+#pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          if (!sm.done[s] && !sm.fallback[s] && bb == sm.T[s]) {
+            const int slot = atomicAdd(&sm.n_coll[s], 1);
+            sm.coll[s][slot] = make_uint2(key, (uint32_t)keys.col(i));
+          }
+        }
+      }
+    });
+  }
+  __syncthreads();
+  // rank them exactly (key desc, column asc); the need-th one sets the rule
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    if (sm.done[s] || sm.fallback[s]) continue;
+    const int n = sm.n_coll[s];
+    for (int i = tid; i < n; i += kT) {
+      const uint2 me = sm.coll[s][i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) {
+        const uint2 o = sm.coll[s][j];
+        rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+      }
+      if (rank == sm.need[s] - 1) {   // exactly one pair
+        sm.rule[s].kthr = me.x;
+        sm.rule[s].cthr = (int)me.y;
+        sm.rule[s].take_eq = 0;
+        sm.rule[s].cmode = 1;
+      }
+    }
+  }
+  __syncthreads();
+  // rare: a bin too large to rank (or no usable value range) -> key-bit radix
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    if (sm.done[s] || !sm.fallback[s]) continue;   // block-uniform
+    const int kk[1] = {k[s]};
+    SelRule keep[2] = {sm.rule[0], sm.rule[1]};
+    radix_select<1>(keys, kk, sm, tid, lane, warp);
+    const SelRule r = sm.rule[0];
+    __syncthreads();
+    if (tid == 0) {
+      sm.rule[0] = keep[0];
+      sm.rule[1] = keep[1];
+      sm.rule[s] = r;
+    }
+    __syncthreads();
+  }
 }
 
 }  // namespace
@@ -250,50 +424,43 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
     }
     bkey[i] = skey(v.x); bkey[i + 1] = skey(v.y); bkey[i + 2] = skey(v.z); bkey[i + 3] = skey(v.w);
   }
-  const RegKeys<kBpt> bk{bkey};
+  const RegKeys<kBpt> bk{bkey, tid};
 
   // ---- pool (selection 1, when asked) and tau (selection 0)
   const int ks[2] = {a.K, a.P_out};
-  if (a.P_out > 0) radix_select<2>(bk, ks, sh.sel, tid, lane, warp);
-  else radix_select<1>(bk, ks, sh.sel, tid, lane, warp);
+  if (a.P_out > 0) vselect<2>(bk, ks, sh.sel, tid, lane, warp);
+  else vselect<1>(bk, ks, sh.sel, tid, lane, warp);
   const SelRule tau = sh.sel.rule[0];
+  const bool few_blocks = sh.sel.n_present <= a.K;   // every present block is a candidate
   if (a.P_out > 0) {
     const SelRule pr = sh.sel.rule[1];
     const int n_pool = min(sh.sel.n_present, a.P_out);
-    int pos, tb;
-    taken_offsets(bk, pr, sh.sel.red, lane, warp, pos, tb);
     int32_t *op = a.out_pool + (size_t)row * a.P_out;
-#pragma unroll
-    for (int i = 0; i < kBpt; ++i) {
-      const uint32_t key = bkey[i];
-      const bool tk = strictly_taken(key, pr) || (tie(key, pr) && tb < pr.take_eq);
-      tb += tie(key, pr);
-      if (tk) {
-        if (pos < a.P_out) {
-          op[pos] = tid * kBpt + i;
-          if (a.out_pool_scores) a.out_pool_scores[(size_t)row * a.P_out + pos] = kval(key);
-        }
-        ++pos;
+    float *ops = a.out_pool_scores ? a.out_pool_scores + (size_t)row * a.P_out : nullptr;
+    for_taken(bk, pr, sh.sel.red, lane, warp, [&](uint32_t key, int i, int pos) {
+      if (pos < a.P_out) {
+        op[pos] = tid * kBpt + i;
+        if (ops) ops[pos] = kval(key);
       }
-    }
+    });
     for (int i = n_pool + tid; i < a.P_out; i += kT) {
       op[i] = -1;
-      if (a.out_pool_scores) a.out_pool_scores[(size_t)row * a.P_out + i] = -INFINITY;
+      if (ops) ops[i] = -INFINITY;
     }
   }
 
-  // ---- candidate blocks: maximum >= tau (every block when fewer than K are present)
-  const uint32_t tkey = sh.sel.n_present <= a.K ? 1u : tau.kthr;
+  // ---- candidate blocks: maximum >= tau (every present block when fewer than K)
+  const uint32_t tkey = few_blocks ? 1u : tau.kthr;
   int mine = 0;
 #pragma unroll
   for (int i = 0; i < kBpt; ++i) mine += bkey[i] != 0u && bkey[i] >= tkey;
   const int cb0 = (int)block_scan((unsigned long long)mine, sh.sel.red, lane, warp);
   const int n_cb = (int)sh.sel.red[kW - 1];
-  int K_take = a.K;
-  SelRule rule;
+  int K_take;
+  float *osc = a.out_scores ? a.out_scores + (size_t)row * a.K : nullptr;
   if (n_cb * 8 <= kCap) {
-    // gather the candidate blocks' scores in column order; entries below tau
-    // (or beyond the row) are absent
+    // gather the candidate blocks' scores in column order; entries below
+    // tau (or beyond the row) cannot be selected
     int slot = cb0 * 8;
 #pragma unroll
     for (int i = 0; i < kBpt; ++i) {
@@ -316,48 +483,32 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
     uint32_t ck[kCpt];
 #pragma unroll
     for (int i = 0; i < kCpt; ++i) ck[i] = sh.cand_key[tid * kCpt + i];
-    const RegKeys<kCpt> cks{ck};
-    radix_select<1>(cks, ks, sh.sel, tid, lane, warp);
-    rule = sh.sel.rule[0];
+    const RegKeys<kCpt> cks{ck, tid};   // candidate positions ascend with the column
+    vselect<1>(cks, ks, sh.sel, tid, lane, warp);
+    const SelRule rule = sh.sel.rule[0];
     K_take = min(sh.sel.n_present, a.K);
-    int pos, tb;
-    taken_offsets(cks, rule, sh.sel.red, lane, warp, pos, tb);
-#pragma unroll
-    for (int i = 0; i < kCpt; ++i) {
-      const uint32_t key = ck[i];
-      const bool tk = strictly_taken(key, rule) || (tie(key, rule) && tb < rule.take_eq);
-      tb += tie(key, rule);
-      if (tk) {
-        if (pos < a.K) {
-          out[pos] = sh.cand_col[tid * kCpt + i];
-          if (a.out_scores) a.out_scores[(size_t)row * a.K + pos] = kval(key);
-        }
-        ++pos;
+    for_taken(cks, rule, sh.sel.red, lane, warp, [&](uint32_t key, int i, int pos) {
+      if (pos < a.K) {
+        out[pos] = sh.cand_col[tid * kCpt + i];
+        if (osc) osc[pos] = kval(key);
       }
-    }
+    });
   } else {
     // heavy ties at tau: select over the whole row
     const RowKeys rk{sc, n, (n + kT - 1) / kT, tid};
     radix_select<1>(rk, ks, sh.sel, tid, lane, warp);
-    rule = sh.sel.rule[0];
+    const SelRule rule = sh.sel.rule[0];
     K_take = min(sh.sel.n_present, a.K);
-    int pos, tb;
-    taken_offsets(rk, rule, sh.sel.red, lane, warp, pos, tb);
-    rk.each([&](uint32_t key, int i) {
-      const bool tk = strictly_taken(key, rule) || (tie(key, rule) && tb < rule.take_eq);
-      tb += tie(key, rule);
-      if (tk) {
-        if (pos < a.K) {
-          out[pos] = tid * rk.npt + i;
-          if (a.out_scores) a.out_scores[(size_t)row * a.K + pos] = kval(key);
-        }
-        ++pos;
+    for_taken(rk, rule, sh.sel.red, lane, warp, [&](uint32_t key, int i, int pos) {
+      if (pos < a.K) {
+        out[pos] = rk.col(i);
+        if (osc) osc[pos] = kval(key);
       }
     });
   }
   for (int i = K_take + tid; i < a.K; i += kT) {
     out[i] = -1;
-    if (a.out_scores) a.out_scores[(size_t)row * a.K + i] = -INFINITY;
+    if (osc) osc[i] = -INFINITY;
   }
 }
 
@@ -393,34 +544,29 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkMergeArgs a
       }
     }
   }
-  const RegKeys<kBpt> ks{key};
+  const RegKeys<kBpt> ks{key, tid};
   const int k[1] = {a.K};
-  radix_select<1>(ks, k, sel, tid, lane, warp);
+  vselect<1>(ks, k, sel, tid, lane, warp);
   const SelRule rule = sel.rule[0];
   const int K_take = min(sel.n_present, a.K);
-  int pos, tb;
-  taken_offsets(ks, rule, sel.red, lane, warp, pos, tb);
   int32_t *out = a.out_ids + (size_t)row * a.K;
-#pragma unroll
-  for (int i = 0; i < kBpt; ++i) {
-    const bool tk = strictly_taken(key[i], rule) || (tie(key[i], rule) && tb < rule.take_eq);
-    tb += tie(key[i], rule);
-    if (tk) {
-      if (pos < a.K) {
-        out[pos] = gid[i];
-        if (a.out_scores) a.out_scores[(size_t)row * a.K + pos] = kval(key[i]);
-      }
-      ++pos;
+  float *osc = a.out_scores ? a.out_scores + (size_t)row * a.K : nullptr;
+  for_taken(ks, rule, sel.red, lane, warp, [&](uint32_t kk, int i, int pos) {
+    if (pos < a.K) {
+      out[pos] = gid[i];
+      if (osc) osc[pos] = kval(kk);
     }
-  }
+  });
   for (int i = K_take + tid; i < a.K; i += kT) {
     out[i] = -1;
-    if (a.out_scores) a.out_scores[(size_t)row * a.K + i] = -INFINITY;
+    if (osc) osc[i] = -INFINITY;
   }
 }
 
 cudaError_t launch_topk_merge(const TopkMergeArgs &a, cudaStream_t s) {
   const size_t smem = sizeof(SelSmem);
+  cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
   return launch_pdl(topk_merge_kernel, dim3(a.rows), dim3(kT), smem, s, dim3(1, 1, 1), a);
 }
 
