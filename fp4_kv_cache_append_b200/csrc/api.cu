@@ -228,7 +228,7 @@ static csa2_status append_impl(const csa2_main_cache *main, const uint16_t *kv, 
     a.cap = main->cap; a.dI = main->d_I; a.m = main->m;
     a.kv = kv; a.gate = gate; a.w_ik = w_ik;
     const int max_new = T == 0 ? 0 : (main->m == 1 ? T : T / 2 + 1);   // upper bound of complete entries
-    a.entries_per_block = max_new >= 64 ? 8 : 1;
+    a.entries_per_block = max_new >= 256 ? 32 : (max_new >= 64 ? 8 : 1);
     a.main_blocks_per_seq = (max_new + a.entries_per_block - 1) / a.entries_per_block;
   }
   if (!main) a.entries_per_block = 1;
@@ -306,8 +306,8 @@ csa2_status csa2_append_project(const csa2_main_cache *main, const uint16_t *h, 
   a.codes = main->codes; a.scales = main->scales; a.ik = main->ik; a.ik_scale = main->ik_scale;
   a.n_entries = main->n_entries; a.B = main->B; a.cap = main->cap; a.D = main->D; a.dI = main->d_I; a.m = 1;
   a.w_ik = w_ik; a.pos0 = pos0; a.T = T; a.status = d->status;
-  a.entries_per_block = 8;
-  a.main_blocks_per_seq = (T + 7) / 8;
+  a.entries_per_block = T >= 256 ? 32 : 8;
+  a.main_blocks_per_seq = (T + a.entries_per_block - 1) / a.entries_per_block;
   e = launch_append_keys(a, s);
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "key projection launch");
 }

@@ -54,19 +54,21 @@ __device__ __forceinline__ float pool_pair(float ka, float kb, float za, float z
   return __fadd_rn(__fmul_rn(wa, ka), __fmul_rn(wb, kb));
 }
 
-// Indexer keys of entries e0 .. e0+count-1 (count <= 8) of sequence b from
-// their dequantised values xh [count][D] (shared memory), with W_ik staged in
-// shared memory as ws [D][dI]: k_i = sum_c x^_c W[c][i] as ONE fused
-// multiply-add chain per output, channels in ascending order from +0; then
-// per entry s_k = amax/448 and E4M3 codes of k/s_k.  Thread t owns output
-// i = t % dI of entries t / dI, t / dI + slots, ... (slots = blockDim / dI);
-// its chains share every W_ik element it reads.  Ends with the block's
-// threads past one barrier; every thread of the block must call it.
+// Indexer keys of entries e0 .. e0+count-1 (count <= kMaxEntries) of
+// sequence b from their dequantised values xh [count][D] (shared memory),
+// with W_ik staged in shared memory as ws [D][dI]: k_i = sum_c x^_c W[c][i]
+// as ONE fused multiply-add chain per output, channels in ascending order
+// from +0; then per entry s_k = amax/448 and E4M3 codes of k/s_k.  Thread t
+// owns output i = t % dI of entries t / dI + k * slots (slots = blockDim /
+// dI, k < kChains): its chains run side by side, share every W_ik element it
+// reads and take 4 channels of an entry per 16-byte load.  Every thread of
+// the block must call it.
+constexpr int kMaxEntries = 32;
 __device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const float *xh, float *kbuf,
                            const uint16_t *ws) {
   const int t = threadIdx.x, D = a.D, dI = a.dI;
   {
-    constexpr int kChains = 2;   // 8 entries over 4 (dI = 128) or 8 (dI = 64) slots of 512 threads
+    constexpr int kChains = 8;   // 32 entries over 4 (dI = 128) slots of 512 threads; dI = 64 uses 4 of them
     const int slots = (int)blockDim.x / dI;
     const int i = t % dI, s0 = t / dI;
     float acc[kChains];
@@ -74,13 +76,21 @@ __device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const 
     for (int k = 0; k < kChains; ++k) acc[k] = 0.0f;
     if (s0 < count) {
       const uint16_t *wcol = ws + i;
-#pragma unroll 8
-      for (int c = 0; c < D; ++c) {
-        const float wv = bf16_to_f32(wcol[c * dI]);
+#pragma unroll 2
+      for (int c = 0; c < D; c += 4) {
+        const float w0 = bf16_to_f32(wcol[c * dI]), w1 = bf16_to_f32(wcol[(c + 1) * dI]);
+        const float w2 = bf16_to_f32(wcol[(c + 2) * dI]), w3 = bf16_to_f32(wcol[(c + 3) * dI]);
 #pragma unroll
         for (int k = 0; k < kChains; ++k) {
           const int jj = s0 + k * slots;
-          if (jj < count) acc[k] = __fmaf_rn(xh[jj * D + c], wv, acc[k]);
+          if (jj < count) {
+            const float4 x = *reinterpret_cast<const float4 *>(xh + jj * D + c);
+            float v = acc[k];
+            v = __fmaf_rn(x.x, w0, v);
+            v = __fmaf_rn(x.y, w1, v);
+            v = __fmaf_rn(x.z, w2, v);
+            acc[k] = __fmaf_rn(x.w, w3, v);
+          }
         }
       }
 #pragma unroll
@@ -91,10 +101,10 @@ __device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const 
     }
   }
   __syncthreads();
-  // ---- FP8 key per entry: warp jj takes entry jj
-  const int warp = t >> 5, lane = t & 31;
-  if (warp < count) {
-    const int jj = warp, e = e0 + jj;
+  // ---- FP8 key per entry: warp w takes entries w, w + warps, ...
+  const int warp = t >> 5, lane = t & 31, nw = (int)blockDim.x >> 5;
+  for (int jj = warp; jj < count; jj += nw) {
+    const int e = e0 + jj;
     float kmax = 0.0f;
     for (int i = lane; i < dI; i += 32) kmax = fmaxf(kmax, fabsf(kbuf[jj * dI + i]));
     for (int o = 16; o > 0; o >>= 1) kmax = fmaxf(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
@@ -108,7 +118,7 @@ __device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const 
   }
 }
 
-// Entries j0 .. j0+count-1 (count <= kEntriesPerBlock) of sequence b.  The
+// Entries j0 .. j0+count-1 (count <= entries_per_block <= kMaxEntries) of sequence b.  The
 // projection reads each W_ik element once for all of the block's entries.
 __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   const int t = threadIdx.x;

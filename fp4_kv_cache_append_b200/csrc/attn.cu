@@ -20,7 +20,8 @@
 //               once P is written, O^T += V^T P^T per 128-channel block (V^T
 //               is the same K^ tile read MN-major) and the row sums
 //               L += 1 P^T with an all-ones A operand held in TMEM
-//   warps 8-11  softmax: thread = key (TMEM lane), 64 head logits; the
+//   warps 8-11  first Q (bf16 -> fp16 B operand) while the gather warps load
+//               the first tile, then softmax: thread = key (TMEM lane), 64 head logits; the
 //               reference max of a head moves only when a tile raises it by
 //               more than 2^8 (O^T and L are then rescaled in TMEM), so P =
 //               2^(s - m) stays within fp16 range; P is written as the MN-
@@ -71,7 +72,7 @@ struct AttnSmem {
   float m_ref[kHeads], alpha[kHeads], lsum[kHeads];
   float red[4][kHeads];
   float wgt[8][kHeads];                               // merge weights of the splits
-  uint64_t chunk_full[D / 64], o_done[D / 128], s_full, p_full, fin;
+  uint64_t chunk_full[D / 64], o_done[D / 128], s_full, p_full, fin, q_ready;
   uint32_t tmem_base;
   int abort;
   int rescale_at;                                     // tile whose softmax moved a reference max
@@ -167,7 +168,7 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   constexpr int NCH = D / 64;                      // 64-channel chunks of a tile
   constexpr int MT = D / 128;                      // O^T TMEM blocks of 128 channels
-  constexpr int QI = kHeads * (D / 8) / kDq;       // 16-byte pieces of Q per dequantise thread
+  constexpr int QI2 = kHeads * (D / 8) / 128;      // 16-byte pieces of Q per softmax thread
   constexpr uint32_t kIdS = mma_idesc(128, kHeads, 0u /*f16*/, 0u /*f16*/);
   constexpr uint32_t kIdO = kIdS | (1u << 15) | (1u << 16);   // A (V^T) and B (P^T) MN-major
   constexpr uint32_t kIdL = kIdS | (1u << 16);                // A (ones, TMEM) K-major, B (P^T) MN-major
@@ -189,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     mbar_init(&S.s_full, 1);
     mbar_init(&S.p_full, 4);
     mbar_init(&S.fin, 1);
+    mbar_init(&S.q_ready, 4);
     S.abort = 0;
     S.rescale_at = -1;
     fence_barrier_init();
@@ -229,30 +231,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   if (warp < kDqWarps) {
     // ================================================ gather + dequantise
     const int r = tid >> 1, hf = tid & 1;   // key slot, 32-channel half of each chunk
-    // Q: bf16 -> fp16 into the B-operand layout (before chunk 0 of the first tile)
-    if (n_tiles > 0) {
-      const uint16_t *qrow = a.q + (size_t)row * a.H * D;
-      uint4 qraw[QI];
-#pragma unroll
-      for (int u = 0; u < QI; ++u) {
-        const int i = tid + u * kDq;
-        const int h = i / (D / 8), pc = i % (D / 8);
-        qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (int u = 0; u < QI; ++u) {
-        const int i = tid + u * kDq;
-        const int h = i / (D / 8), pc = i % (D / 8);
-        const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
-        uint32_t o[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
-          o[k] = *reinterpret_cast<const uint32_t *>(&hv);
-        }
-        *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
-      }
-    }
     int id = n_tiles > 0 ? key_id(a, row, c_begin, n_fp4_tiles, wlo, nwin, r) : -1;
 #pragma unroll 1
     for (int it = 0; it < n_tiles; ++it) {
@@ -345,6 +323,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     const int r = 32 * q + lane;            // key slot = TMEM lane
     const int st = tid - kSmWarp0 * 32;     // 0..127
     const uint32_t srow = tmem + ((uint32_t)(32 * q) << 16);
+    // Q: bf16 -> fp16 into the B-operand layout, while the gather warps load
+    // the first tile's keys (the MMA issuer waits for q_ready)
+    if (n_tiles > 0) {
+      const uint16_t *qrow = a.q + (size_t)row * a.H * D;
+#pragma unroll 1
+      for (int u0 = 0; u0 < QI2; u0 += 16) {
+        uint4 qraw[16];
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const int i = st + (u0 + u) * 128;
+          const int h = i / (D / 8), pc = i % (D / 8);
+          qraw[u] = (u0 + u < QI2 && h < a.H) ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8))
+                                              : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if (u0 + u >= QI2) break;
+          const int i = st + (u0 + u) * 128;
+          const int h = i / (D / 8), pc = i % (D / 8);
+          const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
+            o[k] = *reinterpret_cast<const uint32_t *>(&hv);
+          }
+          *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.q_ready);
+    }
 #pragma unroll 1
     for (int it = 0; it < n_tiles; ++it) {
       const int c = c_begin + it;
@@ -471,7 +482,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     const uint64_t dq0 = smem_desc_kmajor(q_base, 128), dk0 = smem_desc_kmajor(kh_base, 128);
     const uint64_t dv0 = smem_desc_mnmajor_sw128(kh_base, kTile * 128, 1024);
     const uint64_t dp0 = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
-    bool ok = true;
+    bool ok = n_tiles == 0 || wait_or_abort(&S.q_ready, 0, abort);
 #pragma unroll 1
     for (int it = 0; it < n_tiles && ok; ++it) {
       // S^T = K^ Q^T, chunk by chunk as the chunks land

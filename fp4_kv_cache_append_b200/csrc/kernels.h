@@ -38,7 +38,7 @@ struct AppendArgs {
   const int32_t *pos0;
   int T;
   int main_blocks_per_seq, swa_blocks_per_seq;
-  int entries_per_block;   // 1 .. 8
+  int entries_per_block;   // 1, 8 or 32
   unsigned int *status;
   QueryPrep prep;          // optional: the following scan's query, 8 blocks per row
 };
