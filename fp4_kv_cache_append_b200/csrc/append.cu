@@ -54,7 +54,7 @@ __device__ __forceinline__ float pool_pair(float ka, float kb, float za, float z
   return __fadd_rn(__fmul_rn(wa, ka), __fmul_rn(wb, kb));
 }
 
-// Indexer keys of entries e0 .. e0+count-1 (count <= kMaxEntries) of
+// Indexer keys of entries e0 .. e0+count-1 (count <= 32) of
 // sequence b from their dequantised values xh [count][D] (shared memory),
 // with W_ik staged in shared memory as ws [D][dI]: k_i = sum_c x^_c W[c][i]
 // as ONE fused multiply-add chain per output, channels in ascending order
@@ -63,7 +63,6 @@ __device__ __forceinline__ float pool_pair(float ka, float kb, float za, float z
 // dI, k < kChains): its chains run side by side, share every W_ik element it
 // reads and take 4 channels of an entry per 16-byte load.  Every thread of
 // the block must call it.
-constexpr int kMaxEntries = 32;
 __device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const float *xh, float *kbuf,
                            const uint16_t *ws) {
   const int t = threadIdx.x, D = a.D, dI = a.dI;
@@ -118,7 +117,7 @@ __device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const 
   }
 }
 
-// Entries j0 .. j0+count-1 (count <= entries_per_block <= kMaxEntries) of sequence b.  The
+// Entries j0 .. j0+count-1 (count <= entries_per_block <= 32) of sequence b.  The
 // projection reads each W_ik element once for all of the block's entries.
 __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
   const int t = threadIdx.x;

@@ -84,22 +84,6 @@ __device__ __forceinline__ uint32_t sw_off(int r, int pc, int rows) {
   return (uint32_t)((pc >> 3) * rows * 128 + r * 128 + (((pc & 7) ^ (r & 7)) << 4));
 }
 
-// After the call, lane l holds in t[0] the sum over the warp of column l.
-__device__ __forceinline__ void reduce_scatter32(float *t, int lane) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    const bool up = (lane & o) != 0;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      if (j < o) {
-        const float lo = t[j], hi = t[j + o];
-        const float recv = __shfl_xor_sync(0xffffffffu, up ? lo : hi, o);
-        t[j] = (up ? hi : lo) + recv;
-      }
-    }
-  }
-}
-
 // After the call, lane l holds in t[0] the maximum over the warp of column l
 // (the same transposing butterfly; t is consumed).
 __device__ __forceinline__ void reduce_scatter32_max(float *t, int lane) {
@@ -165,10 +149,13 @@ __device__ __forceinline__ int key_id(const AttnArgs &a, int row, int c, int n_f
 }  // namespace
 
 template <int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
+__global__ void __maxnreg__(152) attn_kernel(const AttnArgs a) {
   constexpr int NCH = D / 64;                      // 64-channel chunks of a tile
   constexpr int MT = D / 128;                      // O^T TMEM blocks of 128 channels
-  constexpr int QI2 = kHeads * (D / 8) / 128;      // 16-byte pieces of Q per softmax thread
+  constexpr int QP = kHeads * (D / 8);             // 16-byte pieces of Q
+  constexpr int QS = QP / 2;                       // the softmax warps convert pieces [0, QS)
+  constexpr int QI2 = QS / 128;                    // ... QI2 per softmax thread
+  constexpr int QD = (QP - QS) / kDq;              // the gather warps pieces [QS, QP), QD each
   constexpr uint32_t kIdS = mma_idesc(128, kHeads, 0u /*f16*/, 0u /*f16*/);
   constexpr uint32_t kIdO = kIdS | (1u << 15) | (1u << 16);   // A (V^T) and B (P^T) MN-major
   constexpr uint32_t kIdL = kIdS | (1u << 16);                // A (ones, TMEM) K-major, B (P^T) MN-major
@@ -190,7 +177,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     mbar_init(&S.s_full, 1);
     mbar_init(&S.p_full, 4);
     mbar_init(&S.fin, 1);
-    mbar_init(&S.q_ready, 4);
+    mbar_init(&S.q_ready, 4 + kDqWarps);
     S.abort = 0;
     S.rescale_at = -1;
     fence_barrier_init();
@@ -232,6 +219,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
     // ================================================ gather + dequantise
     const int r = tid >> 1, hf = tid & 1;   // key slot, 32-channel half of each chunk
     int id = n_tiles > 0 ? key_id(a, row, c_begin, n_fp4_tiles, wlo, nwin, r) : -1;
+    // the second half of Q (the softmax warps convert the first half)
+    uint4 qraw[QD];
+    const uint16_t *qrow = a.q + (size_t)row * a.H * D;
+    if (n_tiles > 0) {
+#pragma unroll
+      for (int u = 0; u < QD; ++u) {
+        const int i = QS + tid + u * kDq;
+        const int h = i / (D / 8), pc = i % (D / 8);
+        qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
+      }
+    }
 #pragma unroll 1
     for (int it = 0; it < n_tiles; ++it) {
       const int c = c_begin + it;
@@ -257,20 +255,41 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
           raw[2 * k + 1] = id >= 0 ? __ldg(wp + 4 * k + 1) : make_uint4(0, 0, 0, 0);
         }
       }
-      // the next tile's key and an L2 prefetch of its bytes
-      int id_next = -1;
-      if (it + 1 < n_tiles) {
-        id_next = key_id(a, row, c + 1, n_fp4_tiles, wlo, nwin, r);
-        if (id_next >= 0) {
-          if (c + 1 < n_fp4_tiles) {
-            const size_t er = (size_t)b * a.cap + id_next;
+      if (it == 0) {
+        // the block's later tiles (up to 8) are asked into L2 while this
+        // tile's loads are in flight: their register loads then find them there
+#pragma unroll 1
+        for (int c2 = c + 1; c2 < c_end && c2 < c + 8; ++c2) {
+          const int i2 = key_id(a, row, c2, n_fp4_tiles, wlo, nwin, r);
+          if (i2 < 0) continue;
+          if (c2 < n_fp4_tiles) {
+            const size_t er = (size_t)b * a.cap + i2;
             prefetch_l2(a.codes + er * (D / 2) + hf * (D / 4));
             if (hf == 0) prefetch_l2(a.scales + er * (D / 16));
           } else {
-            prefetch_l2(a.swa_rows + ((size_t)b * a.W_cap + id_next) * D + hf * (D / 2));
+            prefetch_l2(a.swa_rows + ((size_t)b * a.W_cap + i2) * D + hf * (D / 2));
           }
         }
+        // the second half of Q -> fp16 B operand
+#pragma unroll
+        for (int u = 0; u < QD; ++u) {
+          const int i = QS + tid + u * kDq;
+          const int h = i / (D / 8), pc = i % (D / 8);
+          const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+          uint32_t o[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
+            o[k] = *reinterpret_cast<const uint32_t *>(&hv);
+          }
+          *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&S.q_ready);
       }
+      // the next tile's key
+      const int id_next = it + 1 < n_tiles ? key_id(a, row, c + 1, n_fp4_tiles, wlo, nwin, r) : -1;
       bool ok = true;
 #pragma unroll
       for (int k = 0; k < NCH; ++k) {
@@ -553,9 +572,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
         for (int j = 0; j < 32; ++j) S.lsum[32 * half + j] = __uint_as_float(lv[j]);
       }
     }
-    // O / l per head.  One split: bf16, staged head-major [64 heads][D] in
-    // the K^ tile (free once the last O^T MMA completed), then written out in
-    // 16-byte pieces.  Several splits: fp16 partials straight from registers.
+    // O / l per head, staged head-major [64 heads][D] in the K^ tile (free
+    // once the last O^T MMA completed) -- bf16 for one split, fp16 partials
+    // for several -- then written out in 16-byte pieces.
     uint16_t *ob = reinterpret_cast<uint16_t *>(S.kh);
 #pragma unroll 1
     for (int mt = mt_lo; mt < mt_hi; ++mt) {
@@ -575,9 +594,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
           ob[(32 * half + j) * D + ch] = *reinterpret_cast<const uint16_t *>(&bv);
         }
       } else {
-        __half *po = reinterpret_cast<__half *>(a.ws) + ((size_t)row * a.nsplit + split) * kHeads * D + ch;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) po[(size_t)(32 * half + j) * D] = __float2half_rn(__uint_as_float(o[j]) * linv[j]);
+        for (int j = 0; j < 32; ++j) {
+          const __half hv = __float2half_rn(__uint_as_float(o[j]) * linv[j]);
+          ob[(32 * half + j) * D + ch] = *reinterpret_cast<const uint16_t *>(&hv);
+        }
       }
     }
   }
@@ -589,11 +610,24 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       const int n16 = a.H * (D / 8);
 #pragma unroll 4
       for (int i = tid; i < n16; i += kThreads) dst[i] = src[i];
-    } else if (tid < kHeads) {
-      float *pm = partial_stats(a, nrows) + ((size_t)row * a.nsplit + split) * kHeads;
-      float *pl = pm + nrows * a.nsplit * kHeads;
-      pm[tid] = S.m_ref[tid];
-      pl[tid] = S.lsum[tid];
+    } else {
+      // this block's channels [z_lo, z_lo + D / csplit) of every head
+      const int Dz = D / a.csplit, z_lo = mt_lo * 128;
+      const uint4 *src = reinterpret_cast<const uint4 *>(S.kh);
+      uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__half *>(a.ws) +
+                                             ((size_t)row * a.nsplit + split) * kHeads * D);
+      const int per = Dz / 8, n16 = kHeads * per;
+#pragma unroll 4
+      for (int i = tid; i < n16; i += kThreads) {
+        const int h = i / per, pc = z_lo / 8 + i % per;
+        dst[h * (D / 8) + pc] = src[h * (D / 8) + pc];
+      }
+      if (tid < kHeads) {
+        float *pm = partial_stats(a, nrows) + ((size_t)row * a.nsplit + split) * kHeads;
+        float *pl = pm + nrows * a.nsplit * kHeads;
+        pm[tid] = S.m_ref[tid];
+        pl[tid] = S.lsum[tid];
+      }
     }
   }
   tc_fence_before();
@@ -606,6 +640,28 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   // ---- merge of the splits (the row's blocks form one cluster)
   if (a.nsplit > 1) {
     cluster_sync_all();   // every split's partials are written
+    // this split's channel slice; item = (head, 8 channels): 16 bytes per split in, 16 bytes out
+    const int Dz = D / a.csplit, z_lo = (int)blockIdx.z * Dz;   // this block's channel half (or all)
+    const int cs = ((Dz / a.nsplit) + 7) / 8 * 8;
+    const int c_lo = z_lo + split * cs;
+    const int c_hi = c_lo + cs < z_lo + Dz ? c_lo + cs : z_lo + Dz;
+    const int ng = c_hi > c_lo ? (c_hi - c_lo) / 8 : 0;
+    const int n_items = a.H * ng;
+    const __half *base = reinterpret_cast<const __half *>(a.ws) + (size_t)row * a.nsplit * kHeads * D;
+    uint4 x[kMergeItems][8];
+    auto load_items = [&](int it0) {   // kMergeItems items' loads in flight
+#pragma unroll
+      for (int v = 0; v < kMergeItems; ++v) {
+        const int it = it0 + v * kThreads;
+        const int h = it / (ng > 0 ? ng : 1), ch = c_lo + 8 * (it % (ng > 0 ? ng : 1));
+#pragma unroll
+        for (int s = 0; s < 8; ++s)
+          x[v][s] = (it < n_items && s < a.nsplit)
+                        ? __ldcg(reinterpret_cast<const uint4 *>(base + ((size_t)s * kHeads + h) * D + ch))
+                        : make_uint4(0, 0, 0, 0);
+      }
+    };
+    load_items(tid);   // the first round of partials is in flight with the statistics
     const float *pm = partial_stats(a, nrows) + (size_t)row * a.nsplit * kHeads;
     const float *pl = pm + nrows * a.nsplit * kHeads;
     if (tid < kHeads) {   // all 2 x nsplit loads in flight together
@@ -629,27 +685,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       for (int s = 0; s < 8; ++s) S.wgt[s][tid] = ms[s] * inv;
     }
     __syncthreads();
-    // this split's channel slice; item = (head, 8 channels): 16 bytes per split in, 16 bytes out
-    const int Dz = D / a.csplit, z_lo = (int)blockIdx.z * Dz;   // this block's channel half (or all)
-    const int cs = ((Dz / a.nsplit) + 7) / 8 * 8;
-    const int c_lo = z_lo + split * cs;
-    const int c_hi = c_lo + cs < z_lo + Dz ? c_lo + cs : z_lo + Dz;
-    const int ng = c_hi > c_lo ? (c_hi - c_lo) / 8 : 0;
-    const int n_items = a.H * ng;
-    const __half *base = reinterpret_cast<const __half *>(a.ws) + (size_t)row * a.nsplit * kHeads * D;
 #pragma unroll 1
-    for (int it0 = tid; it0 < n_items; it0 += kMergeItems * kThreads) {   // kMergeItems items' loads in flight
-      uint4 x[kMergeItems][8];
-#pragma unroll
-      for (int v = 0; v < kMergeItems; ++v) {
-        const int it = it0 + v * kThreads;
-        const int h = it / ng, ch = c_lo + 8 * (it % ng);
-#pragma unroll
-        for (int s = 0; s < 8; ++s)
-          x[v][s] = (it < n_items && s < a.nsplit)
-                        ? __ldcg(reinterpret_cast<const uint4 *>(base + ((size_t)s * kHeads + h) * D + ch))
-                        : make_uint4(0, 0, 0, 0);
-      }
+    for (int it0 = tid; it0 < n_items; it0 += kMergeItems * kThreads) {
+      if (it0 != tid) load_items(it0);
 #pragma unroll
       for (int v = 0; v < kMergeItems; ++v) {
         const int it = it0 + v * kThreads;

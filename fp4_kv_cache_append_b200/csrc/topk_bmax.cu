@@ -8,8 +8,8 @@
 // non-finite = absent, ascending output, -1 padding; block score = max of
 // its present columns).
 //
-// One 1024-thread block per row.  Thread t holds the keys of blocks
-// 16t .. 16t+15 (order-preserving 32-bit keys of the block maxima, 0 =
+// One 512-thread block per row.  Thread t holds the keys of blocks
+// 32t .. 32t+31 (order-preserving 32-bit keys of the block maxima, 0 =
 // absent).  Two selections run side by side over them:
 //   * the pool: the P_out blocks with the largest maxima;
 //   * tau: the K-th largest block maximum.
@@ -36,9 +36,9 @@ namespace csa2 {
 
 namespace {
 
-constexpr int kT = 1024;
+constexpr int kT = 512;
 constexpr int kW = kT / 32;
-constexpr int kBpt = 16;           // block maxima per thread: rows of up to 16,384 blocks
+constexpr int kBpt = 32;           // block maxima per thread: rows of up to 16,384 blocks
 constexpr int kCap = 8192;         // candidate entries in shared memory
 constexpr int kCpt = kCap / kT;    // candidates per thread
 
@@ -66,7 +66,8 @@ struct SelRule {
 };
 
 struct SelSmem {
-  uint32_t hist[2][256];
+  uint32_t hist[2][256];             // radix rounds
+  uint32_t vhist[256][8];            // value bins, 8 copies per bin (fewer colliding atomics)
   uint32_t prefix[2], mask[2];
   int need[2], done[2];
   SelRule rule[2];
@@ -82,6 +83,7 @@ struct Smem {
   SelSmem sel;
   uint32_t cand_key[kCap];
   int32_t cand_col[kCap];
+  int32_t cand_blk[kCap / 8];        // candidate blocks, ascending
 };
 
 // Exclusive block scan of v; afterwards red[kW-1] holds the block total.
@@ -278,7 +280,7 @@ __device__ void vselect(const Keys &keys, const int *k, SelSmem &sm, int tid, in
   if (tid == 0) { sm.kmin = 0xFFFFFFFFu; sm.kmax = 0u; }
   block_scan((unsigned long long)mine, sm.red, lane, warp);   // its barriers order the resets above
   if (lane == 0) { atomicMin(&sm.kmin, mn); atomicMax(&sm.kmax, mx); }
-  if (tid < 256 * NS) (&sm.hist[0][0])[tid] = 0u;
+  for (int i = tid; i < 256 * 8; i += kT) (&sm.vhist[0][0])[i] = 0u;
   if (tid < NS) {
     const int present = (int)sm.red[kW - 1];
     sm.done[tid] = present <= k[tid];
@@ -295,14 +297,9 @@ __device__ void vselect(const Keys &keys, const int *k, SelSmem &sm, int tid, in
   const float vlo = kval(sm.kmin), span = kval(sm.kmax) - vlo;
   const float inv = 256.0f / span;
   const bool ok = span > 0.f && isfinite(span) && isfinite(inv);
-  if (ok) {   // value-bin histogram
+  if (ok) {   // value-bin histogram (one for every selection)
     keys.each([&](uint32_t key, int) {
-      if (key) {
-        const int bb = vbin(key, vlo, inv);
-#pragma unroll
-        for (int s = 0; s < NS; ++s)
-          if (!sm.done[s]) atomicAdd(&sm.hist[s][bb], 1u);
-      }
+      if (key) atomicAdd(&sm.vhist[vbin(key, vlo, inv)][lane & 7], 1u);
     });
   }
   __syncthreads();
@@ -313,7 +310,12 @@ __device__ void vselect(const Keys &keys, const int *k, SelSmem &sm, int tid, in
     } else {
       uint32_t v[8], lsum = 0;
 #pragma unroll
-      for (int i = 0; i < 8; ++i) { v[i] = sm.hist[s][255 - 8 * lane - i]; lsum += v[i]; }
+      for (int i = 0; i < 8; ++i) {
+        const uint4 c0 = *reinterpret_cast<const uint4 *>(&sm.vhist[255 - 8 * lane - i][0]);
+        const uint4 c1 = *reinterpret_cast<const uint4 *>(&sm.vhist[255 - 8 * lane - i][4]);
+        v[i] = c0.x + c0.y + c0.z + c0.w + c1.x + c1.y + c1.z + c1.w;
+        lsum += v[i];
+      }
       uint32_t cum = lsum;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -410,7 +412,7 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
   const float *sc = a.scores + (size_t)row * a.ld;
   int32_t *out = a.out_idx + (size_t)row * a.K;
 
-  // ---- block-maximum keys, 16 consecutive blocks per thread
+  // ---- block-maximum keys, 32 consecutive blocks per thread
   uint32_t bkey[kBpt];
 #pragma unroll
   for (int i = 0; i < kBpt; i += 4) {
@@ -459,26 +461,26 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
   int K_take;
   float *osc = a.out_scores ? a.out_scores + (size_t)row * a.K : nullptr;
   if (n_cb * 8 <= kCap) {
-    // gather the candidate blocks' scores in column order; entries below
-    // tau (or beyond the row) cannot be selected
-    int slot = cb0 * 8;
+    // the candidate blocks in ascending order, then their scores loaded by
+    // all threads at once (column order); entries below tau (or beyond the
+    // row) cannot be selected
+    int slot = cb0;
 #pragma unroll
-    for (int i = 0; i < kBpt; ++i) {
-      if (bkey[i] != 0u && bkey[i] >= tkey) {
-        const int c0 = (tid * kBpt + i) * 8;
-        const float4 x = __ldcg(reinterpret_cast<const float4 *>(sc + c0));
-        const float4 y = __ldcg(reinterpret_cast<const float4 *>(sc + c0) + 1);
-        const float v[8] = {x.x, x.y, x.z, x.w, y.x, y.y, y.z, y.w};
+    for (int i = 0; i < kBpt; ++i)
+      if (bkey[i] != 0u && bkey[i] >= tkey) sh.cand_blk[slot++] = tid * kBpt + i;
+    __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t key = c0 + j < n ? skey(v[j]) : 0u;
-          sh.cand_key[slot + j] = key >= tkey ? key : 0u;
-          sh.cand_col[slot + j] = c0 + j;
-        }
-        slot += 8;
+    for (int u = 0; u < kCpt; ++u) {
+      const int j = tid + u * kT;
+      uint32_t key = 0u;
+      int col = 0;
+      if (j < n_cb * 8) {
+        col = sh.cand_blk[j >> 3] * 8 + (j & 7);
+        key = col < n ? skey(__ldcg(sc + col)) : 0u;
       }
+      sh.cand_key[j] = key >= tkey ? key : 0u;
+      sh.cand_col[j] = col;
     }
-    for (int i = n_cb * 8 + tid; i < kCap; i += kT) sh.cand_key[i] = 0u;
     __syncthreads();
     uint32_t ck[kCpt];
 #pragma unroll
