@@ -62,7 +62,7 @@ constexpr int kSmBar = 1;                    // named barrier of the softmax war
 // TMEM columns: S^T [0, 64), O^T blocks [64, 64 + 64 MT), L [320, 384), ones [384, 416)
 constexpr uint32_t kColS = 0, kColO = 64, kColL = 320, kColOnes = 384, kTmemCols = 512;
 // Merge items (head, 8 channels) per thread whose loads are in flight together.
-constexpr int kMergeItems = 2;
+constexpr int kMergeItems = 1;
 
 template <int D>
 struct AttnSmem {
@@ -149,7 +149,7 @@ __device__ __forceinline__ int key_id(const AttnArgs &a, int row, int c, int n_f
 }  // namespace
 
 template <int D>
-__global__ void __maxnreg__(152) attn_kernel(const AttnArgs a) {
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
   constexpr int NCH = D / 64;                      // 64-channel chunks of a tile
   constexpr int MT = D / 128;                      // O^T TMEM blocks of 128 channels
   constexpr int QP = kHeads * (D / 8);             // 16-byte pieces of Q
@@ -222,13 +222,29 @@ __global__ void __maxnreg__(152) attn_kernel(const AttnArgs a) {
     // the second half of Q (the softmax warps convert the first half)
     uint4 qraw[QD];
     const uint16_t *qrow = a.q + (size_t)row * a.H * D;
-    if (n_tiles > 0) {
+    if (n_tiles > 0) {   // loaded while the first key ids load, converted before the tile's gather
 #pragma unroll
       for (int u = 0; u < QD; ++u) {
         const int i = QS + tid + u * kDq;
         const int h = i / (D / 8), pc = i % (D / 8);
         qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
       }
+#pragma unroll
+      for (int u = 0; u < QD; ++u) {
+        const int i = QS + tid + u * kDq;
+        const int h = i / (D / 8), pc = i % (D / 8);
+        const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
+          o[k] = *reinterpret_cast<const uint32_t *>(&hv);
+        }
+        *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+      fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.q_ready);
     }
 #pragma unroll 1
     for (int it = 0; it < n_tiles; ++it) {
@@ -270,23 +286,6 @@ __global__ void __maxnreg__(152) attn_kernel(const AttnArgs a) {
             prefetch_l2(a.swa_rows + ((size_t)b * a.W_cap + i2) * D + hf * (D / 2));
           }
         }
-        // the second half of Q -> fp16 B operand
-#pragma unroll
-        for (int u = 0; u < QD; ++u) {
-          const int i = QS + tid + u * kDq;
-          const int h = i / (D / 8), pc = i % (D / 8);
-          const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
-          uint32_t o[4];
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
-            o[k] = *reinterpret_cast<const uint32_t *>(&hv);
-          }
-          *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
-        }
-        fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.q_ready);
       }
       // the next tile's key
       const int id_next = it + 1 < n_tiles ? key_id(a, row, c + 1, n_fp4_tiles, wlo, nwin, r) : -1;
