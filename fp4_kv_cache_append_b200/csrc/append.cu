@@ -143,50 +143,69 @@ __device__ void append_entries(const AppendArgs &a, int b, int j0, float *sm) {
     for (int i = t; i < D * dI / 8; i += blockDim.x) dst[i] = src[i];
   }
 
-  // ---- pool + FP4 per entry (thread t: channels 2t, 2t+1; 8 threads per group)
-  for (int jj = 0; jj < count && t < D / 2; ++jj) {
-    const int e = p0 / m + j0 + jj;
-    float x0, x1;
-    if (m == 1) {
-      const uint32_t v = reinterpret_cast<const uint32_t *>(a.kv + ((size_t)b * a.T + (e - p0)) * D)[t];
-      x0 = bf16_to_f32((uint16_t)(v & 0xFFFFu));
-      x1 = bf16_to_f32((uint16_t)(v >> 16));
-    } else {
-      const int ta = 2 * e - p0;  // -1 only for the block's first entry with p0 odd: the pending token
-      const uint16_t *kva = ta < 0 ? a.pending_kv + (size_t)b * D : a.kv + ((size_t)b * a.T + ta) * D;
-      const uint16_t *za = ta < 0 ? a.pending_gate + (size_t)b * D : a.gate + ((size_t)b * a.T + ta) * D;
-      const uint16_t *kvb = a.kv + ((size_t)b * a.T + ta + 1) * D;
-      const uint16_t *zb = a.gate + ((size_t)b * a.T + ta + 1) * D;
-      const uint32_t ka = reinterpret_cast<const uint32_t *>(kva)[t];
-      const uint32_t kb = reinterpret_cast<const uint32_t *>(kvb)[t];
-      const uint32_t ga = reinterpret_cast<const uint32_t *>(za)[t];
-      const uint32_t gb = reinterpret_cast<const uint32_t *>(zb)[t];
-      x0 = pool_pair(bf16_to_f32(ka & 0xFFFFu), bf16_to_f32(kb & 0xFFFFu), bf16_to_f32(ga & 0xFFFFu),
-                     bf16_to_f32(gb & 0xFFFFu));
-      x1 = pool_pair(bf16_to_f32(ka >> 16), bf16_to_f32(kb >> 16), bf16_to_f32(ga >> 16), bf16_to_f32(gb >> 16));
+  // ---- pool + FP4 per entry: thread t owns channels 2p, 2p+1 (p = t % (D/2),
+  // 8 threads per 16-channel group) of entries t / (D/2) + k * (blockDim /
+  // (D/2)); each round's loads (8 entries) are issued before any is used
+  {
+    const int P2 = D / 2, G2 = (int)blockDim.x / P2, p = t % P2;
+    for (int base = t / P2; base < count; base += 8 * G2) {
+      uint32_t ka[8], kb[8], ga[8], gb[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int jj = base + r * G2;
+        if (jj >= count) break;
+        const int e = p0 / m + j0 + jj;
+        if (m == 1) {
+          ka[r] = reinterpret_cast<const uint32_t *>(a.kv + ((size_t)b * a.T + (e - p0)) * D)[p];
+        } else {
+          const int ta = 2 * e - p0;  // -1 only for the block's first entry with p0 odd: the pending token
+          const uint16_t *kva = ta < 0 ? a.pending_kv + (size_t)b * D : a.kv + ((size_t)b * a.T + ta) * D;
+          const uint16_t *za = ta < 0 ? a.pending_gate + (size_t)b * D : a.gate + ((size_t)b * a.T + ta) * D;
+          ka[r] = reinterpret_cast<const uint32_t *>(kva)[p];
+          kb[r] = reinterpret_cast<const uint32_t *>(a.kv + ((size_t)b * a.T + ta + 1) * D)[p];
+          ga[r] = reinterpret_cast<const uint32_t *>(za)[p];
+          gb[r] = reinterpret_cast<const uint32_t *>(a.gate + ((size_t)b * a.T + ta + 1) * D)[p];
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int jj = base + r * G2;
+        if (jj >= count) break;
+        const int e = p0 / m + j0 + jj;
+        float x0, x1;
+        if (m == 1) {
+          x0 = bf16_to_f32((uint16_t)(ka[r] & 0xFFFFu));
+          x1 = bf16_to_f32((uint16_t)(ka[r] >> 16));
+        } else {
+          x0 = pool_pair(bf16_to_f32(ka[r] & 0xFFFFu), bf16_to_f32(kb[r] & 0xFFFFu), bf16_to_f32(ga[r] & 0xFFFFu),
+                         bf16_to_f32(gb[r] & 0xFFFFu));
+          x1 = pool_pair(bf16_to_f32(ka[r] >> 16), bf16_to_f32(kb[r] >> 16), bf16_to_f32(ga[r] >> 16),
+                         bf16_to_f32(gb[r] >> 16));
+        }
+        float amax = fmaxf(fabsf(x0), fabsf(x1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+        uint32_t sb = amax == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(amax, 6.0f));
+        const float sc = e4m3_to_f32(sb);
+        uint32_t c0 = 0, c1 = 0;
+        if (sc != 0.0f) {
+          c0 = f32_to_e2m1(__fdiv_rn(x0, sc));
+          c1 = f32_to_e2m1(__fdiv_rn(x1, sc));
+        } else {
+          sb = 0;
+        }
+        if (e < a.cap) {
+          const size_t row = (size_t)b * a.cap + e;
+          a.codes[row * (D / 2) + p] = (uint8_t)(c0 | (c1 << 4));
+          if ((p & 7) == 0) a.scales[row * (D / 16) + (p >> 3)] = (uint8_t)sb;
+        } else if (p == 0) {
+          flag(a.status, CSA2_DEV_APPEND_RANGE);
+        }
+        xh[jj * D + 2 * p] = __fmul_rn(e2m1_to_f32(c0), sc);
+        xh[jj * D + 2 * p + 1] = __fmul_rn(e2m1_to_f32(c1), sc);
+      }
     }
-    float amax = fmaxf(fabsf(x0), fabsf(x1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
-    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
-    uint32_t sb = amax == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(amax, 6.0f));
-    const float s = e4m3_to_f32(sb);
-    uint32_t c0 = 0, c1 = 0;
-    if (s != 0.0f) {
-      c0 = f32_to_e2m1(__fdiv_rn(x0, s));
-      c1 = f32_to_e2m1(__fdiv_rn(x1, s));
-    } else {
-      sb = 0;
-    }
-    if (e < a.cap) {
-      const size_t row = (size_t)b * a.cap + e;
-      a.codes[row * (D / 2) + t] = (uint8_t)(c0 | (c1 << 4));
-      if ((t & 7) == 0) a.scales[row * (D / 16) + (t >> 3)] = (uint8_t)sb;
-    } else if (t == 0) {
-      flag(a.status, CSA2_DEV_APPEND_RANGE);
-    }
-    xh[jj * D + 2 * t] = __fmul_rn(e2m1_to_f32(c0), s);
-    xh[jj * D + 2 * t + 1] = __fmul_rn(e2m1_to_f32(c1), s);
   }
   // m = 2: the chunk's last token opens a pair -> it waits in the pending
   // buffer.  Block j0 == 0 is the only one that reads or writes it; it reads

@@ -79,10 +79,15 @@ struct SelSmem {
   uint2 coll[2][kColl];              // (key, column) of the threshold bin
 };
 
+struct MergeSmem {
+  SelSmem sel;
+  uint32_t key[kBpt * kT];
+};
+
 struct Smem {
   SelSmem sel;
-  uint32_t cand_key[kCap];
-  int32_t cand_col[kCap];
+  uint32_t bkey[kBpt * kT];          // block-maximum keys (SmemKeys layout)
+  uint32_t cand_key[kCap];           // candidate keys (SmemKeys layout)
   int32_t cand_blk[kCap / 8];        // candidate blocks, ascending
 };
 
@@ -111,16 +116,18 @@ __device__ __forceinline__ unsigned long long block_scan(unsigned long long v, u
   return (warp ? red[warp - 1] : 0ull) + x - v;
 }
 
-// Keys held in registers: thread t's element i is column t * N + i.
-template <int N>
-struct RegKeys {
+// Keys in shared memory: thread t's element i is column t * npt + i and
+// lives at k[i * kT + t] (consecutive threads read consecutive words).  The
+// loops stay rolled: each block runs this code once, so its size costs as
+// much as its execution.
+struct SmemKeys {
   const uint32_t *k;
-  int t;
-  __device__ __forceinline__ int col(int i) const { return t * N + i; }
+  int npt, t;
+  __device__ __forceinline__ int col(int i) const { return t * npt + i; }
   template <typename F>
   __device__ __forceinline__ void each(F f) const {
-#pragma unroll
-    for (int i = 0; i < N; ++i) f(k[i], i);
+#pragma unroll 1
+    for (int i = 0; i < npt; ++i) f(k[i * kT + t], i);
   }
 };
 
@@ -413,8 +420,7 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
   int32_t *out = a.out_idx + (size_t)row * a.K;
 
   // ---- block-maximum keys, 32 consecutive blocks per thread
-  uint32_t bkey[kBpt];
-#pragma unroll
+#pragma unroll 1
   for (int i = 0; i < kBpt; i += 4) {
     const int b0 = tid * kBpt + i;
     float4 v = make_float4(NAN, NAN, NAN, NAN);
@@ -424,9 +430,12 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
       if (b0 + 1 < nb) v.y = __ldcg(bm + b0 + 1);
       if (b0 + 2 < nb) v.z = __ldcg(bm + b0 + 2);
     }
-    bkey[i] = skey(v.x); bkey[i + 1] = skey(v.y); bkey[i + 2] = skey(v.z); bkey[i + 3] = skey(v.w);
+    sh.bkey[i * kT + tid] = skey(v.x);
+    sh.bkey[(i + 1) * kT + tid] = skey(v.y);
+    sh.bkey[(i + 2) * kT + tid] = skey(v.z);
+    sh.bkey[(i + 3) * kT + tid] = skey(v.w);
   }
-  const RegKeys<kBpt> bk{bkey, tid};
+  const SmemKeys bk{sh.bkey, kBpt, tid};   // each thread reads only its own keys
 
   // ---- pool (selection 1, when asked) and tau (selection 0)
   const int ks[2] = {a.K, a.P_out};
@@ -441,7 +450,7 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
     float *ops = a.out_pool_scores ? a.out_pool_scores + (size_t)row * a.P_out : nullptr;
     for_taken(bk, pr, sh.sel.red, lane, warp, [&](uint32_t key, int i, int pos) {
       if (pos < a.P_out) {
-        op[pos] = tid * kBpt + i;
+        op[pos] = bk.col(i);
         if (ops) ops[pos] = kval(key);
       }
     });
@@ -454,44 +463,39 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
   // ---- candidate blocks: maximum >= tau (every present block when fewer than K)
   const uint32_t tkey = few_blocks ? 1u : tau.kthr;
   int mine = 0;
-#pragma unroll
-  for (int i = 0; i < kBpt; ++i) mine += bkey[i] != 0u && bkey[i] >= tkey;
+  bk.each([&](uint32_t key, int) { mine += key != 0u && key >= tkey; });
   const int cb0 = (int)block_scan((unsigned long long)mine, sh.sel.red, lane, warp);
   const int n_cb = (int)sh.sel.red[kW - 1];
   int K_take;
   float *osc = a.out_scores ? a.out_scores + (size_t)row * a.K : nullptr;
   if (n_cb * 8 <= kCap) {
     // the candidate blocks in ascending order, then their scores loaded by
-    // all threads at once (column order); entries below tau (or beyond the
-    // row) cannot be selected
+    // all threads at once; entries below tau (or beyond the row) cannot be
+    // selected.  Candidate position j (column order) is element j % kCpt of
+    // thread j / kCpt.
     int slot = cb0;
-#pragma unroll
-    for (int i = 0; i < kBpt; ++i)
-      if (bkey[i] != 0u && bkey[i] >= tkey) sh.cand_blk[slot++] = tid * kBpt + i;
+    bk.each([&](uint32_t key, int i) {
+      if (key != 0u && key >= tkey) sh.cand_blk[slot++] = bk.col(i);
+    });
     __syncthreads();
-#pragma unroll
-    for (int u = 0; u < kCpt; ++u) {
-      const int j = tid + u * kT;
+#pragma unroll 1
+    for (int j = tid; j < kCap; j += kT) {
       uint32_t key = 0u;
-      int col = 0;
       if (j < n_cb * 8) {
-        col = sh.cand_blk[j >> 3] * 8 + (j & 7);
+        const int col = sh.cand_blk[j >> 3] * 8 + (j & 7);
         key = col < n ? skey(__ldcg(sc + col)) : 0u;
       }
-      sh.cand_key[j] = key >= tkey ? key : 0u;
-      sh.cand_col[j] = col;
+      sh.cand_key[(j % kCpt) * kT + j / kCpt] = key >= tkey ? key : 0u;
     }
     __syncthreads();
-    uint32_t ck[kCpt];
-#pragma unroll
-    for (int i = 0; i < kCpt; ++i) ck[i] = sh.cand_key[tid * kCpt + i];
-    const RegKeys<kCpt> cks{ck, tid};   // candidate positions ascend with the column
+    const SmemKeys cks{sh.cand_key, kCpt, tid};
     vselect<1>(cks, ks, sh.sel, tid, lane, warp);
     const SelRule rule = sh.sel.rule[0];
     K_take = min(sh.sel.n_present, a.K);
     for_taken(cks, rule, sh.sel.red, lane, warp, [&](uint32_t key, int i, int pos) {
       if (pos < a.K) {
-        out[pos] = sh.cand_col[tid * kCpt + i];
+        const int j = cks.col(i);
+        out[pos] = sh.cand_blk[j >> 3] * 8 + (j & 7);
         if (osc) osc[pos] = kval(key);
       }
     });
@@ -524,38 +528,34 @@ __global__ void __launch_bounds__(kT, 1) topk_bmax_kernel(const TopkBmaxArgs a) 
 // selection's column tie rule is the entry tie rule.
 __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkMergeArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  SelSmem &sel = *reinterpret_cast<SelSmem *>(smem_raw);
+  MergeSmem &ms = *reinterpret_cast<MergeSmem *>(smem_raw);
   const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   pdl_launch_dependents();
   pdl_wait();
   const int n = a.G * a.n_seg;
-  uint32_t key[kBpt];
-  int32_t gid[kBpt];
-#pragma unroll
-  for (int i = 0; i < kBpt; ++i) {
-    const int j = tid * kBpt + i;
-    key[i] = 0u;
-    gid[i] = -1;
+  // candidate j (segment-major order = entry order) is element j % kBpt of thread j / kBpt
+#pragma unroll 1
+  for (int j = tid; j < kBpt * kT; j += kT) {
+    uint32_t key = 0u;
     if (j < n) {
       const int g = j / a.n_seg, c = j % a.n_seg;
       const size_t at = ((size_t)g * a.rows + row) * a.n_seg + c;
-      const int id = a.ids[at];
-      if (id >= 0) {
-        key[i] = skey(a.scores[at]);
-        gid[i] = id + a.seg_base[g];
-      }
+      if (a.ids[at] >= 0) key = skey(a.scores[at]);
     }
+    ms.key[(j % kBpt) * kT + j / kBpt] = key;
   }
-  const RegKeys<kBpt> ks{key, tid};
+  __syncthreads();
+  const SmemKeys ks{ms.key, kBpt, tid};
   const int k[1] = {a.K};
-  vselect<1>(ks, k, sel, tid, lane, warp);
-  const SelRule rule = sel.rule[0];
-  const int K_take = min(sel.n_present, a.K);
+  vselect<1>(ks, k, ms.sel, tid, lane, warp);
+  const SelRule rule = ms.sel.rule[0];
+  const int K_take = min(ms.sel.n_present, a.K);
   int32_t *out = a.out_ids + (size_t)row * a.K;
   float *osc = a.out_scores ? a.out_scores + (size_t)row * a.K : nullptr;
-  for_taken(ks, rule, sel.red, lane, warp, [&](uint32_t kk, int i, int pos) {
+  for_taken(ks, rule, ms.sel.red, lane, warp, [&](uint32_t kk, int i, int pos) {
     if (pos < a.K) {
-      out[pos] = gid[i];
+      const int j = ks.col(i), g = j / a.n_seg, c = j % a.n_seg;
+      out[pos] = a.ids[((size_t)g * a.rows + row) * a.n_seg + c] + a.seg_base[g];
       if (osc) osc[pos] = kval(kk);
     }
   });
@@ -566,7 +566,7 @@ __global__ void __launch_bounds__(kT, 1) topk_merge_kernel(const TopkMergeArgs a
 }
 
 cudaError_t launch_topk_merge(const TopkMergeArgs &a, cudaStream_t s) {
-  const size_t smem = sizeof(SelSmem);
+  const size_t smem = sizeof(MergeSmem);
   cudaError_t e = cudaFuncSetAttribute(topk_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_merge_kernel, dim3(a.rows), dim3(kT), smem, s, dim3(1, 1, 1), a);
