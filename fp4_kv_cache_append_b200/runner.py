@@ -42,7 +42,7 @@ class Step:
     """Caches, inputs and buffers of one workload; `run()` enqueues one step."""
 
     def __init__(self, wl: I.Workload, seed: int = 0, device: str = "cuda", copies: int = 1,
-                 prefill_chunk: int = 16384):
+                 prefill_chunk: int = 16384, fused: bool = False):
         self.wl, self.seed, self.device = wl, seed, device
         self.prefill_chunk = prefill_chunk
         self.plan = PLANS[wl.mode]
@@ -101,9 +101,12 @@ class Step:
         ws_at = C.csa2_attn_workspace_size(B, self.T_q, wl.H, D, wl.K, wl.window)
         self.ws_topk = C.workspace(max(ws_full, ws_re), dev)
         self.ws_attn = C.workspace(ws_at, dev)
-        # Full layers of contexts up to 131,072 entries select from the block
-        # maxima their scan writes (csa2_index_topk); longer ones scan, then select
-        self.fused = wl.mode in ("full", "prefill") and self.cap <= 131072
+        # fused: the Full layer selects from the block maxima its scan writes
+        # (csa2_index_topk, contexts up to 131,072 entries); otherwise the scan
+        # writes the scores and csa2_topk selects from them.  The second is
+        # the faster today (measured: the fused selection's one block per row
+        # is instruction-bound), so it is the default.
+        self.fused = fused and wl.mode in ("full", "prefill") and self.cap <= 131072
         ws_i = (C.csa2_index_topk_workspace_size(self.rows, self.cap, wl.dI) if self.fused
                 else C.csa2_index_workspace_size(self.rows, wl.dI))
         self.ws_index = C.workspace(ws_i, dev)
