@@ -94,7 +94,7 @@ KERNEL_SOURCES = {   # what builds each entry point's kernels
     "index_full": ("index.cu", "common.cuh", "kernels.h"),
     "index_topk": ("index.cu", "topk_bmax.cu", "common.cuh", "kernels.h"),
     "index_reindex": ("index.cu", "common.cuh", "kernels.h"),
-    "attn": ("attn.cu", "common.cuh", "kernels.h"),
+    "attn": ("attn.cu", "attn_lat.cu", "common.cuh", "kernels.h"),
     "topk": ("topk_cluster.cu", "topk.cu", "common.cuh", "kernels.h"),
     "append": ("append.cu", "common.cuh", "kernels.h"),
 }

@@ -575,6 +575,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
     p.nsplit = 1;
     p.chunks_per_split = 1 << 20;
     p.csplit = 1;
+    p.one_wave = (int64_t)main->B * T_q <= d->sms ? 1 : 0;
   }
   AttnArgs a{};
   a.codes = main->codes; a.scales = main->scales; a.cap = main->cap; a.D = main->D;
@@ -582,7 +583,8 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   a.q = q; a.q_pos = q_pos; a.B = main->B; a.T_q = T_q; a.H = H; a.idx = K > 0 ? idx : nullptr; a.K = K;
   a.scale = softmax_scale; a.out = out;
   a.ws = p.nsplit > 1 ? static_cast<float *>(ws) : nullptr;
-  a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.csplit = p.csplit; a.status = d->status;
+  a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.csplit = p.csplit; a.one_wave = p.one_wave;
+  a.status = d->status;
   cudaError_t e = launch_attn(a, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "attention launch");
 }

@@ -15,7 +15,9 @@
 //               into the K-major 128B-swizzled K^ tile, chunk by chunk; a
 //               chunk is overwritten only after the previous tile's O^T MMAs
 //               that read it completed
-//   warp 12     tcgen05.mma issuer: S^T = K^ Q^T chunk by chunk as chunks
+//   warp 12     tcgen05.mma issuer (converged warp, one elected lane issues;
+//               a lane-0-only branch issues MMAs several times slower):
+//               S^T = K^ Q^T chunk by chunk as chunks
 //               land (M = 128 keys, N = 64 heads, K = 16, kind::f16), then,
 //               once P is written, O^T += V^T P^T per 128-channel block (V^T
 //               is the same K^ tile read MN-major) and the row sums
@@ -328,9 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
         for (int j = 0; j < 4; ++j)
           *reinterpret_cast<uint4 *>(S.kh + sw_off(r, 8 * k + 4 * hf + j, kTile)) =
               make_uint4(h[4 * j], h[4 * j + 1], h[4 * j + 2], h[4 * j + 3]);
-        fence_proxy_async();   // generic stores -> visible to the tensor core
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&S.chunk_full[k]);
+        if (k & 1) {   // chunks are handed over in pairs: one proxy fence per two
+          fence_proxy_async();   // generic stores -> visible to the tensor core
+          __syncwarp();
+          if (lane == 0) { mbar_arrive(&S.chunk_full[k - 1]); mbar_arrive(&S.chunk_full[k]); }
+        }
       }
       if (!ok) break;
       id = id_next;
@@ -494,47 +498,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.p_full);
     }
-  } else if (lane == 0) {
-    // ================================================ MMA issuer
+  } else {
+    // ================================================ MMA issuer: the whole warp runs
+    // the loop converged (every lane polls the barriers), one elected lane
+    // issues the MMAs and their commits
     const uint32_t kh_base = smem_u32(S.kh), q_base = smem_u32(S.q), p_base = smem_u32(S.p);
     const uint64_t dq0 = smem_desc_kmajor(q_base, 128), dk0 = smem_desc_kmajor(kh_base, 128);
     const uint64_t dv0 = smem_desc_mnmajor_sw128(kh_base, kTile * 128, 1024);
     const uint64_t dp0 = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
-    bool ok = n_tiles == 0 || wait_or_abort(&S.q_ready, 0, abort);
+    auto all_wait = [&](uint64_t *bar, uint32_t parity) {
+      return __all_sync(0xffffffffu, wait_or_abort(bar, parity, abort)) != 0;
+    };
+    bool ok = n_tiles == 0 || all_wait(&S.q_ready, 0);
 #pragma unroll 1
     for (int it = 0; it < n_tiles && ok; ++it) {
+      // the bases pass through an opaque copy each tile, so that the
+      // unrolled loops below form each descriptor next to its MMA instead of
+      // holding all of them in registers across the tile loop
+      uint64_t dk = dk0, dq = dq0, dv = dv0, dp = dp0;
+      asm volatile("" : "+l"(dk), "+l"(dq), "+l"(dv), "+l"(dp));
       // S^T = K^ Q^T, chunk by chunk as the chunks land
-#pragma unroll 1
-      for (int k = 0; k < NCH; ++k) {
-        if (!wait_or_abort(&S.chunk_full[k], it & 1, abort)) { ok = false; break; }
-        tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)   // descriptors advance by (byte offset >> 4)
-          tc_mma_f16(tmem + kColS, dk0 + ((k * (kTile * 128) + kk * 32) >> 4),
-                     dq0 + ((k * (kHeads * 128) + kk * 32) >> 4), kIdS, (k > 0 || kk > 0) ? 1u : 0u);
+      for (int k = 0; k < NCH; ++k) {
+        if (!all_wait(&S.chunk_full[k], it & 1)) { ok = false; break; }
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)   // descriptors advance by (byte offset >> 4)
+            tc_mma_f16(tmem + kColS, dk + ((k * (kTile * 128) + kk * 32) >> 4),
+                       dq + ((k * (kHeads * 128) + kk * 32) >> 4), kIdS, (k > 0 || kk > 0) ? 1u : 0u);
+        }
+        __syncwarp();
       }
       if (!ok) break;
-      tc_commit(&S.s_full);
-      if (!wait_or_abort(&S.p_full, it & 1, abort)) { ok = false; break; }
+      if (elect_one()) tc_commit(&S.s_full);
+      __syncwarp();
+      if (!all_wait(&S.p_full, it & 1)) { ok = false; break; }
       tc_fence_after();
       const uint32_t acc0 = it > 0 ? 1u : 0u;
-      // L^T += 1 P^T (every lane gets the per-head sums of P)
+      if (elect_one()) {
+        // L^T += 1 P^T (every lane gets the per-head sums of P)
 #pragma unroll
-      for (int ks = 0; ks < kTile / 16; ++ks)
-        tc_mma_f16_ta(tmem + kColL, tmem + kColOnes, dp0 + (((2 * ks) * 1024) >> 4), kIdL, (ks > 0) ? 1u : acc0);
-      // O^T += V^T P^T per 128-channel block; each block's commit frees its two K^ chunks
+        for (int ks = 0; ks < kTile / 16; ++ks)
+          tc_mma_f16_ta(tmem + kColL, tmem + kColOnes, dp + (((2 * ks) * 1024) >> 4), kIdL, (ks > 0) ? 1u : acc0);
+        // O^T += V^T P^T per 128-channel block; each block's commit frees its two K^ chunks
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        if (mt >= mt_lo && mt < mt_hi) {
+        for (int mt = 0; mt < MT; ++mt) {
+          if (mt >= mt_lo && mt < mt_hi) {
 #pragma unroll
-          for (int ks = 0; ks < kTile / 16; ++ks)
-            tc_mma_f16(tmem + kColO + mt * kHeads, dv0 + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
-                       dp0 + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0) ? 1u : acc0);
+            for (int ks = 0; ks < kTile / 16; ++ks)
+              tc_mma_f16(tmem + kColO + mt * kHeads, dv + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
+                         dp + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0) ? 1u : acc0);
+          }
+          tc_commit(&S.o_done[mt]);
         }
-        tc_commit(&S.o_done[mt]);
       }
+      __syncwarp();
     }
-    tc_commit(&S.fin);   // arrives once every MMA issued above is done
+    if (elect_one()) tc_commit(&S.fin);   // arrives once every MMA issued above is done
+    __syncwarp();
   }
 
   // ---- epilogue: O^T (TMEM lane = channel within a 128-channel block)
@@ -743,6 +765,11 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   // small batches: two blocks per split, each issuing the O^T MMAs of, and
   // writing and merging, half of the channels (both compute S and P)
   p.csplit = (nsplit > 1 && D % 256 == 0 && (long long)rows * nsplit * 2 <= sms) ? 2 : 1;
+  // Measured on B200 (dec_full shapes, 1 to 4096 rows): while every block of
+  // the launch is resident at once, the form in which all warps take each
+  // phase of a tile in turn is the faster (by about 2 us up to 128 rows);
+  // from two waves on, the pipelined form below (by 2-8%).
+  p.one_wave = (long long)rows * nsplit * p.csplit <= sms ? 1 : 0;
   // fp16 partials [rows][nsplit][64][D] then f32 max and sum [rows][nsplit][64] each
   p.bytes = nsplit > 1 ? (size_t)rows * nsplit * kHeads * ((size_t)D * 2 + 2 * sizeof(float)) : 0;
   return p;
@@ -758,6 +785,7 @@ static cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s) {
+  if (a.one_wave) return launch_attn_lat(a, s);
   switch (a.D) {
     case 128: return launch_attn_t<128>(a, s);
     case 256: return launch_attn_t<256>(a, s);

@@ -20,7 +20,7 @@ PKG = os.path.dirname(HERE)
 ROOT = os.path.dirname(PKG)
 OBJ = os.path.join(ROOT, "_build", "csa2")
 LIB = os.path.join(PKG, "lib", "libcsa2.so")
-SOURCES = ["api.cu", "append.cu", "project.cu", "index.cu", "topk.cu", "topk_cluster.cu", "topk_bmax.cu", "attn.cu", "shard.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "append.cu", "project.cu", "index.cu", "topk.cu", "topk_cluster.cu", "topk_bmax.cu", "attn.cu", "attn_lat.cu", "shard.cu", "noalloc.cu"]
 HEADERS = ["common.cuh", "kernels.h", os.path.join("..", "..", "include", "csa2.h")]
 
 

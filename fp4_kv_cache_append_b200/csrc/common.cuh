@@ -269,6 +269,17 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One lane of a converged warp (the lowest active one, the same lane on every
+// call with the same active set).  tcgen05.mma / tcgen05.commit are issued
+// under it from code the whole warp runs: the descriptors then stay warp-
+// uniform, which keeps the issue of back-to-back MMAs near the tensor core's
+// own rate (a lane-0-only branch issues them several times slower).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile("{\n .reg .pred e;\n elect.sync _|e, 0xffffffff;\n selp.u32 %0, 1, 0, e;\n}\n" : "=r"(p));
+  return p != 0;
+}
+
 // Named barrier over `nthreads` threads (whole warps) that also returns
 // whether any of them passed a true predicate.
 __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool pred) {
