@@ -51,6 +51,7 @@ namespace csa2 {
 namespace {
 
 constexpr int kThreads = 256;
+constexpr int kMmaWarp = 4;        // issues the MMAs (converged, one elected lane)
 constexpr int kTile = 128;         // keys per tile (M of S^T)
 constexpr int kHeads = 64;         // heads padded to 64 (N)
 constexpr float kLog2e = 1.4426950408889634f;
@@ -199,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
     S.rescale = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&S.tmem_base, kCols);
     tmem_relinquish();
   }
@@ -331,18 +332,21 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
     tc_fence_before();
     __syncthreads();
 
-    // ---- 2. S^T = K^ Q^T
-    if (tid == 128) {
+    // ---- 2. S^T = K^ Q^T (warp 4 converged, one elected lane issues)
+    if (warp == kMmaWarp) {
       // descriptors advance by (byte offset >> 4) in their start-address field
       tc_fence_after();
       const uint64_t da = smem_desc_kmajor(kh_base, 128), db = smem_desc_kmajor(q_base, 128);
+      if (elect_one()) {
 #pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const uint32_t off = (uint32_t)((ks & 3) * 32);
-        tc_mma_f16(tmem, da + (((ks >> 2) * (kTile * 128) + off) >> 4), db + (((ks >> 2) * (kHeads * 128) + off) >> 4),
-                   kIdS, ks > 0 ? 1u : 0u);
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t off = (uint32_t)((ks & 3) * 32);
+          tc_mma_f16(tmem, da + (((ks >> 2) * (kTile * 128) + off) >> 4),
+                     db + (((ks >> 2) * (kHeads * 128) + off) >> 4), kIdS, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(&S.sbar);
       }
-      tc_commit(&S.sbar);
+      __syncwarp();
     }
     // the next tile's key ids (the other buffer) while the MMAs run
     if (c + 1 < c_end) load_key_ids<D>(a, row, b, c + 1, n_fp4_tiles, wlo, nwin, S.key_ent[(c + 1) & 1], tid, true);
@@ -453,19 +457,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
     if (tid == 0) S.rescale = 0;
 
     // ---- 4. O^T += V^T P^T
-    if (tid == 128) {
+    if (warp == kMmaWarp) {
       tc_fence_after();
       const uint64_t da = smem_desc_mnmajor_sw128(kh_base, kTile * 128, 1024);
       const uint64_t db = smem_desc_mnmajor_sw128(p_base, kTile * 128, 1024);
+      if (elect_one()) {
 #pragma unroll
-      for (int mt = 0; mt < MT; ++mt) {
-        if (mt < mt_lo || mt >= mt_hi) continue;
+        for (int mt = 0; mt < MT; ++mt) {
+          if (mt < mt_lo || mt >= mt_hi) continue;
 #pragma unroll
-        for (int ks = 0; ks < kTile / 16; ++ks)
-          tc_mma_f16(tmem + kHeads + mt * kHeads, da + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
-                     db + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0 || !first) ? 1u : 0u);
+          for (int ks = 0; ks < kTile / 16; ++ks)
+            tc_mma_f16(tmem + kHeads + mt * kHeads, da + (((2 * mt) * (kTile * 128) + (2 * ks) * 1024) >> 4),
+                       db + (((2 * ks) * 1024) >> 4), kIdO, (ks > 0 || !first) ? 1u : 0u);
+        }
+        tc_commit(&S.obar);
       }
-      tc_commit(&S.obar);
+      __syncwarp();
     }
     ++n_done;
   }
@@ -476,11 +483,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
   const bool failed = __syncthreads_or(!ok);
   if (failed) {
     if (tid == 0) flag(a.status, CSA2_DEV_TIMEOUT);
-    if (tid == 128 && n_done > 0) {   // let every issued MMA finish before TMEM is freed
-      mbar_init(&S.sbar, 1);
-      fence_barrier_init();
-      tc_commit(&S.sbar);
-      mbar_wait_bounded(&S.sbar, 0, kWaitLimit);
+    if (warp == kMmaWarp && n_done > 0) {   // let every issued MMA finish before TMEM is freed
+      if (elect_one()) {                     // the lane that issued them
+        mbar_init(&S.sbar, 1);
+        fence_barrier_init();
+        tc_commit(&S.sbar);
+        mbar_wait_bounded(&S.sbar, 0, kWaitLimit);
+      }
+      __syncwarp();
     }
   } else {
     tc_fence_after();
@@ -536,7 +546,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kCols);
   }
