@@ -267,6 +267,31 @@ __global__ void append_kernel(const AppendArgs a) {
   }
 }
 
+// One indexer-key output as one fused multiply-add chain over the channels in
+// ascending order from +0: x^ (binary32, shared) times column `wcol` of the
+// staged W_ik slice (bf16, row stride OPB).  The operands of 32 channels are
+// loaded into registers before their 32 multiply-adds, so the loop runs near
+// the multiply-add latency.
+template <int OPB>
+__device__ __forceinline__ float dec_key_chain_t(const float *xh, const uint16_t *wcol, int D) {
+  float acc = 0.0f;
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 32) {
+    float xs[32], ws[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      xs[j] = xh[c0 + j];
+      ws[j] = bf16_to_f32(wcol[(c0 + j) * OPB]);
+    }
+#pragma unroll
+    for (int j = 0; j < 32; ++j) acc = __fmaf_rn(xs[j], ws[j], acc);
+  }
+  return acc;
+}
+__device__ __forceinline__ float dec_key_chain(const float *xh, const uint16_t *wcol, int D, int OPB) {
+  return OPB == 16 ? dec_key_chain_t<16>(xh, wcol, D) : dec_key_chain_t<8>(xh, wcol, D);
+}
+
 // Decode (one new token per sequence, m = 1): a cluster of 8 blocks per
 // sequence.  Every block quantises the new entry (the same binary32 steps as
 // append_entries, so all blocks hold the same x^); block c projects indexer
@@ -277,7 +302,7 @@ __global__ void append_kernel(const AppendArgs a) {
 constexpr int kDecCl = 8;
 
 __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_decode_kernel(const AppendArgs a) {
-  __shared__ float xh[512];
+  __shared__ alignas(16) float xh[512];
   __shared__ alignas(16) uint16_t wsl[512 * 16];   // W_ik[:, c*OPB .. c*OPB+OPB), row-major [D][OPB]
   __shared__ float kmx[kDecCl];                    // the blocks' local key maxima
   cg::cluster_group cl = cg::this_cluster();
@@ -361,11 +386,7 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
   float k = 0.0f;
   if (t < 32) {
     if (t < OPB) {
-      const uint16_t *wcol = wsl + t;
-      float acc = 0.0f;
-#pragma unroll 8
-      for (int cc = 0; cc < D; ++cc) acc = __fmaf_rn(xh[cc], bf16_to_f32(wcol[cc * OPB]), acc);
-      k = acc;
+      k = dec_key_chain(xh, wsl + t, D, OPB);
     }
     float m = t < OPB ? fabsf(k) : 0.0f;
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
