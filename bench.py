@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--copies", type=int, default=4)
     ap.add_argument("--min-ms", type=float, default=3000.0,
                     help="timed repeats of K steps continue until they span this long (at least 5 repeats)")
-    ap.add_argument("--configs", default="dec_group,long,enc_prefill",
+    ap.add_argument("--configs", default="dec_group,long,enc_prefill,ced_project",
                     help="other workloads to time on rank 0 of a one-GPU run (comma list, or 'none')")
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -477,6 +477,9 @@ def run_other_configs(args, hbm, barrier):
     out = {}
     fp8 = 2.0 * bf16_peak()
     for name in args.configs:
+        if name == "ced_project":
+            out[name] = ced_project_config(hbm, barrier)
+            continue
         copies, n_steps = OTHER_CONFIGS[name]
         wl = I.WORKLOADS[name]
         t0 = time.perf_counter()
@@ -518,6 +521,61 @@ def run_other_configs(args, hbm, barrier):
         gc.collect()
         torch.cuda.empty_cache()
     return out
+
+
+CED_SHAPE = dict(T=8192, d_model=4096, D=512, dI=128)
+
+
+def ced_project_config(hbm, barrier):
+    """The CED decoder-KV producer (csa2_append_project): one prefill chunk's
+    decoder-layer KV kv = H W_KV (bf16 tcgen05 GEMM, FP4 E2M1/E4M3 quantised
+    in its epilogue) plus the entries' FP8 indexer keys, B = 1, T = 8,192
+    tokens, d_model = 4,096 (the pages give no hidden size: our choice),
+    D = 512, d_I = 128.  H ~ N(0, 1), W_KV ~ N(0, 1/d_model), W_IK ~ N(0, 1/D)
+    (bf16).  Three H copies (201 MB, larger than L2) rotate; a CUDA graph of
+    12 calls per repeat, median over repeats."""
+    import torch
+
+    from fp4_kv_cache_append_b200 import csa2 as C
+    T, dm, D, dI = (CED_SHAPE[k] for k in ("T", "d_model", "D", "dI"))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(20261203)
+    dev = "cuda"
+    copies = 3
+    Hs = [torch.randn(1, T, dm, generator=g, device=dev).to(torch.bfloat16) for _ in range(copies)]
+    w_kv = (torch.randn(dm, D, generator=g, device=dev) / dm ** 0.5).to(torch.bfloat16)
+    w_ik = (torch.randn(D, dI, generator=g, device=dev) / D ** 0.5).to(torch.bfloat16)
+    main = C.MainCache(1, T, D, dI, 1, device=dev)
+    pos0 = torch.zeros(1, dtype=torch.int32, device=dev)
+    for cp in range(copies):
+        C.csa2_append_project(main, Hs[cp], w_kv, w_ik, pos0)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    n = 12
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for i in range(n):
+            C.csa2_append_project(main, Hs[i % copies], w_kv, w_ik, pos0)
+    for _ in range(3):
+        graph.replay()
+    reps = timed_repeats(graph.replay, 200.0, 5, barrier)
+    ms = statistics.median(reps) / n
+    gemm_flops = 2.0 * T * dm * D
+    key_flops = 2.0 * T * D * dI
+    nbytes = T * dm * 2 + dm * D * 2 + D * dI * 2 + T * (D // 2 + D // 16 + dI + 4)
+    peak = bf16_peak()
+    tflops = gemm_flops / (ms * 1e-3) / 1e12
+    del graph
+    assert C.csa2_device_status() == 0
+    return {"workload": "CED decoder-KV producer: kv = H W_KV (bf16 GEMM, FP4-quantised in the epilogue) + FP8 "
+                        f"indexer keys; B 1, T {T}, d_model {dm} (our choice: the pages give no hidden size), D {D}, "
+                        f"d_I {dI}",
+            "ms_per_call": ms, "tokens_per_s": T / (ms * 1e-3), "repeats": len(reps), "calls_per_repeat": n,
+            "gemm_flops": gemm_flops, "key_flops": key_flops, "bytes_per_call": nbytes,
+            "gemm_tflops": tflops, "peak_tflops": peak, "peak_kind": "dense bf16 burst (measured, else fallback)",
+            "frac_bf16": tflops / peak, "gbs": nbytes / (ms * 1e-3) / 1e9,
+            "frac_hbm": nbytes / (ms * 1e-3) / 1e9 / hbm,
+            "l2": f"{copies} rotating H copies ({copies * T * dm * 2 // 2**20} MiB)"}
 
 
 WORKLOAD_DESCS = {

@@ -63,41 +63,53 @@ __device__ __forceinline__ float pool_pair(float ka, float kb, float za, float z
 // dI, k < kChains): its chains run side by side, share every W_ik element it
 // reads and take 4 channels of an entry per 16-byte load.  Every thread of
 // the block must call it.
-__device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const float *xh, float *kbuf,
-                           const uint16_t *ws) {
-  const int t = threadIdx.x, D = a.D, dI = a.dI;
-  {
-    constexpr int kChains = 8;   // 32 entries over 4 (dI = 128) slots of 512 threads; dI = 64 uses 4 of them
-    const int slots = (int)blockDim.x / dI;
-    const int i = t % dI, s0 = t / dI;
-    float acc[kChains];
+template <int D, int DI>
+__device__ __forceinline__ void entry_chains(int count, const float *xh, float *kbuf, const uint16_t *ws) {
+  constexpr int kChains = 8;   // 32 entries over 4 (d_I = 128) slots of 512 threads; d_I = 64 uses 4 of them
+  constexpr int kSlots = 512 / DI;
+  const int t = threadIdx.x;
+  const int i = t % DI, s0 = t / DI;
+  if (s0 >= count) return;
+  // which of this thread's chains exist, decided once (warp-uniform)
+  bool act[kChains];
 #pragma unroll
-    for (int k = 0; k < kChains; ++k) acc[k] = 0.0f;
-    if (s0 < count) {
-      const uint16_t *wcol = ws + i;
+  for (int k = 0; k < kChains; ++k) act[k] = s0 + k * kSlots < count;
+  float acc[kChains];
+#pragma unroll
+  for (int k = 0; k < kChains; ++k) acc[k] = 0.0f;
+  const uint16_t *wcol = ws + i;
+  const float *xr = xh + s0 * D;   // chain k reads row s0 + k * kSlots: a constant offset
 #pragma unroll 2
-      for (int c = 0; c < D; c += 4) {
-        const float w0 = bf16_to_f32(wcol[c * dI]), w1 = bf16_to_f32(wcol[(c + 1) * dI]);
-        const float w2 = bf16_to_f32(wcol[(c + 2) * dI]), w3 = bf16_to_f32(wcol[(c + 3) * dI]);
+  for (int c = 0; c < D; c += 4) {
+    const float w0 = bf16_to_f32(wcol[c * DI]), w1 = bf16_to_f32(wcol[(c + 1) * DI]);
+    const float w2 = bf16_to_f32(wcol[(c + 2) * DI]), w3 = bf16_to_f32(wcol[(c + 3) * DI]);
 #pragma unroll
-        for (int k = 0; k < kChains; ++k) {
-          const int jj = s0 + k * slots;
-          if (jj < count) {
-            const float4 x = *reinterpret_cast<const float4 *>(xh + jj * D + c);
-            float v = acc[k];
-            v = __fmaf_rn(x.x, w0, v);
-            v = __fmaf_rn(x.y, w1, v);
-            v = __fmaf_rn(x.z, w2, v);
-            acc[k] = __fmaf_rn(x.w, w3, v);
-          }
-        }
-      }
-#pragma unroll
-      for (int k = 0; k < kChains; ++k) {
-        const int jj = s0 + k * slots;
-        if (jj < count) kbuf[jj * dI + i] = acc[k];
+    for (int k = 0; k < kChains; ++k) {
+      if (act[k]) {
+        const float4 x = *reinterpret_cast<const float4 *>(xr + k * kSlots * D + c);
+        float v = acc[k];
+        v = __fmaf_rn(x.x, w0, v);
+        v = __fmaf_rn(x.y, w1, v);
+        v = __fmaf_rn(x.z, w2, v);
+        acc[k] = __fmaf_rn(x.w, w3, v);
       }
     }
+  }
+#pragma unroll
+  for (int k = 0; k < kChains; ++k)
+    if (act[k]) kbuf[(s0 + k * kSlots) * DI + i] = acc[k];
+}
+
+__device__ void entry_keys(const AppendArgs &a, int b, int e0, int count, const float *xh, float *kbuf,
+                           const uint16_t *ws) {
+  const int t = threadIdx.x, dI = a.dI;
+  switch (a.D * 1000 + dI) {   // the chains with compile-time strides
+    case 512128: entry_chains<512, 128>(count, xh, kbuf, ws); break;
+    case 512064: entry_chains<512, 64>(count, xh, kbuf, ws); break;
+    case 256128: entry_chains<256, 128>(count, xh, kbuf, ws); break;
+    case 256064: entry_chains<256, 64>(count, xh, kbuf, ws); break;
+    case 128128: entry_chains<128, 128>(count, xh, kbuf, ws); break;
+    default: entry_chains<128, 64>(count, xh, kbuf, ws); break;
   }
   __syncthreads();
   // ---- FP8 key per entry: warp w takes entries w, w + warps, ...
