@@ -176,6 +176,138 @@ def _check_scores(got, ref):
     assert np.all(err <= SCORE_RTOL * np.abs(ref) + atol), f"max err {err.max()} (max ref {np.abs(ref).max()})"
 
 
+@pytest.mark.parametrize("D,dI,H_I,n,T_q,m", [(128, 64, 4, 1000, 1, 1), (512, 128, 64, 2047, 3, 1),
+                                              (256, 128, 17, 700, 2, 1), (512, 128, 64, 900, 4, 2)])
+def test_index_full_vs_oracle(D, dI, H_I, n, T_q, m):
+    B = 2
+    cap = (n // m + 127) // 128 * 128 + 128
+    T = n
+    gm, _, om, _, _ = build_pair(B=B, cap=cap, D=D, dI=dI, m=m, T=T, pos0=[0, 0], seed=n + dI, swa=False)
+    q, w = _rows_queries(B, T_q, H_I, dI, seed=7)
+    # causal positions: the last T_q tokens, and one early query
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[1, 0] = 300
+    scores = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nval = torch.zeros(B * T_q, dtype=torch.int32, device="cuda")
+    C.csa2_index_full(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), scores, nval)
+    torch.cuda.synchronize()
+    sc = scores.cpu().numpy()
+    nv = nval.cpu().numpy()
+    for b in range(B):
+        for j in range(T_q):
+            r = b * T_q + j
+            n_vis = oracle.n_visible(int(om.n_entries[b]), int(qpos[b, j]), m)
+            assert nv[r] == n_vis
+            ref = oracle.index_scores(om, b, bits(q[b, j]), w[b, j].numpy(), n_vis)
+            _check_scores(sc[r, :n_vis], ref)
+            assert np.all(np.isnan(sc[r, n_vis:])), "columns beyond n_vis must not be written"
+    assert C.csa2_device_status() == 0
+
+
+@pytest.mark.parametrize("D,dI,H_I,T_q", [(512, 128, 64, 1), (256, 64, 17, 3)])
+def test_index_full_prepared_by_the_append(D, dI, H_I, T_q):
+    """Append + query preparation in one launch, then the prepared scan: the
+    cache bytes of the appended token, and scores bit-identical to the plain
+    scan (which itself is checked against the oracle above)."""
+    B, n = 2, 3000
+    cap = (n + 1 + 127) // 128 * 128
+    gm, gs, om, osw, W = build_pair(B=B, cap=cap, D=D, dI=dI, m=1, T=n, pos0=[0, 0], seed=31 + D)
+    q, w = _rows_queries(B, T_q, H_I, dI, seed=32)
+    g = gen(33)
+    kv = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+    kvs = torch.randn(B, 1, D, generator=g).to(torch.bfloat16)
+    pos = np.array([n, n], np.int32)
+    qpos = np.array([[n - T_q + 1 + j for j in range(T_q)] for _ in range(B)], np.int32)
+    qpos[:, -1] = n
+    ws = C.workspace(C.csa2_index_workspace_size(B * T_q, dI))
+    C.csa2_append_quant_ex(gm, kv.cuda(), None, W.cuda(), gs, kvs.cuda(), torch.from_numpy(pos).cuda(), 1,
+                           q.cuda(), w.cuda(), ws)
+    oracle.append(om, bits(kv), None, bits(W), osw, bits(kvs), pos, 1)
+    got = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nv = torch.empty(B * T_q, dtype=torch.int32, device="cuda")
+    C.csa2_index_full_prepared(gm, torch.from_numpy(qpos).cuda(), got, nv, ws=ws)
+    plain = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    C.csa2_index_full(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), plain, nv)
+    torch.cuda.synchronize()
+    assert_cache_equal(gm, om, gs, osw)
+    a, b_ = got.cpu().numpy(), plain.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b_.view(np.uint32))
+    # preparation only (T = 0): the same workspace contents
+    ws2 = C.workspace(C.csa2_index_workspace_size(B * T_q, dI))
+    C.csa2_append_quant_ex(gm, None, None, None, None, None, torch.from_numpy(pos).cuda(), 0, q.cuda(), w.cuda(), ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(ws.cpu(), ws2.cpu())
+    assert C.csa2_device_status() == 0
+
+
+@pytest.mark.parametrize("T_q", [1, 4])
+def test_index_scan_wait_that_runs_out_flags_and_recovers(T_q):
+    """Failure detection without a fault: with csa2_debug_inject_timeout the
+    scan's MMA issuer waits on a barrier that nothing arrives on; the wait
+    runs out, the scan sets CSA2_DEV_TIMEOUT, stops every role, drains its
+    copies and MMAs, frees its tensor memory and returns.  The context stays
+    usable: the next scans give the reference scores again."""
+    B, n, D, dI, H_I = 2, 3000, 256, 128, 64
+    gm, _, om, _, _ = build_pair(B=B, cap=3072, D=D, dI=dI, m=1, T=n, pos0=[0, 0], seed=91, swa=False)
+    g = gen(92)
+    qi = torch.randn(B, T_q, H_I, dI, generator=g).to(torch.bfloat16).cuda()
+    w = torch.rand(B, T_q, H_I, generator=g).cuda()
+    qpos = torch.tensor(np.stack([np.arange(n - T_q, n)] * B), dtype=torch.int32).cuda()
+    ref = torch.zeros(B * T_q, 3072, device="cuda")
+    C.csa2_index_full(gm, qi, w, qpos, ref)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    bad = torch.zeros_like(ref)
+    C.csa2_debug_inject_timeout(64)
+    try:
+        C.csa2_index_full(gm, qi, w, qpos, bad)
+        torch.cuda.synchronize()
+    finally:
+        C.csa2_debug_inject_timeout(0)
+    assert C.csa2_device_status(clear=True) & C.DEV_TIMEOUT
+    assert not torch.equal(bad, ref)   # the scan gave up before writing its scores
+    again = torch.zeros_like(ref)
+    for _ in range(2):
+        C.csa2_index_full(gm, qi, w, qpos, again)
+    torch.cuda.synchronize()
+    assert C.csa2_device_status() == 0
+    assert torch.equal(again, ref)
+
+
+@pytest.mark.parametrize("T_q,m", [(8, 1), (6, 1), (4, 2)])
+def test_index_full_row_groups_match_single_rows(T_q, m):
+    """T_q a multiple of 4 (or 2) takes the multi-row scan, which puts 4 (or 2)
+    query rows on one MMA; every row's scores must equal, bit for bit, those
+    of the one-row scan of that row alone (same per-entry head reduction)."""
+    B, D, dI, H_I, n = 2, 512, 128, 64, 5000
+    cap = (n // m + 127) // 128 * 128 + 128
+    gm, _, om, _, _ = build_pair(B=B, cap=cap, D=D, dI=dI, m=m, T=n, pos0=[0, 0], seed=41 + T_q, swa=False)
+    q, w = _rows_queries(B, T_q, H_I, dI, seed=42)
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[1, 1] = 777   # rows of one group with different causal limits
+    grouped = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nval = torch.zeros(B * T_q, dtype=torch.int32, device="cuda")
+    C.csa2_index_full(gm, q.cuda(), w.cuda(), torch.from_numpy(qpos).cuda(), grouped, nval)
+    single = torch.full((B * T_q, cap), float("nan"), device="cuda")
+    nv1 = torch.zeros(B, dtype=torch.int32, device="cuda")
+    for j in range(T_q):
+        out = torch.full((B, cap), float("nan"), device="cuda")
+        C.csa2_index_full(gm, q[:, j:j + 1].contiguous().cuda(), w[:, j:j + 1].contiguous().cuda(),
+                          torch.from_numpy(qpos[:, j:j + 1].copy()).cuda(), out, nv1)
+        single[j::T_q] = out
+    torch.cuda.synchronize()
+    a, b_ = grouped.cpu().numpy(), single.cpu().numpy()
+    assert np.array_equal(a.view(np.uint32), b_.view(np.uint32))
+    nv = nval.cpu().numpy()
+    for b in range(B):
+        for j in (0, T_q - 1):
+            r = b * T_q + j
+            n_vis = oracle.n_visible(int(om.n_entries[b]), int(qpos[b, j]), m)
+            assert nv[r] == n_vis
+            _check_scores(a[r, :n_vis], oracle.index_scores(om, b, bits(q[b, j]), w[b, j].numpy(), n_vis))
+    assert C.csa2_device_status() == 0
+
+
 # ------------------------------------------------------------------ projected append (CED producer)
 
 
