@@ -673,6 +673,41 @@ def test_attention_multi_tile_splits(B, T_q):
     assert C.csa2_device_status() == 0
 
 
+@pytest.mark.parametrize("D,H,K,window,scale_mul,use_ws", [(512, 64, 512, 128, 1.0, True),
+                                                           (512, 64, 100, 128, 64.0, True),
+                                                           (256, 17, 300, 200, 1.0, True),
+                                                           (128, 8, 512, 64, 32.0, False),
+                                                           (512, 64, 0, 128, 1.0, True)])
+def test_attention_many_waves(D, H, K, window, scale_mul, use_ws):
+    """200 query rows: more blocks than SMs, so the launch takes the
+    pipelined form (64-key tiles in two buffers).  Large softmax scales make
+    the reference max move between tiles (the in-TMEM rescale path); K = 100
+    leaves a ragged last tile; no workspace gives one split per row."""
+    B, T_q, n, cap = 50, 4, 900, 1024
+    gm, gs, om, osw, _ = build_pair(B=B, cap=cap, D=D, dI=64, m=1, T=n, pos0=[0] * B, seed=D + K + 3, s_swa=0.5,
+                                    window=window, W_cap=max(window, 128))
+    g = gen(K + 5)
+    q = torch.randn(B, T_q, H, D, generator=g).to(torch.bfloat16)
+    qpos = np.stack([np.arange(n - T_q, n) for _ in range(B)]).astype(np.int32)
+    qpos[1, 2] = 30   # fewer rows than the window
+    if K > 0:
+        idx = torch.stack([torch.stack([I.random_indices(int(qpos[b, j]) + 1, K, g, n_missing=(b + j) % 3)
+                                        for j in range(T_q)]) for b in range(B)])
+        idx_d = idx.cuda()
+    else:
+        idx, idx_d = None, None
+    out = torch.empty(B, T_q, H, D, dtype=torch.bfloat16, device="cuda")
+    ws = C.workspace(C.csa2_attn_workspace_size(B, T_q, H, D, K, window)) if use_ws else None
+    scale = scale_mul / math.sqrt(D)
+    C.csa2_sparse_attn_decode(gm, gs, q.cuda(), torch.from_numpy(qpos).cuda(), idx_d, scale, out, ws=ws)
+    torch.cuda.synchronize()
+    for b, j in [(0, 0), (1, 2), (B // 2, 1), (B - 1, T_q - 1)]:
+        sel = idx[b, j].numpy() if K > 0 else np.zeros(0, np.int32)
+        ref = oracle.attention(om, osw, b, bits(q[b, j]), sel, int(qpos[b, j]), scale)
+        _check_attn(out[b, j], ref)
+    assert C.csa2_device_status() == 0
+
+
 @pytest.mark.parametrize("D,H,B,T_q,window,W_cap,use_ws", [(512, 64, 2, 1, 128, 128, True),
                                                            (512, 64, 8, 1, 128, 128, False),
                                                            (256, 17, 3, 4, 128, 200, True),
