@@ -32,7 +32,7 @@
 //   warps 8-11  first Q (bf16 -> fp16 B operand), then softmax: warp q reads
 //               the S^T lanes of keys 16q .. 16q+15 with the 16x32bx2 TMEM
 //               load, thread = (key, 32-head half); the reference max of a
-//               head moves only when a tile raises it by more than 2^8 (O^T
+//               head moves only when a tile raises it by more than 2^15 (O^T
 //               and L are then rescaled in TMEM, after the previous tile's
 //               O^T MMAs completed), so P = 2^(s - m) stays within fp16
 //               range; P is written as the MN-major B operand [key][head]
@@ -65,7 +65,10 @@ constexpr int kTile = 64;                    // keys per tile (M of S^T)
 constexpr int kPlanTile = 128;               // the split planner's unit (the latency form's tile)
 constexpr int kHeads = 64;                   // heads padded to 64 (N)
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kLazy = 8.0f;                // log2 headroom before the reference max moves
+// log2 headroom before a head's reference max moves: P = 2^(s - m_ref) stays
+// below 2^15 (fp16 holds up to 65,504; L and O^T accumulate in fp32), and each
+// move costs a wait for the previous tile's O^T and a TMEM rescale
+constexpr float kLazy = 15.0f;
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kSmBar = 1;                    // named barrier of the softmax warps
 // TMEM columns: S^T of two tiles [0, 128), O^T blocks [128, 128 + 64 MT), L [384, 448), ones [448, 480)
@@ -387,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       };
       load_logits();
       // after the first tile the reference max usually holds: the per-head
-      // maxima are needed only when a logit exceeds it by more than 2^8
+      // maxima are needed only when a logit exceeds it by more than 2^15
       bool over = first;
       if (!first) {
         const float4 *mp = reinterpret_cast<const float4 *>(S.m_ref + 32 * hh);
