@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
   prep_query_head<DI>(a, blockIdx.x, blockIdx.y * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
 }
 
-template <int DI, bool REINDEX>
+template <int DI, bool REINDEX, bool BMAX>
 __global__ void __launch_bounds__(kThreads, 4) index_kernel(const __grid_constant__ CUtensorMap ik_map,
                                                             const IndexArgs a) {
   constexpr int KS = DI / 32;   // MMA k-steps (32 bytes of E4M3 each)
@@ -276,7 +276,7 @@ __global__ void __launch_bounds__(kThreads, 4) index_kernel(const __grid_constan
       float *out = a.scores + (size_t)row * a.ld;
       if (REINDEX) out[tile * kTileRows + r] = valid ? sum * sk : -INFINITY;
       else if (valid) out[e] = sum * sk;
-      if (!REINDEX && a.bmax) {   // the maximum of each block of 8 entries (8 consecutive lanes)
+      if (BMAX) {   // the maximum of each block of 8 entries (8 consecutive lanes)
         float m = valid ? sum * sk : -INFINITY;
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
         m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
@@ -346,7 +346,7 @@ struct MultiSmem {
   int n_issued, n_mma;
 };
 
-template <int DI, int R>
+template <int DI, int R, bool BMAX>
 __global__ void __launch_bounds__(multi_threads<R>(), 1) index_multi_kernel(const __grid_constant__ CUtensorMap ik_map,
                                                                            const IndexArgs a) {
   constexpr int KS = DI / 32;
@@ -499,7 +499,7 @@ __global__ void __launch_bounds__(multi_threads<R>(), 1) index_multi_kernel(cons
         }
         const float sc = ((s4[0] + s4[1]) + (s4[2] + s4[3])) * sk;
         if (e < nv_mine[k]) a.scores[(size_t)(row0 + my_row + k) * a.ld + e] = sc;
-        if (a.bmax) {   // the maximum of each block of 8 entries (8 consecutive lanes)
+        if (BMAX) {   // the maximum of each block of 8 entries (8 consecutive lanes)
           float m = e < nv_mine[k] ? sc : -INFINITY;
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
           m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
@@ -543,8 +543,8 @@ size_t index_workspace_bytes(int rows, int dI) {
   return q + (size_t)rows * kHeads * 4;
 }
 
-template <int DI, int R>
-static cudaError_t launch_multi(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
+template <int DI, int R, bool BMAX>
+static cudaError_t launch_multi_t(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
   if (!a.prepared) {
     cudaError_t pe = launch_pdl(index_prep_kernel<DI>, dim3(a.B * a.T_q, kHeads / 8), dim3(256), 0, s, dim3(1, 1, 1), a);
     if (pe != cudaSuccess) return pe;
@@ -553,21 +553,29 @@ static cudaError_t launch_multi(const CUtensorMap &map, const IndexArgs &a, cuda
   // second block of the kernel shares the SM (it would wait in tcgen05.alloc)
   size_t smem = sizeof(MultiSmem<DI, R>) + 1024;
   if (R == 4 && smem < 120 * 1024) smem = 120 * 1024;
-  auto k = index_multi_kernel<DI, R>;
+  auto k = index_multi_kernel<DI, R, BMAX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.ctas_per_row, a.B * (a.T_q / R));
   return launch_pdl(k, grid, dim3(multi_threads<R>()), smem, s, dim3(1, 1, 1), map, a);
 }
 
-template <int DI, bool REINDEX>
+// The block-maxima output of the fused selection is a separate instantiation:
+// its few extra instructions in the epilogue loop slowed the prefill scan by
+// 14% when it was a run-time branch.
+template <int DI, int R>
+static cudaError_t launch_multi(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
+  return a.bmax ? launch_multi_t<DI, R, true>(map, a, s) : launch_multi_t<DI, R, false>(map, a, s);
+}
+
+template <int DI, bool REINDEX, bool BMAX>
 static cudaError_t launch_t(const CUtensorMap &map, const IndexArgs &a, cudaStream_t s) {
   if (!a.prepared) {
     cudaError_t pe = launch_pdl(index_prep_kernel<DI>, dim3(a.B * a.T_q, kHeads / 8), dim3(256), 0, s, dim3(1, 1, 1), a);
     if (pe != cudaSuccess) return pe;
   }
   const size_t smem = sizeof(IndexSmem<DI>) + 1024;
-  auto k = index_kernel<DI, REINDEX>;
+  auto k = index_kernel<DI, REINDEX, BMAX>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(a.ctas_per_row, a.B * a.T_q);
@@ -579,8 +587,9 @@ cudaError_t launch_index(const CUtensorMap &map, const IndexArgs &a, bool reinde
   const int R = index_rows_per_block(a.T_q, reindex);
   if (R == 4) return a.dI == 128 ? launch_multi<128, 4>(map, a, s) : launch_multi<64, 4>(map, a, s);
   if (R == 2) return a.dI == 128 ? launch_multi<128, 2>(map, a, s) : launch_multi<64, 2>(map, a, s);
-  if (a.dI == 128) return reindex ? launch_t<128, true>(map, a, s) : launch_t<128, false>(map, a, s);
-  return reindex ? launch_t<64, true>(map, a, s) : launch_t<64, false>(map, a, s);
+  if (reindex) return a.dI == 128 ? launch_t<128, true, false>(map, a, s) : launch_t<64, true, false>(map, a, s);
+  if (a.bmax) return a.dI == 128 ? launch_t<128, false, true>(map, a, s) : launch_t<64, false, true>(map, a, s);
+  return a.dI == 128 ? launch_t<128, false, false>(map, a, s) : launch_t<64, false, false>(map, a, s);
 }
 
 }  // namespace csa2
