@@ -71,6 +71,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 15.0f;
 constexpr uint32_t kWaitLimit = 1u << 22;
 constexpr int kSmBar = 1;                    // named barrier of the softmax warps
+constexpr int kEpiBar = 2;                   // named barrier of the epilogue (gather) warps
 // TMEM columns: S^T of two tiles [0, 128), O^T blocks [128, 128 + 64 MT), L [384, 448), ones [448, 480)
 constexpr uint32_t kColS = 0, kColO = 128, kColL = 384, kColOnes = 448, kTmemCols = 512;
 // Merge items (head, 8 channels) per thread whose loads are in flight together.
@@ -81,7 +82,7 @@ struct AttnSmem {
   alignas(1024) uint8_t kh[2][(D / 64) * kTile * 128];   // two K^ tiles: D/64 chunks of [64 keys x 128 B]
   alignas(1024) uint8_t q[(D / 64) * kHeads * 128];      // Q: D/64 chunks of [64 heads x 128 B]
   alignas(1024) uint8_t p[2][kTile * 128];               // P of two tiles: [64 keys][64 heads] fp16, MN-major
-  float m_ref[kHeads], alpha[kHeads], lsum[kHeads];
+  float m_ref[kHeads], alpha[kHeads], lsum[kHeads], linv[kHeads];
   float red[4][kHeads];
   float wgt[8][kHeads];                                  // merge weights of the splits
   uint64_t chunk_full[2][D / 128];                       // per buffer, per pair of chunks
@@ -591,15 +592,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const AttnArgs a) {
       }
       // window rows entered O^T unscaled: a block that saw window tiles scales its O
       const float osc = c_end > n_fp4_tiles && n_tiles > 0 ? a.s_swa : 1.0f;
+      // every lane holds every head's sum: the quarter-0 warps take one head
+      // per lane, so each head's reciprocal is formed once
+      if (quarter == 0) {
+        float l = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        const float l = __uint_as_float(lv[j]);
-        linv[j] = l > 0.f ? osc / l : 0.f;
+        for (int j = 0; j < 32; ++j) l = j == lane ? __uint_as_float(lv[j]) : l;
+        S.lsum[32 * half + lane] = l;
+        S.linv[32 * half + lane] = l > 0.f ? osc / l : 0.f;
       }
-      if (quarter == 0 && lane == 0) {
+      named_bar(kEpiBar, kDq);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) S.lsum[32 * half + j] = __uint_as_float(lv[j]);
-      }
+      for (int j = 0; j < 32; ++j) linv[j] = S.linv[32 * half + j];
     }
     // O / l per head, staged head-major [64 heads][D] in the K^ tile (free
     // once the last O^T MMA completed) -- bf16 for one split, fp16 partials

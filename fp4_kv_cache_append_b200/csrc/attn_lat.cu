@@ -70,7 +70,7 @@ struct AttnSmem {
   alignas(1024) uint8_t p[kTile * 128];               // P: [128 keys][64 heads] fp16, MN-major
   int key_ent[2][kTile];                              // entry id or window slot, -1 = masked
   float red[4][kHeads];
-  float m_ref[kHeads], l_run[kHeads], alpha[kHeads];
+  float m_ref[kHeads], l_run[kHeads], alpha[kHeads], linv[kHeads];
   float wgt[8][kHeads];                               // merge weights of the splits
   uint64_t sbar, obar;
   uint32_t tmem_base;
@@ -499,12 +499,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
     // the K^ tile (free once the last O^T MMA completed), then written out in
     // 16-byte pieces.  Several splits: fp16 partials straight from registers
     // (a channel per lane; staging measured slower on this latency-bound path).
+    // 1 / l per head, once per head (not per thread)
+    if (tid < kHeads) {
+      const float l = S.l_run[tid];
+      S.linv[tid] = l > 0.f ? 1.f / l : 0.f;
+    }
+    __syncthreads();
     float linv[32];
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const float l = S.l_run[32 * half + j];
-      linv[j] = l > 0.f ? 1.f / l : 0.f;
-    }
+    for (int j = 0; j < 32; ++j) linv[j] = S.linv[32 * half + j];
     uint16_t *ob = reinterpret_cast<uint16_t *>(S.kh);
 #pragma unroll 1
     for (int mt = mt_lo; mt < mt_hi; ++mt) {
