@@ -575,7 +575,8 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
     p.nsplit = 1;
     p.chunks_per_split = 1 << 20;
     p.csplit = 1;
-    p.one_wave = (int64_t)main->B * T_q <= d->sms ? 1 : 0;
+    p.latency_form = ((int64_t)main->B * T_q <= d->sms && K <= 128 && swa->window <= 128 && (K == 0 || swa->window == 0))
+                         ? 1 : 0;   // one 128-key tile per row
   }
   AttnArgs a{};
   a.codes = main->codes; a.scales = main->scales; a.cap = main->cap; a.D = main->D;
@@ -583,7 +584,7 @@ csa2_status csa2_sparse_attn_decode(const csa2_main_cache *main, const csa2_swa_
   a.q = q; a.q_pos = q_pos; a.B = main->B; a.T_q = T_q; a.H = H; a.idx = K > 0 ? idx : nullptr; a.K = K;
   a.scale = softmax_scale; a.out = out;
   a.ws = p.nsplit > 1 ? static_cast<float *>(ws) : nullptr;
-  a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.csplit = p.csplit; a.one_wave = p.one_wave;
+  a.nsplit = p.nsplit; a.chunks_per_split = p.chunks_per_split; a.csplit = p.csplit; a.latency_form = p.latency_form;
   a.status = d->status;
   cudaError_t e = launch_attn(a, reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? CSA2_OK : cuda_fail(e, "attention launch");

@@ -777,11 +777,13 @@ AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms) {
   // small batches: two blocks per split, each issuing the O^T MMAs of, and
   // writing and merging, half of the channels (both compute S and P)
   p.csplit = (nsplit > 1 && D % 256 == 0 && (long long)rows * nsplit * 2 <= sms) ? 2 : 1;
-  // Measured on B200 (dec_full shapes, 1 to 4096 rows): while every block of
-  // the launch is resident at once, the form in which all warps take each
-  // phase of a tile in turn is the faster (by about 2 us up to 128 rows);
-  // from two waves on, the pipelined form below (by 2-8%).
-  p.one_wave = (long long)rows * nsplit * p.csplit <= sms ? 1 : 0;
+  // Measured on B200 (dec_full shapes, 1 to 4,096 rows): the form in which
+  // all warps take each phase of a tile in turn is the faster while every
+  // block of the launch is resident at once and runs a single 128-key tile
+  // (by about 2 us at 8 and 16 rows); once blocks run several tiles, or the
+  // launch takes several waves, the pipelined form below (43 vs 45 us at 128
+  // rows, 251 vs 295 us at 1,024).
+  p.latency_form = ((long long)rows * nsplit * p.csplit <= sms && cps <= 1) ? 1 : 0;
   // fp16 partials [rows][nsplit][64][D] then f32 max and sum [rows][nsplit][64] each
   p.bytes = nsplit > 1 ? (size_t)rows * nsplit * kHeads * ((size_t)D * 2 + 2 * sizeof(float)) : 0;
   return p;
@@ -797,7 +799,7 @@ static cudaError_t launch_attn_t(const AttnArgs &a, cudaStream_t s) {
 }
 
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s) {
-  if (a.one_wave) return launch_attn_lat(a, s);
+  if (a.latency_form) return launch_attn_lat(a, s);
   switch (a.D) {
     case 128: return launch_attn_t<128>(a, s);
     case 256: return launch_attn_t<256>(a, s);

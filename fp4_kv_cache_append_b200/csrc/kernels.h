@@ -201,16 +201,16 @@ struct AttnArgs {
   float *ws;              // split partials (nullptr when unsplit)
   int nsplit, chunks_per_split;
   int csplit;             // 2: a pair of blocks per split, each with half of the O channels
-  int one_wave;           // every block of the launch resident at once: the latency form
+  int latency_form;       // attn_lat.cu: every block resident at once, one 128-key tile per block
   unsigned int *status;
 };
 struct AttnPlan {
   int nsplit, chunks_per_split, csplit;
-  int one_wave;           // rows x nsplit x csplit blocks fit on the SMs (one block per SM)
+  int latency_form;       // rows x nsplit x csplit blocks fit on the SMs and each split is one tile
   size_t bytes;
 };
 AttnPlan plan_attn(int B, int T_q, int H, int D, int K, int window, int sms);
-// Launches the latency form (attn_lat.cu) when a.one_wave, else the pipelined form.
+// Launches the latency form (attn_lat.cu) when a.latency_form, else the pipelined form.
 cudaError_t launch_attn(const AttnArgs &a, cudaStream_t s);
 cudaError_t launch_attn_lat(const AttnArgs &a, cudaStream_t s);
 
