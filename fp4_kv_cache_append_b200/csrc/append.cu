@@ -279,29 +279,48 @@ __global__ void append_kernel(const AppendArgs a) {
   }
 }
 
-// One indexer-key output as one fused multiply-add chain over the channels in
-// ascending order from +0: x^ (binary32, shared) times column `wcol` of the
-// staged W_ik slice (bf16, row stride OPB).  The operands of 32 channels are
-// loaded into registers before their 32 multiply-adds, so the loop runs near
-// the multiply-add latency.
-template <int OPB>
-__device__ __forceinline__ float dec_key_chain_t(const float *xh, const uint16_t *wcol, int D) {
-  float acc = 0.0f;
-#pragma unroll 1
-  for (int c0 = 0; c0 < D; c0 += 32) {
-    float xs[32], ws[32];
+// Operands of channels c0 .. c0+31 of one indexer-key output: x^ (binary32)
+// and the output's row of the transposed W_ik slice (bf16, channels contiguous).
+__device__ __forceinline__ void dec_key_load(const float *xh, const uint16_t *wrow, int c0, float4 (&x)[8],
+                                             uint4 (&w)[4]) {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      xs[j] = xh[c0 + j];
-      ws[j] = bf16_to_f32(wcol[(c0 + j) * OPB]);
+  for (int j = 0; j < 8; ++j) x[j] = reinterpret_cast<const float4 *>(xh + c0)[j];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) w[j] = reinterpret_cast<const uint4 *>(wrow + c0)[j];
+}
+// 32 multiply-adds in ascending channel order; a 32-bit word holds the bf16 of
+// an even channel in its low half and of the next channel in its high half.
+__device__ __forceinline__ float dec_key_chunk(float acc, const float4 (&x)[8], const uint4 (&w)[4]) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t u[4] = {w[j].x, w[j].y, w[j].z, w[j].w};
+    const float v[8] = {x[2 * j].x, x[2 * j].y, x[2 * j].z, x[2 * j].w,
+                        x[2 * j + 1].x, x[2 * j + 1].y, x[2 * j + 1].z, x[2 * j + 1].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      acc = __fmaf_rn(v[2 * k], __uint_as_float(u[k] << 16), acc);
+      acc = __fmaf_rn(v[2 * k + 1], __uint_as_float(u[k] & 0xFFFF0000u), acc);
     }
-#pragma unroll
-    for (int j = 0; j < 32; ++j) acc = __fmaf_rn(xs[j], ws[j], acc);
   }
   return acc;
 }
-__device__ __forceinline__ float dec_key_chain(const float *xh, const uint16_t *wcol, int D, int OPB) {
-  return OPB == 16 ? dec_key_chain_t<16>(xh, wcol, D) : dec_key_chain_t<8>(xh, wcol, D);
+// One indexer-key output as one fused multiply-add chain over the channels in
+// ascending order from +0.  The next 32 channels' operands are loaded while
+// the current 32 multiply-adds run, so the chain runs at the multiply-add
+// latency (D is a multiple of 64).
+__device__ __forceinline__ float dec_key_chain(const float *xh, const uint16_t *wrow, int D) {
+  float acc = 0.0f;
+  float4 xa[8], xb[8];
+  uint4 wa[4], wb[4];
+  dec_key_load(xh, wrow, 0, xa, wa);
+#pragma unroll 1
+  for (int c0 = 0; c0 < D; c0 += 64) {
+    dec_key_load(xh, wrow, c0 + 32, xb, wb);
+    acc = dec_key_chunk(acc, xa, wa);
+    if (c0 + 64 < D) dec_key_load(xh, wrow, c0 + 64, xa, wa);
+    acc = dec_key_chunk(acc, xb, wb);
+  }
+  return acc;
 }
 
 // Decode (one new token per sequence, m = 1): a cluster of 8 blocks per
@@ -312,10 +331,11 @@ __device__ __forceinline__ float dec_key_chain(const float *xh, const uint16_t *
 // blocks push into each other's shared memory before one cluster barrier.
 // Block 0 writes the FP4 codes, the scales, the key scale and n_entries.
 constexpr int kDecCl = 8;
+constexpr int kWT = 512 + 8;   // row stride (bf16) of the transposed W_ik slice: rows on distinct banks
 
 __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_decode_kernel(const AppendArgs a) {
   __shared__ alignas(16) float xh[512];
-  __shared__ alignas(16) uint16_t wsl[512 * 16];   // W_ik[:, c*OPB .. c*OPB+OPB), row-major [D][OPB]
+  __shared__ alignas(16) uint16_t wsl[16 * kWT];   // W_ik[:, c*OPB .. c*OPB+OPB) transposed: [OPB][D (+8)]
   __shared__ float kmx[kDecCl];                    // the blocks' local key maxima
   cg::cluster_group cl = cg::this_cluster();
   const int c = (int)cl.block_rank();
@@ -342,7 +362,6 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
   {
     const int ppr = OPB * 2 / 16;   // 16-byte pieces per W row of the slice
     const uint4 *src = reinterpret_cast<const uint4 *>(a.w_ik);
-    uint4 *dst = reinterpret_cast<uint4 *>(wsl);
     uint4 wv[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -350,9 +369,17 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
       if (i < D * ppr) wv[u] = __ldg(src + ((size_t)(i / ppr) * dI + c * OPB) * 2 / 16 + i % ppr);
     }
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 4; ++u) {   // piece = channel i / ppr, outputs 8 (i % ppr) .. + 7
       const int i = t + u * 256;
-      if (i < D * ppr) dst[i] = wv[u];
+      if (i < D * ppr) {
+        const int ch = i / ppr, o0 = 8 * (i % ppr);
+        const uint32_t w[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          wsl[(o0 + 2 * k) * kWT + ch] = (uint16_t)(w[k] & 0xFFFFu);
+          wsl[(o0 + 2 * k + 1) * kWT + ch] = (uint16_t)(w[k] >> 16);
+        }
+      }
     }
   }
 
@@ -398,7 +425,7 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
   float k = 0.0f;
   if (t < 32) {
     if (t < OPB) {
-      k = dec_key_chain(xh, wsl + t, D, OPB);
+      k = dec_key_chain(xh, wsl + t * kWT, D);
     }
     float m = t < OPB ? fabsf(k) : 0.0f;
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));

@@ -204,8 +204,35 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
     tmem_alloc(&S.tmem_base, kCols);
     tmem_relinquish();
   }
-  pdl_wait();
+  // ---- Q: bf16 -> fp16 into the B-operand layout.  The query and its
+  // position are inputs of the call that no launch of this library writes, so
+  // they are read before the wait for the previous launch (the Top-K that
+  // produces the entry ids).
   const int t = a.q_pos[row];
+  {
+    const uint16_t *qrow = a.q + (size_t)row * a.H * D;
+    uint4 qraw[QI];
+#pragma unroll
+    for (int u = 0; u < QI; ++u) {
+      const int i = tid + u * kThreads;
+      const int h = i / (D / 8), pc = i % (D / 8);
+      qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < QI; ++u) {
+      const int i = tid + u * kThreads;
+      const int h = i / (D / 8), pc = i % (D / 8);
+      const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
+      uint32_t o[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
+        o[k] = *reinterpret_cast<const uint32_t *>(&hv);
+      }
+      *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  pdl_wait();
 
   // ---- keys of this split
   const int n_fp4_tiles = (a.K + kTile - 1) / kTile;
@@ -217,17 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
   int c_end = c_begin + a.chunks_per_split;
   if (c_end > total) c_end = total;
 
-  // ---- Q loads and the first tile's key ids are issued together
-  uint4 qraw[QI];
-  {
-    const uint16_t *qrow = a.q + (size_t)row * a.H * D;
-#pragma unroll
-    for (int u = 0; u < QI; ++u) {
-      const int i = tid + u * kThreads;
-      const int h = i / (D / 8), pc = i % (D / 8);
-      qraw[u] = h < a.H ? __ldg(reinterpret_cast<const uint4 *>(qrow + (size_t)h * D + pc * 8)) : make_uint4(0, 0, 0, 0);
-    }
-  }
+  // ---- the first tile's key ids
   if (c_begin < c_end) load_key_ids<D>(a, row, b, c_begin, n_fp4_tiles, wlo, nwin, S.key_ent[c_begin & 1], tid, false);
   if (tid < kHeads) { S.m_ref[tid] = -INFINITY; S.l_run[tid] = 0.f; S.alpha[tid] = 1.f; }
   tc_fence_before();
@@ -268,22 +285,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_lat_kernel(const AttnArgs a)
         const int id = ids[r];
         raw[u] = id >= 0 ? __ldg(reinterpret_cast<const uint4 *>(a.swa_rows + ((size_t)b * a.W_cap + id) * D) + g)
                          : make_uint4(0, 0, 0, 0);
-      }
-    }
-    // ---- Q: bf16 -> fp16 into the B-operand layout (first tile only)
-    if (c == c_begin) {
-#pragma unroll
-      for (int u = 0; u < QI; ++u) {
-        const int i = tid + u * kThreads;
-        const int h = i / (D / 8), pc = i % (D / 8);
-        const uint32_t w[4] = {qraw[u].x, qraw[u].y, qraw[u].z, qraw[u].w};
-        uint32_t o[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const __half2 hv = __floats2half2_rn(bf16_to_f32(w[k] & 0xFFFFu), bf16_to_f32(w[k] >> 16));
-          o[k] = *reinterpret_cast<const uint32_t *>(&hv);
-        }
-        *reinterpret_cast<uint4 *>(S.q + sw_off(h, pc, kHeads)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
     }
     // the previous tile's O^T MMAs read K^ and P: wait before overwriting

@@ -145,8 +145,11 @@ struct Shared {
   Sel sel[2];
 };
 
-__device__ __forceinline__ void cluster_arrive() {
-  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+// Relaxed: every remote access a thread makes before its final arrive has
+// completed by then (remote reads were consumed, remote writes were released
+// by an earlier cluster barrier), so the arrive needs no release fence.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() {
   asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
@@ -469,7 +472,7 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
       sh.total[s] = ctot;
     }
   }
-  cluster_arrive();   // no remote shared memory is read after this point
+  cluster_arrive_relaxed();   // no remote shared memory is read after this point
   __syncthreads();
 
   // ---- write the chosen columns in order

@@ -531,6 +531,30 @@ def test_topk_exact_on_hard_distributions(kind, n):
     np.testing.assert_array_equal(pool.cpu().numpy(), refp)
 
 
+@pytest.mark.parametrize("kind,n,P", [("normal", 65536, 2048), ("few_values", 40000, 2048), ("normal", 30001, 0)])
+def test_topk_cluster_rows_past_one_wave(kind, n, P):
+    """Rows of at most 65,536 columns go through one 8-block thread-block
+    cluster per row; 160 rows run as several waves of clusters, exact against
+    the oracle with ragged n_valid, absent scores and empty rows."""
+    rows, K = 160, 512
+    rng = np.random.default_rng(zlib.crc32(f"wave/{kind}/{n}".encode()))
+    s = rng.standard_normal((rows, n)).astype(np.float32) if kind == "normal" else _hard_scores(kind, rows, n, rng)
+    s[3, rng.choice(n, n // 10, replace=False)] = -np.inf
+    n_valid = rng.integers(n // 2, n + 1, rows).astype(np.int32)
+    n_valid[5], n_valid[6] = 100, 0
+    out = torch.empty(rows, K, dtype=torch.int32, device="cuda")
+    pool = torch.empty(rows, max(P, 1), dtype=torch.int32, device="cuda")
+    ws = C.workspace(C.csa2_topk_workspace_size(rows, n, K, P))
+    C.csa2_topk(torch.from_numpy(s).cuda(), n, K, out, n_valid=torch.from_numpy(n_valid).cuda(), P_out=P,
+                out_pool=pool if P else None, ws=ws)
+    torch.cuda.synchronize()
+    np.testing.assert_array_equal(out.cpu().numpy(), _ref_topk_rows(s, n_valid, K))
+    if P:
+        refp = np.stack([oracle.block_pool(s[r, :n_valid[r]].astype(np.float64), P) for r in range(rows)])
+        np.testing.assert_array_equal(pool.cpu().numpy(), refp)
+    assert C.csa2_device_status() == 0
+
+
 @pytest.mark.parametrize("kind", ["normal", "outlier", "constant", "huge_range", "two_clusters", "tiny", "few_values"])
 @pytest.mark.parametrize("pad", [3, 0])
 def test_topk_many_long_rows(kind, pad):
