@@ -252,12 +252,14 @@ __device__ void append_window_row(const AppendArgs &a, int b, int r) {
 }
 
 // Blocks beyond the cache work prepare the following scan's indexer query:
-// 8 blocks per query row, warp w of block j handles head 8j + w.
+// 8 blocks per query row, warp w of block j handles head 8j + w.  WAIT: the
+// codes are formed before the wait for the previous launch, stored after it.
+template <bool WAIT>
 __device__ __forceinline__ void prep_block(const AppendArgs &a, int i) {
   const int row = i / 8, h = (i % 8) * 8 + (int)(threadIdx.x >> 5);
   if (row >= a.prep.rows || threadIdx.x >= 256) return;
-  if (a.prep.dI == 128) prep_query_head<128>(a.prep, row, h, threadIdx.x & 31);
-  else prep_query_head<64>(a.prep, row, h, threadIdx.x & 31);
+  if (a.prep.dI == 128) prep_query_head<128, WAIT>(a.prep, row, h, threadIdx.x & 31);
+  else prep_query_head<64, WAIT>(a.prep, row, h, threadIdx.x & 31);
 }
 
 __global__ void append_kernel(const AppendArgs a) {
@@ -267,7 +269,7 @@ __global__ void append_kernel(const AppendArgs a) {
   const int nm = a.B * a.main_blocks_per_seq;
   const int nw = a.B * a.swa_blocks_per_seq;
   if ((int)blockIdx.x >= nm + nw) {
-    prep_block(a, (int)blockIdx.x - nm - nw);
+    prep_block<false>(a, (int)blockIdx.x - nm - nw);
     return;
   }
   if ((int)blockIdx.x < nm) {
@@ -330,6 +332,11 @@ __device__ __forceinline__ float dec_key_chain(const float *xh, const uint16_t *
 // window row; the FP8 key scale needs the maximum over all outputs, which the
 // blocks push into each other's shared memory before one cluster barrier.
 // Block 0 writes the FP4 codes, the scales, the key scale and n_entries.
+// The kernel reads only inputs that no launch of the library writes (the
+// token, its window copy, W_ik, the positions, the indexer query), so all of
+// its arithmetic runs while the previous launch (the previous step's
+// attention, which reads the cache and the window ring) is still running; it
+// waits for that launch only before its first store.
 constexpr int kDecCl = 8;
 constexpr int kWT = 512 + 8;   // row stride (bf16) of the transposed W_ik slice: rows on distinct banks
 
@@ -342,14 +349,16 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
   const int b = blockIdx.y, t = threadIdx.x;
   const int D = a.D, dI = a.dI, OPB = dI / kDecCl;
   pdl_launch_dependents();
-  pdl_wait();
   if (b >= a.B) {   // a cluster of query-preparation blocks (no cluster barrier)
-    prep_block(a, (b - a.B) * kDecCl + c);
+    prep_block<true>(a, (b - a.B) * kDecCl + c);
     return;
   }
   const int p0 = a.pos0[b];
-  if (p0 < 0) {   // the same in every block of the cluster: none of them waits
-    if (t == 0 && c == 0) flag(a.status, CSA2_DEV_BAD_POSITION);
+  if (p0 < 0) {   // the same in every block of the cluster: none of them waits at the cluster barrier
+    if (t == 0 && c == 0) {
+      pdl_wait();
+      flag(a.status, CSA2_DEV_BAD_POSITION);
+    }
     return;
   }
   const int e = p0;   // m = 1: token p0 completes entry p0
@@ -384,6 +393,7 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
   }
 
   // ---- FP4: thread t < D/2 owns channels 2t, 2t+1 (8 threads per 16-channel group)
+  uint32_t code_pair = 0u, scale_byte = 0u;
   if (t < D / 2) {
     const float x0 = bf16_to_f32((uint16_t)(kvp & 0xFFFFu)), x1 = bf16_to_f32((uint16_t)(kvp >> 16));
     float amax = fmaxf(fabsf(x0), fabsf(x1));
@@ -399,24 +409,17 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
     } else {
       sb = 0;
     }
-    if (c == 0) {
-      if (e < a.cap) {
-        const size_t row = (size_t)b * a.cap + e;
-        a.codes[row * (D / 2) + t] = (uint8_t)(c0 | (c1 << 4));
-        if ((t & 7) == 0) a.scales[row * (D / 16) + (t >> 3)] = (uint8_t)sb;
-      } else if (t == 0) {
-        flag(a.status, CSA2_DEV_APPEND_RANGE);
-      }
-    }
+    code_pair = c0 | (c1 << 4);
+    scale_byte = sb;
     xh[2 * t] = __fmul_rn(e2m1_to_f32(c0), sc);
     xh[2 * t + 1] = __fmul_rn(e2m1_to_f32(c1), sc);
   }
   // ---- window: channels [2*wch*c, 2*wch*(c+1)) of the ring slot p0 mod W_cap
+  uint32_t win_pair = 0u;
   if (a.swa_rows && t < wch) {
     const uint32_t lo = f32_to_e4m3(__fdiv_rn(bf16_to_f32((uint16_t)(swp & 0xFFFFu)), a.s_swa));
     const uint32_t hi = f32_to_e4m3(__fdiv_rn(bf16_to_f32((uint16_t)(swp >> 16)), a.s_swa));
-    uint8_t *dst = a.swa_rows + ((size_t)b * a.W_cap + (p0 % a.W_cap)) * D;
-    reinterpret_cast<uint16_t *>(dst)[c * wch + t] = (uint16_t)(lo | (hi << 8));
+    win_pair = lo | (hi << 8);
   }
   __syncthreads();
   // ---- indexer key: thread o < OPB forms output c*OPB + o as one fused
@@ -432,16 +435,35 @@ __global__ void __cluster_dims__(kDecCl, 1, 1) __launch_bounds__(256) append_dec
     if (t < kDecCl) *cl.map_shared_rank(&kmx[c], t) = m;   // push into every block
   }
   cl.sync();
+  float sk = 0.0f;
+  uint32_t kcode = 0u;
   if (t < OPB) {
     float kmax = kmx[0];
 #pragma unroll
     for (int r = 1; r < kDecCl; ++r) kmax = fmaxf(kmax, kmx[r]);
-    const float sk = __fdiv_rn(kmax, 448.0f);
+    sk = __fdiv_rn(kmax, 448.0f);
+    kcode = sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(k, sk));
+  }
+
+  // ---- stores, once the previous launch has finished with the cache
+  pdl_wait();
+  if (c == 0 && t < D / 2) {
     if (e < a.cap) {
       const size_t row = (size_t)b * a.cap + e;
-      a.ik[row * dI + c * OPB + t] = (uint8_t)(sk == 0.0f ? 0u : f32_to_e4m3(__fdiv_rn(k, sk)));
-      if (c == 0 && t == 0) a.ik_scale[row] = sk;
+      a.codes[row * (D / 2) + t] = (uint8_t)code_pair;
+      if ((t & 7) == 0) a.scales[row * (D / 16) + (t >> 3)] = (uint8_t)scale_byte;
+    } else if (t == 0) {
+      flag(a.status, CSA2_DEV_APPEND_RANGE);
     }
+  }
+  if (a.swa_rows && t < wch) {
+    uint8_t *dst = a.swa_rows + ((size_t)b * a.W_cap + (p0 % a.W_cap)) * D;
+    reinterpret_cast<uint16_t *>(dst)[c * wch + t] = (uint16_t)win_pair;
+  }
+  if (t < OPB && e < a.cap) {
+    const size_t row = (size_t)b * a.cap + e;
+    a.ik[row * dI + c * OPB + t] = (uint8_t)kcode;
+    if (c == 0 && t == 0) a.ik_scale[row] = sk;
   }
   if (c == 0 && t == 0) a.n_entries[b] = p0 + 1;
 }

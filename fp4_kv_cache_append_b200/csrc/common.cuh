@@ -346,8 +346,11 @@ __host__ __device__ constexpr uint32_t mma_idesc(int m, int n, uint32_t a_fmt, u
 // One warp prepares head h of query row `row` (see QueryPrep in kernels.h):
 // E4M3 codes of q_h / s_q with s_q = amax(q_h)/448 (binary32 divisions, round
 // to nearest even), written into the 128B (dI = 128) or 64B (dI = 64) swizzled
-// B operand, and w_h * s_q.  Heads >= H_I are zero.
-template <int DI, typename Prep>
+// B operand, and w_h * s_q.  Heads >= H_I are zero.  The query and the head
+// weights are inputs that no launch of the library writes; WAIT makes the warp
+// wait for the previous launch only before its stores (the buffer they go to
+// may still be read by the previous scan).
+template <int DI, bool WAIT, typename Prep>
 __device__ __forceinline__ void prep_query_head(const Prep &p, int row, int h, int lane) {
   constexpr int MASK = DI == 128 ? 7 : 3;
   const uint16_t *qrow = p.q_idx + (size_t)row * p.H_I * DI;
@@ -363,13 +366,14 @@ __device__ __forceinline__ void prep_query_head(const Prep &p, int row, int h, i
     for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   }
   const float sq = __fdiv_rn(amax, 448.0f);
+  uint32_t code[DI / 32];
 #pragma unroll
-  for (int i = 0; i < DI / 32; ++i) {
-    const int c = lane + 32 * i;
-    const uint32_t code = (h < p.H_I && sq != 0.f) ? f32_to_e4m3(__fdiv_rn(v[i], sq)) : 0u;
-    q8[swz<MASK>(h * DI + c)] = (uint8_t)code;
-  }
-  if (lane == 0) p.wq[(size_t)row * 64 + h] = h < p.H_I ? p.w[(size_t)row * p.H_I + h] * sq : 0.f;
+  for (int i = 0; i < DI / 32; ++i) code[i] = (h < p.H_I && sq != 0.f) ? f32_to_e4m3(__fdiv_rn(v[i], sq)) : 0u;
+  const float wq = (lane == 0 && h < p.H_I) ? p.w[(size_t)row * p.H_I + h] * sq : 0.f;
+  if (WAIT) pdl_wait();
+#pragma unroll
+  for (int i = 0; i < DI / 32; ++i) q8[swz<MASK>(h * DI + lane + 32 * i)] = (uint8_t)code[i];
+  if (lane == 0) p.wq[(size_t)row * 64 + h] = wq;
 }
 
 }  // namespace csa2

@@ -102,12 +102,11 @@ __device__ __forceinline__ void head_reduce_reg(float *s4, const float *w, const
 }  // namespace
 
 // Indexer query of each row (prep_query_head): grid (rows, 8) x 256 threads,
-// one warp per head.
+// one warp per head; the codes are formed while the previous launch runs.
 template <int DI>
 __global__ void __launch_bounds__(256) index_prep_kernel(const IndexArgs a) {
   pdl_launch_dependents();
-  pdl_wait();
-  prep_query_head<DI>(a, blockIdx.x, blockIdx.y * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
+  prep_query_head<DI, true>(a, blockIdx.x, blockIdx.y * 8 + (threadIdx.x >> 5), threadIdx.x & 31);
 }
 
 template <int DI, bool REINDEX, bool BMAX>

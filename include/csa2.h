@@ -21,9 +21,11 @@
  *    start while the library's previous kernel on the stream is still
  *    running, and reads what that kernel (or any earlier one) wrote only
  *    after it has completed.  Before that point a kernel reads only inputs
- *    that no kernel of the library writes (the attention query and the query
- *    positions); whatever wrote those must precede the call in stream order,
- *    as it does for any kernel or copy that is not one of the library's.
+ *    that no kernel of the library writes (new tokens and their window
+ *    copies, W_ik, positions, indexer queries and head weights, attention
+ *    queries) and stores nothing; whatever wrote those inputs must precede
+ *    the call in stream order, as it does for any kernel or copy that is not
+ *    one of the library's.
  *  - bf16 tensors are passed as their 16-bit patterns (uint16_t).
  *  - Device pointers must be 16-byte aligned.
  *  - In-kernel anomalies (an index outside the cache, a ring position below
