@@ -310,8 +310,9 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
       const int s = tid / kBins, b = tid % kBins;
       const bool act = sh.sel[s].state == kActive;
       const int h = act ? (int)*cl.map_shared_rank(&sh.hsum[buf][s][b % kSeg], b / kSeg) : 0;
-      const int pre = (int)block_scan<unsigned long long>((unsigned long long)h, sh.red, lane, warp);
-      const int h0 = (int)sh.red[kBins / 32 - 1], tot = (int)sh.red[31];
+      uint32_t *red32 = reinterpret_cast<uint32_t *>(sh.red);   // counts of a row fit 32 bits
+      const int pre = (int)block_scan<uint32_t>((uint32_t)h, red32, lane, warp);
+      const int h0 = (int)red32[kBins / 32 - 1], tot = (int)red32[31];
       const int above = s == 0 ? h0 - pre - h : tot - pre - h;   // keys in higher bins
       const int need = sh.sel[s].need;
       if (act && above < need && above + h >= need) {
@@ -359,35 +360,41 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
 
     // 5. collect the region's keys in block 0 and rank them
 #pragma unroll 1
-    for (int s = 0; s < 2; ++s) {
-      const Sel &l = sh.sel[s];
-      if (l.state != kCollect) continue;
-      const uint32_t lo = l.lo, hi = l.hi;
-      const bool vreg = l.vreg;
-      const int T0 = l.T0;
-      const float v_lo = l.v_lo, inv = l.inv;
+    // both selections in one pass: one warp scan of (entries | blocks << 16),
+    // the two slot reservations in block 0 in flight together
+    {
+      const auto in_region = [&](const Sel &l, uint32_t kk) {
+        return l.state == kCollect && kk &&
+               (l.vreg ? vbin(l.v_lo, l.inv, kk) == l.T0 : (kk >= l.lo && kk <= l.hi));
+      };
+      const Sel &l0 = sh.sel[0], &l1 = sh.sel[1];
       bool in[kN];
-      int m = 0;
+      int m0 = 0;
 #pragma unroll
       for (int k = 0; k < kN; ++k) {
-        const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
-        in[k] = kk && (vreg ? vbin(v_lo, inv, kk) == T0 : (kk >= lo && kk <= hi));
-        m += in[k];
+        in[k] = in_region(l0, key[k]);
+        m0 += in[k];
       }
-      const int incl = warp_incl_scan(m, lane);
-      const int wtot = __shfl_sync(0xffffffffu, incl, 31);
-      uint32_t wbase = 0u;
-      if (lane == 31 && wtot > 0) wbase = atomicAdd(cl.map_shared_rank(&sh.cand_n[s], 0), (uint32_t)wtot);
-      int pos = (int)__shfl_sync(0xffffffffu, wbase, 31) + incl - m;
-      uint2 *dst = cl.map_shared_rank(&sh.cand[s][0], 0);
+      const int m1 = in_region(l1, bkey) ? 1 : 0;
+      const uint32_t mm = (uint32_t)m0 | ((uint32_t)m1 << 16);   // a warp holds at most 256 entries
+      const uint32_t incl = warp_incl_scan(mm, lane);
+      const uint32_t wtot = __shfl_sync(0xffffffffu, incl, 31);
+      uint32_t wb0 = 0u, wb1 = 0u;
+      if (lane == 31) {
+        if (wtot & 0xFFFFu) wb0 = atomicAdd(cl.map_shared_rank(&sh.cand_n[0], 0), wtot & 0xFFFFu);
+        if (wtot >> 16) wb1 = atomicAdd(cl.map_shared_rank(&sh.cand_n[1], 0), wtot >> 16);
+      }
+      int pos = (int)__shfl_sync(0xffffffffu, wb0, 31) + (int)(incl & 0xFFFFu) - m0;
+      const int pos1 = (int)__shfl_sync(0xffffffffu, wb1, 31) + (int)(incl >> 16) - m1;
+      uint2 *dst = cl.map_shared_rank(&sh.cand[0][0], 0);
 #pragma unroll
       for (int k = 0; k < kN; ++k) {
-        const uint32_t kk = s == 0 ? key[k] : (k == 0 ? bkey : 0u);
         if (in[k]) {
-          if (pos < kCand) dst[pos] = make_uint2(kk, (uint32_t)(s == 0 ? c0 + k : blk));
+          if (pos < kCand) dst[pos] = make_uint2(key[k], (uint32_t)(c0 + k));
           ++pos;
         }
       }
+      if (m1 && pos1 < kCand) cl.map_shared_rank(&sh.cand[1][0], 0)[pos1] = make_uint2(bkey, (uint32_t)blk);
     }
     cl.sync();
     {
@@ -402,9 +409,12 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
         const uint2 me = sh.loc[s][i];
         int rank = 0;
 #pragma unroll 1
-        for (int j = 0; j < n; ++j) {
-          const uint2 o = sh.loc[s][j];
-          rank += (o.x > me.x) || (o.x == me.x && o.y < me.y);
+        for (int j = 0; j < n; j += 4) {   // four pairs in flight
+          uint2 o[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) o[u] = sh.loc[s][j + u < n ? j + u : j];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) rank += j + u < n && ((o[u].x > me.x) || (o[u].x == me.x && o[u].y < me.y));
         }
         if (rank == sh.sel[s].need - 1) {   // exactly one pair
           sh.sel[s].kthr = me.x;
@@ -435,19 +445,34 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
     }
     const int t1 = nsel > 1 && bkey && !cm1 && bkey == kthr1;
     const int s1 = nsel > 1 && bkey && (bkey > kthr1 || (cm1 && bkey == kthr1 && blk <= cthr1));
-    const unsigned long long v = (unsigned long long)t0 | ((unsigned long long)s0 << 16) |
-                                 ((unsigned long long)t1 << 32) | ((unsigned long long)s1 << 48);
-    const unsigned long long ex = block_scan<unsigned long long>(v, sh.red, lane, warp);
-    tie_base0 = (int)(ex & 0xFFFFu);
-    tie_base1 = (int)((ex >> 32) & 0xFFFFu);
-    pos0 = (int)((ex >> 16) & 0xFFFFu);   // the output positions when no tie is shared by count
-    pos1 = (int)((ex >> 48) & 0xFFFFu);
-    if (tid == 0) {
-      const unsigned long long tot = sh.red[31];
-      sh.cnt[0] = (int)(tot & 0xFFFFu);
-      sh.cnt[1] = (int)((tot >> 16) & 0xFFFFu);
-      sh.cnt[2] = (int)((tot >> 32) & 0xFFFFu);
-      sh.cnt[3] = (int)((tot >> 48) & 0xFFFFu);
+    if (cm0 && cm1) {   // no ties shared by count (block-uniform): the two strict counts in 32 bits
+      uint32_t *red32 = reinterpret_cast<uint32_t *>(sh.red);
+      const uint32_t ex = block_scan<uint32_t>((uint32_t)s0 | ((uint32_t)s1 << 16), red32, lane, warp);
+      tie_base0 = tie_base1 = 0;
+      pos0 = (int)(ex & 0xFFFFu);
+      pos1 = (int)(ex >> 16);
+      if (tid == 0) {
+        const uint32_t tot = red32[31];
+        sh.cnt[0] = 0;
+        sh.cnt[1] = (int)(tot & 0xFFFFu);
+        sh.cnt[2] = 0;
+        sh.cnt[3] = (int)(tot >> 16);
+      }
+    } else {
+      const unsigned long long v = (unsigned long long)t0 | ((unsigned long long)s0 << 16) |
+                                   ((unsigned long long)t1 << 32) | ((unsigned long long)s1 << 48);
+      const unsigned long long ex = block_scan<unsigned long long>(v, sh.red, lane, warp);
+      tie_base0 = (int)(ex & 0xFFFFu);
+      tie_base1 = (int)((ex >> 32) & 0xFFFFu);
+      pos0 = (int)((ex >> 16) & 0xFFFFu);   // the output positions when no tie is shared by count
+      pos1 = (int)((ex >> 48) & 0xFFFFu);
+      if (tid == 0) {
+        const unsigned long long tot = sh.red[31];
+        sh.cnt[0] = (int)(tot & 0xFFFFu);
+        sh.cnt[1] = (int)((tot >> 16) & 0xFFFFu);
+        sh.cnt[2] = (int)((tot >> 32) & 0xFFFFu);
+        sh.cnt[3] = (int)((tot >> 48) & 0xFFFFu);
+      }
     }
   }
   cl.sync();
