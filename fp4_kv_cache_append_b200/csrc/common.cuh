@@ -168,6 +168,18 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, i
       : "memory");
 }
 
+// L2 prefetch of one box of a 2D tensor map (x 16-byte aligned).  A prefetch
+// only warms L2, the point of coherence, so it may run before the data's
+// producer has finished: a later load still sees the producer's stores.
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap *map, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(x), "r"(y)
+               : "memory");
+}
+// L2 prefetch of a contiguous range (16-byte aligned, size a multiple of 16).
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // 1D bulk copy global -> shared (both 16-byte aligned, size a multiple of 16),
 // completing on `bar`.
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
