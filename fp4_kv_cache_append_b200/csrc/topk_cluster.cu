@@ -358,8 +358,7 @@ __global__ void __cluster_dims__(kCl, 1, 1) __launch_bounds__(kT, 1) topk_cluste
     __syncthreads();
     if (sh.sel[0].state != kCollect && sh.sel[1].state != kCollect) continue;   // cluster-uniform
 
-    // 5. collect the region's keys in block 0 and rank them
-#pragma unroll 1
+    // 5. collect the region's keys in block 0 and rank them;
     // both selections in one pass: one warp scan of (entries | blocks << 16),
     // the two slot reservations in block 0 in flight together
     {
