@@ -666,12 +666,13 @@ def run_e2e(st, n_steps):
     to pinned host memory.  The step's inputs live back to back (16-byte
     aligned) in one pinned host buffer, so a step's H2D transfer is a single
     copy; the API calls read a device copy of it through views.  Steps are
-    pipelined as a serving loop would run them: the calls are captured once
-    into CUDA graphs (per input stage and cache copy) and replayed, two device
-    input stages and two output buffers let the H2D copy of step i+1 (on an
-    upload stream) and the D2H copy of step i (on a download stream) overlap
-    step i's kernels, and the host waits for step i-1's result on the host
-    before it issues step i+1."""
+    pipelined as a serving loop would run them: one CUDA graph per step
+    (captured once per input stage and cache copy, then replayed) holds the
+    step's calls and, on two side branches, the H2D copy of the next step's
+    inputs into the other input stage and the D2H copy of the previous step's
+    output, so both copies overlap the step's kernels and the host issues one
+    launch per step; the host waits for step i-1's graph (and with it step
+    i-2's result on the host) before it issues step i+1."""
     import torch
 
     slots = [("kv_new", None), ("kv_swa_new", 0), ("q", 0), ("q_idx", 0), ("w", 0), ("pos0", None), ("q_pos", None)]
@@ -709,56 +710,53 @@ def run_e2e(st, n_steps):
                 getattr(st, n)[i] = v
         st.out[0] = outs[k]
 
-    comp = torch.cuda.current_stream()
-    up, down = torch.cuda.Stream(), torch.cuda.Stream()
-    ev = lambda: torch.cuda.Event()
-    h2d_done, comp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
     for i in range(3):
         use(i % 2)
         st.run(copy=i % len(st.main))
     torch.cuda.synchronize()
-    # the step's API calls, captured once per (input stage, cache copy) as a
-    # serving loop would, and replayed every step
+    # graph (k, c): step on input stage k and cache copy c, writing outs[k];
+    # side branches: host -> stage 1-k (the next step's inputs) and
+    # outs[1-k] -> out_host[1-k] (the previous step's result)
     ncp = len(st.main)
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
     graphs = [[torch.cuda.CUDAGraph() for _ in range(ncp)] for _ in range(2)]
     for k in range(2):
         use(k)
         for c in range(ncp):
             with torch.cuda.graph(graphs[k][c]):
+                cap = torch.cuda.current_stream()
+                up.wait_stream(cap)
+                with torch.cuda.stream(up):
+                    stages[1 - k].copy_(host_stage, non_blocking=True)
+                down.wait_stream(cap)
+                with torch.cuda.stream(down):
+                    out_host[1 - k].copy_(outs[1 - k], non_blocking=True)
                 st.run(copy=c)
+                cap.wait_stream(up)
+                cap.wait_stream(down)
     torch.cuda.synchronize()
+    comp = torch.cuda.current_stream()
+    done = [torch.cuda.Event(), torch.cuda.Event()]
     t0 = time.perf_counter()
-    with torch.cuda.stream(up):
-        stages[0].copy_(host_stage, non_blocking=True)
-        h2d_done[0].record(up)
+    stages[0].copy_(host_stage, non_blocking=True)   # step 0's inputs
     for i in range(n_steps):
         k = i % 2
-        if i + 1 < n_steps:   # the next step's inputs, once its stage's previous reader (step i-1) finished
-            with torch.cuda.stream(up):
-                if i >= 1:
-                    up.wait_event(comp_done[1 - k])
-                stages[1 - k].copy_(host_stage, non_blocking=True)
-                h2d_done[1 - k].record(up)
-        comp.wait_event(h2d_done[k])
-        if i >= 2:
-            comp.wait_event(d2h_done[k])   # step i-2's output has left this buffer
         graphs[k][i % ncp].replay()
-        comp_done[k].record(comp)
-        with torch.cuda.stream(down):
-            down.wait_event(comp_done[k])
-            out_host[k].copy_(outs[k], non_blocking=True)
-            d2h_done[k].record(down)
+        done[k].record(comp)
         if i >= 1:
-            d2h_done[1 - k].synchronize()   # step i-1's result is on the host
-    d2h_done[(n_steps - 1) % 2].synchronize()
+            done[1 - k].synchronize()   # step i-1's graph ran: step i-2's result is on the host
+    k = (n_steps - 1) % 2
+    out_host[k].copy_(outs[k], non_blocking=True)   # the last step's result
+    comp.synchronize()
     dt = time.perf_counter() - t0
     use(0)
     return {"value": n_steps / dt, "unit": "steps/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "steps": n_steps, "note": "the step's calls through fp4_kv_cache_append_b200.csa2, captured once per "
-                                      "(input stage, cache copy) into CUDA graphs and replayed; per step one packed "
-                                      "H2D copy of the step's inputs from pinned memory and one D2H copy of its "
-                                      "output to pinned memory, pipelined one step deep (copies of neighbouring "
-                                      "steps overlap a step's kernels; the host waits for each result)"}
+            "steps": n_steps, "note": "the step's calls through fp4_kv_cache_append_b200.csa2 in one CUDA graph per "
+                                      "step (captured once per input stage and cache copy, replayed); the graph "
+                                      "also copies the next step's inputs (one packed H2D copy from pinned memory) "
+                                      "and the previous step's output (one D2H copy to pinned memory) on side "
+                                      "branches that overlap the kernels; the host waits for every graph, so each "
+                                      "result reaches the host two steps after its own"}
 
 
 # --------------------------------------------------------------------------- oracle (CPU) legs
