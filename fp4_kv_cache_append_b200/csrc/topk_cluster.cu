@@ -80,8 +80,14 @@ struct Sel {
   int take_eq;
 };
 
+// Value bin of key k: (v - v_lo) * inv rounded to the nearest integer by
+// adding 1.5 * 2^23 (the FP32 adder rounds it into the low mantissa bits: a
+// full-rate add instead of a quarter-rate float-to-int conversion), clamped to
+// [0, kBins).  Explicit roundings keep every call site the same function; the
+// levels rely only on it being monotone in the key.
 __device__ __forceinline__ int vbin(float v_lo, float inv, uint32_t k) {
-  const int b = (int)((kval(k) - v_lo) * inv);
+  const float t = __fmul_rn(__fsub_rn(kval(k), v_lo), inv);   // in [0, kBins] up to rounding
+  const int b = __float_as_int(__fadd_rn(t, 12582912.0f)) - 0x4B400000;
   return b < 0 ? 0 : (b > kBins - 1 ? kBins - 1 : b);
 }
 __device__ __forceinline__ int key_shift(uint32_t lo, uint32_t hi) {
